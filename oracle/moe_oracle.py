@@ -1,0 +1,281 @@
+"""CPU oracle of the single-GPU MoE FFN layer forward, in float64.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path imports, calls or runs this
+module: only the tests, the smoke check of the package entry file and the CPU
+baseline leg of the benchmark do.  It shares no code with the CUDA library.
+
+It is the plain definition of the layer, written so that each step can be checked
+against the pages by eye:
+
+  * router logits z = x @ W_r^T                    ("MoE" chapter index, §0 data-path
+                                                    diagram; routing primer §三)
+  * scores s = softmax(z_t) or sigmoid(z)          (routing primer §三)
+  * selection score c = s + bias, bias used only   ("MoE" §0: "+bias, only for
+    for choosing                                    selection"; §2.2 aux-free bias)
+  * grouped top-k: group score, keep the best      (routing primer §六, §七, §九, §十)
+    groups, mask the rest, then top-K
+  * weights from the unbiased s, renormalised      (routing primer §四)
+    over the K chosen, then times routed_scale
+  * token-expert pairs bucketed by expert          (routing primer §5.1)
+  * per-expert SwiGLU FFN                          (routing primer §一, §5.2)
+      W_down (SiLU(W_gate x) * W_up x)
+  * weighted combine y_t = sum_k w_tk y_tk         (routing primer §5.3)
+    plus the always-active shared expert           ("MoE" §0 diagram, §2.1)
+
+Readings where the pages are silent (each also listed in the design notes):
+  - W_r is stored [E, H] (logits x @ W_r^T).
+  - The group stage ranks groups by the biased selection score c; the group score is
+    the sum of the `group_topn` largest c in the group (1 = the group maximum used in
+    the routing primer's §七 example).
+  - Order and ties: experts (and groups) are taken in descending score; an exact tie
+    goes to the lower index.
+  - Pairs p = t*K + k are bucketed stably: inside an expert, rows follow p.
+  - Each expert's rows start at a multiple of `block_m`; pad rows carry no pair.
+  - Renormalise first, then multiply by routed_scale; the shared expert is added with
+    weight 1.
+  - FP8 workload: e4m3 (max 448, round to nearest even, saturating); one
+    power-of-two scale per 1x128 activation block and per 128x128 weight block;
+    the SwiGLU output h is re-quantised per row and 128 columns before the down
+    projection ("SwiGLU / FP8 Cast" stage of the Mega MoE pipeline on the MoE
+    optimisation blog, §5.1).
+  - No residual is added; the layer returns routed + shared only.
+
+Parity status: routed_scale and group_topn = 2 are not fixed by any worked example on
+the pages; they are pinned only by self-consistency (weights sum to routed_scale;
+group_topn and routed_scale reduce to the printed examples when set to 1).
+"""
+from __future__ import annotations
+
+
+import numpy as np
+
+FP8_MAX = 448.0
+QBLOCK = 128
+
+
+# ----------------------------------------------------------------------------------
+# e4m3 (OCP FP8, "fn" variant: no infinities, 0x7F/0xFF are NaN, max 448)
+# ----------------------------------------------------------------------------------
+def decode_e4m3(codes) -> np.ndarray:
+    """Value of each e4m3 byte: sign bit 7, 4 exponent bits (bias 7), 3 mantissa
+    bits; exponent field 0 is subnormal (m/8 * 2^-6); S.1111.111 is NaN."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    normal = (1.0 + m / 8.0) * np.power(2.0, e - 7.0)
+    sub = (m / 8.0) * 2.0 ** -6
+    v = sign * np.where(e == 0, sub, normal)
+    return np.where((c & 0x7F) == 0x7F, np.nan, v)
+
+
+def _e4m3_positive_grid():
+    codes = np.arange(0x7F, dtype=np.uint8)        # 0x00 .. 0x7E: all finite, >= 0
+    return codes, decode_e4m3(codes)
+
+
+def quantize_e4m3(v) -> np.ndarray:
+    """Nearest e4m3 value to each element (ties to the even code, i.e. the one whose
+    mantissa LSB is 0), saturating at +-448.  Returned as float64 values."""
+    v = np.asarray(v, dtype=np.float64)
+    codes, grid = _e4m3_positive_grid()
+    a = np.minimum(np.abs(v), FP8_MAX)
+    hi = np.clip(np.searchsorted(grid, a, side="left"), 0, len(grid) - 1)
+    lo = np.clip(hi - 1, 0, len(grid) - 1)
+    d_lo = a - grid[lo]
+    d_hi = grid[hi] - a
+    take_hi = (d_hi < d_lo) | ((d_hi == d_lo) & ((codes[hi] & 1) == 0))
+    q = np.where(take_hi, grid[hi], grid[lo])
+    return np.copysign(q, v)
+
+
+def pow2_scale(amax) -> np.ndarray:
+    """2^ceil(log2(amax / 448)) taken exactly from the binary exponent; 1 where
+    amax == 0."""
+    amax = np.asarray(amax, dtype=np.float64)
+    mant, expo = np.frexp(np.where(amax > 0, amax, FP8_MAX) / FP8_MAX)   # mant in [0.5, 1)
+    e = np.where(mant == 0.5, expo - 1, expo)
+    return np.where(amax > 0, np.ldexp(1.0, e), 1.0)
+
+
+def dequant_blocks(codes, scales, rows_per_block: int) -> np.ndarray:
+    """codes [R, C] e4m3 with scales [R/rows_per_block, C/128] -> float64 [R, C]."""
+    v = decode_e4m3(codes)
+    s = np.repeat(np.repeat(np.asarray(scales, np.float64), rows_per_block, axis=0), QBLOCK, axis=1)
+    return v * s
+
+
+def quantize_rows_1x128(h) -> np.ndarray:
+    """Re-quantise an activation matrix [R, C] to e4m3 with one power-of-two scale per
+    row and 128 columns; returns the dequantised float64 values."""
+    h = np.asarray(h, np.float64)
+    R, C = h.shape
+    b = h.reshape(R, C // QBLOCK, QBLOCK)
+    s = pow2_scale(np.abs(b).max(axis=2))
+    return (quantize_e4m3(b / s[:, :, None]) * s[:, :, None]).reshape(R, C)
+
+
+# ----------------------------------------------------------------------------------
+# Router, scores, selection
+# ----------------------------------------------------------------------------------
+def router_logits(x, w_r) -> np.ndarray:
+    """z[t, e] = sum_h x[t, h] * W_r[e, h]  (x @ W_r^T)."""
+    return np.asarray(x, np.float64) @ np.asarray(w_r, np.float64).T
+
+
+def scores(z, score_fn: int) -> np.ndarray:
+    """score_fn 0: softmax over the experts of each token; 1: sigmoid per expert."""
+    z = np.asarray(z, np.float64)
+    if score_fn == 0:
+        ez = np.exp(z - z.max(axis=1, keepdims=True))
+        return ez / ez.sum(axis=1, keepdims=True)
+    return 1.0 / (1.0 + np.exp(-z))
+
+
+def _desc_order(v) -> np.ndarray:
+    """Indices by descending value; equal values keep ascending index order."""
+    return np.argsort(-np.asarray(v, np.float64), kind="stable")
+
+
+def select_experts(c_row, K: int, n_group: int = 1, topk_group: int = 1, group_topn: int = 1):
+    """Top-K experts of one token by selection score c_row [E], descending.
+
+    With n_group > 1 the E experts form n_group consecutive groups; a group's score is
+    the sum of its `group_topn` largest c; only the `topk_group` best groups stay
+    candidates and the others are masked before the final top-K."""
+    c = np.asarray(c_row, np.float64).copy()
+    E = c.shape[0]
+    if n_group > 1:
+        gs = E // n_group
+        groups = c.reshape(n_group, gs)
+        gscore = np.array([np.sort(groups[j])[::-1][:group_topn].sum() for j in range(n_group)])
+        keep = _desc_order(gscore)[:topk_group]
+        allowed = np.zeros(E, dtype=bool)
+        for j in keep:
+            allowed[j * gs:(j + 1) * gs] = True
+        c = np.where(allowed, c, -np.inf)
+    return _desc_order(c)[:K]
+
+
+def route_from_scores(s, K: int, bias=None, n_group: int = 1, topk_group: int = 1,
+                      group_topn: int = 1, renormalize: bool = True, routed_scale: float = 1.0):
+    """Routing decision from scores s [T, E]: ids [T, K] int32, weights [T, K] float64."""
+    s = np.asarray(s, np.float64)
+    T, E = s.shape
+    c = s + (np.asarray(bias, np.float64)[None, :] if bias is not None else 0.0)
+    ids = np.empty((T, K), dtype=np.int32)
+    w = np.empty((T, K), dtype=np.float64)
+    for t in range(T):
+        sel = select_experts(c[t], K, n_group, topk_group, group_topn)
+        ids[t] = sel
+        wt = s[t, sel]
+        if renormalize:
+            wt = wt / wt.sum()
+        w[t] = wt * routed_scale
+    return ids, w
+
+
+def route(x, w_r, bias, wl):
+    """Full routing of workload `wl` (any object with K, score_fn, n_group, topk_group,
+    group_topn, renormalize, routed_scale).  Returns ids, weights, scores."""
+    s = scores(router_logits(x, w_r), wl.score_fn)
+    ids, w = route_from_scores(s, wl.K, bias, wl.n_group, wl.topk_group, wl.group_topn,
+                               bool(wl.renormalize), wl.routed_scale)
+    return ids, w, s
+
+
+# ----------------------------------------------------------------------------------
+# Dispatch: pairs bucketed by expert
+# ----------------------------------------------------------------------------------
+def permute(ids, E: int, block_m: int):
+    """Bucket the P = T*K pairs p = t*K + k by expert, stably in p.
+
+    Returns counts [E], offsets_padded [E+1] (expert e's rows start at
+    offsets_padded[e], a multiple of block_m), row_of_pair [P] and pair_of_row
+    [offsets_padded[E]] (-1 on pad rows)."""
+    flat = np.asarray(ids, np.int64).reshape(-1)
+    P = flat.shape[0]
+    counts = np.zeros(E, dtype=np.int64)
+    for e in flat:
+        counts[e] += 1
+    padded = ((counts + block_m - 1) // block_m) * block_m
+    offsets = np.zeros(E + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(padded)
+    row_of_pair = np.empty(P, dtype=np.int64)
+    pair_of_row = np.full(int(offsets[E]), -1, dtype=np.int64)
+    fill = offsets[:E].copy()
+    for p in range(P):
+        e = flat[p]
+        row_of_pair[p] = fill[e]
+        pair_of_row[fill[e]] = p
+        fill[e] += 1
+    return (counts.astype(np.int32), offsets.astype(np.int32),
+            row_of_pair.astype(np.int32), pair_of_row.astype(np.int32))
+
+
+# ----------------------------------------------------------------------------------
+# Expert FFN and combine
+# ----------------------------------------------------------------------------------
+def silu(g):
+    return g / (1.0 + np.exp(-g))
+
+
+def swiglu_ffn(xr, wg, wu, wd, quantize_h: bool = False):
+    """W_down (SiLU(W_gate x) * W_up x) for each row of xr [n, H]; weights [out, in]."""
+    xr = np.asarray(xr, np.float64)
+    g = xr @ np.asarray(wg, np.float64).T
+    u = xr @ np.asarray(wu, np.float64).T
+    h = silu(g) * u
+    if quantize_h:
+        h = quantize_rows_1x128(h)
+    return h @ np.asarray(wd, np.float64).T
+
+
+def expert_outputs(x, ids, expert_weights, E: int, block_m: int, quantize_h: bool = False):
+    """y_perm [P_pad, H]: the output of every pair's expert on its token, laid out in
+    the bucketed row order of `permute` (pad rows are zero).  `expert_weights(e)`
+    returns (W_gate[e], W_up[e], W_down[e]) as arrays [I,H], [I,H], [H,I]."""
+    x = np.asarray(x, np.float64)
+    K = ids.shape[1]
+    counts, offsets, row_of_pair, pair_of_row = permute(ids, E, block_m)
+    y = np.zeros((int(offsets[E]), x.shape[1]), dtype=np.float64)
+    for e in range(E):
+        n = int(counts[e])
+        if n == 0:
+            continue
+        rows = np.arange(offsets[e], offsets[e] + n)
+        toks = pair_of_row[rows] // K
+        wg, wu, wd = expert_weights(e)
+        y[rows] = swiglu_ffn(x[toks], wg, wu, wd, quantize_h)
+    return y, row_of_pair
+
+
+def combine(y_perm, row_of_pair, w, y_shared=None) -> np.ndarray:
+    """out[t] = sum_k w[t, k] * y_perm[row_of_pair[t*K + k]]  (+ y_shared[t])."""
+    w = np.asarray(w, np.float64)
+    T, K = w.shape
+    y_perm = np.asarray(y_perm, np.float64)
+    out = np.zeros((T, y_perm.shape[1]), dtype=np.float64)
+    for t in range(T):
+        for k in range(K):
+            out[t] += w[t, k] * y_perm[row_of_pair[t * K + k]]
+    if y_shared is not None:
+        out += np.asarray(y_shared, np.float64)
+    return out
+
+
+def forward_given_routing(x, ids, w, expert_weights, E: int, shared=None,
+                          quantize_h: bool = False, block_m: int = 1):
+    """Layer output [T, H] for a given routing decision (ids, w).  `shared` is
+    (W_gate, W_up, W_down) of the shared expert or None."""
+    y_perm, row_of_pair = expert_outputs(x, ids, expert_weights, E, block_m, quantize_h)
+    y_sh = swiglu_ffn(x, *shared) if shared is not None else None
+    return combine(y_perm, row_of_pair, w, y_sh)
+
+
+def layer_forward(x, w_r, bias, expert_weights, wl, shared=None):
+    """Route, then run the chosen experts and combine.  Returns (out, ids, w, s)."""
+    ids, w, s = route(x, w_r, bias, wl)
+    out = forward_given_routing(x, ids, w, expert_weights, wl.E, shared,
+                                quantize_h=(wl.dtype == 1))
+    return out, ids, w, s

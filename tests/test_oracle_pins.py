@@ -1,0 +1,330 @@
+"""Pins of the fp64 oracle against what the pages and the mathematics fix.
+
+None of these tests needs a GPU.  Each pin checks the oracle against something other
+than itself: the worked examples printed in "MoE 路由入门：从 Dense FFN 到 GroupedTopK"
+(fixtures under tests/golden/), library routines that compute the same textbook
+quantity (scipy softmax/expit, torch.topk, torch's SwiGLU pieces, torch's e4m3 cast),
+closed-form invariants, and brute force over tiny inputs.
+"""
+import itertools
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+import torch.nn.functional as F
+
+from oracle import moe_oracle as o
+from tests.conftest import load_golden
+
+
+# ------------------------------------------------------------------ worked examples
+def test_top2_worked_example_raw_and_renormalised():
+    g = load_golden("top2_worked_example.txt")
+    s = np.array(g["scores"])
+    ids, w = o.route_from_scores(s, g["K"], renormalize=False)
+    assert ids.tolist() == g["topk_ids"]
+    np.testing.assert_allclose(w, g["topk_weights"], rtol=0, atol=1e-15)
+    ids2, w2 = o.route_from_scores(s, g["K"], renormalize=True)
+    assert ids2.tolist() == g["topk_ids"]
+    np.testing.assert_allclose(w2[0], g["renormalized_token0"], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(w2.sum(axis=1), 1.0, rtol=0, atol=1e-15)
+
+
+def test_top2_worked_example_through_softmax():
+    # Each row of the printed scores sums to 1, so logits z = log(s) reproduce them
+    # exactly through the softmax router.
+    g = load_golden("top2_worked_example.txt")
+    s = np.array(g["scores"])
+    z = np.log(s)
+    s2 = o.scores(z, 0)
+    np.testing.assert_allclose(s2, s, rtol=1e-14, atol=0)
+    ids, w = o.route_from_scores(s2, g["K"], renormalize=False)
+    assert ids.tolist() == g["topk_ids"]
+    np.testing.assert_allclose(w, g["topk_weights"], rtol=1e-14)
+
+
+def test_bucket_example():
+    g = load_golden("bucket_example.txt")
+    ids = np.array([[e for (t, e) in g["pairs"][i * g["K"]:(i + 1) * g["K"]]] for i in range(g["T"])])
+    counts, offs, row_of_pair, pair_of_row = o.permute(ids, g["E"], 1)
+    assert counts.tolist() == g["counts"]
+    assert ids.size == g["P"] == g["T"] * g["K"]
+    for e in range(g["E"]):
+        rows = range(offs[e], offs[e] + counts[e])
+        assert [int(pair_of_row[r]) // g["K"] for r in rows] == g["buckets"][e]
+
+
+@pytest.mark.parametrize("group_topn", [1, 2])
+def test_grouped_topk_example(group_topn):
+    g = load_golden("grouped_topk_example.txt")
+    c = np.array(g["scores"])
+    kw = dict(n_group=g["n_group"], topk_group=g["topk_group"], group_topn=group_topn)
+    assert o.select_experts(c, 3).tolist() == g["plain_top3"]
+    assert o.select_experts(c, 3, **kw).tolist() == g["grouped_top3"]
+    assert o.select_experts(c, 4).tolist() == g["plain_top4"]
+    assert o.select_experts(c, 4, **kw).tolist() == g["grouped_top4"]
+
+
+def test_grouped_topk_example_group_scores():
+    # With group_topn = 1 the group score is the group maximum the page prints, and the
+    # kept groups are the two best of those.
+    g = load_golden("grouped_topk_example.txt")
+    c = np.array(g["scores"]).reshape(g["n_group"], -1)
+    np.testing.assert_allclose(c.max(axis=1), g["group_scores"])
+    # the oracle masks exactly the groups outside kept_groups: ask for all survivors
+    n_keep = g["topk_group"] * c.shape[1]
+    sel = o.select_experts(c.ravel(), n_keep, n_group=g["n_group"], topk_group=g["topk_group"])
+    assert sorted({int(e) // c.shape[1] for e in sel}) == sorted(g["kept_groups"])
+
+
+# ------------------------------------------------------------------ library routines
+def test_scores_match_scipy():
+    rng = np.random.default_rng(1)
+    z = rng.normal(size=(17, 33)) * 3
+    np.testing.assert_allclose(o.scores(z, 0), scipy.special.softmax(z, axis=1), rtol=1e-13)
+    np.testing.assert_allclose(o.scores(z, 1), scipy.special.expit(z), rtol=1e-13)
+
+
+def test_router_logits_orientation():
+    # z = x @ W_r^T with W_r stored [E, H]: logit (t, e) is the dot product of token t
+    # with row e, checked element by element.
+    rng = np.random.default_rng(2)
+    x, w_r = rng.normal(size=(3, 5)), rng.normal(size=(4, 5))
+    z = o.router_logits(x, w_r)
+    assert z.shape == (3, 4)
+    for t in range(3):
+        for e in range(4):
+            assert z[t, e] == pytest.approx(sum(x[t, h] * w_r[e, h] for h in range(5)), rel=1e-13)
+
+
+@pytest.mark.parametrize("K", [1, 2, 8])
+def test_plain_topk_matches_torch_topk(K):
+    rng = np.random.default_rng(K)
+    s = rng.random((50, 64))
+    ids, w = o.route_from_scores(s, K, renormalize=False)
+    tv, ti = torch.topk(torch.from_numpy(s), K, dim=1, sorted=True)
+    assert (ids == ti.numpy()).all()
+    np.testing.assert_array_equal(w, tv.numpy())
+
+
+def test_sigmoid_plain_topk_is_topk_of_logits():
+    # no bias, one group: top-k of sigmoid scores = top-k of the logits (monotone)
+    rng = np.random.default_rng(3)
+    z = rng.normal(size=(40, 32))
+    ids, _ = o.route_from_scores(o.scores(z, 1), 4, renormalize=True)
+    assert (ids == torch.topk(torch.from_numpy(z), 4, dim=1).indices.numpy()).all()
+
+
+def test_ties_go_to_lower_index():
+    s = np.array([[0.25, 0.25, 0.25, 0.25], [0.1, 0.3, 0.3, 0.3]])
+    ids, _ = o.route_from_scores(s, 2)
+    assert ids.tolist() == [[0, 1], [1, 2]]
+    c = np.array([0.5, 0.5, 0.5, 0.5, 0.9, 0.1, 0.1, 0.1])
+    # groups of 2: scores [0.5, 0.5, 0.9, 0.1] -> groups 2 then 0 (tie 0/1 -> 0)
+    assert o.select_experts(c, 3, n_group=4, topk_group=2).tolist() == [4, 0, 1]
+
+
+# ------------------------------------------------------------------ brute force
+def _bruteforce_grouped(c, K, n_group, topk_group, group_topn):
+    E = len(c)
+    gs = E // n_group
+    gscore = [max(sum(comb) for comb in itertools.combinations(c[j * gs:(j + 1) * gs], group_topn))
+              for j in range(n_group)]
+    best_groups = max(itertools.combinations(range(n_group), topk_group),
+                      key=lambda gsub: sum(gscore[j] for j in gsub))
+    allowed = [e for e in range(E) if e // gs in best_groups]
+    best = max(itertools.combinations(allowed, K), key=lambda sub: sum(c[e] for e in sub))
+    return set(best)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_grouped_topk_bruteforce(seed):
+    rng = np.random.default_rng(100 + seed)
+    E, n_group, topk_group, K, topn = 16, 4, 2, 3, 2
+    c = rng.random(E)
+    sel = o.select_experts(c, K, n_group, topk_group, topn)
+    assert set(sel.tolist()) == _bruteforce_grouped(c, K, n_group, topk_group, topn)
+    assert all(c[sel[i]] >= c[sel[i + 1]] for i in range(K - 1))
+
+
+def test_bias_only_chooses_and_scale_applies_after_renorm():
+    s = np.array([[0.5, 0.3, 0.2]])
+    bias = np.array([0.0, 0.0, 0.5])
+    ids, w = o.route_from_scores(s, 1, bias=bias, renormalize=False)
+    assert ids.tolist() == [[2]] and w[0, 0] == pytest.approx(0.2)
+    ids, w = o.route_from_scores(s, 2, bias=bias, renormalize=True, routed_scale=2.5)
+    assert ids.tolist() == [[2, 0]]
+    np.testing.assert_allclose(w[0], [2.5 * 0.2 / 0.7, 2.5 * 0.5 / 0.7], rtol=1e-14)
+
+
+def test_weights_sum_to_routed_scale():
+    rng = np.random.default_rng(4)
+    s = scipy.special.expit(rng.normal(size=(30, 64)))
+    bias = rng.normal(size=64) * 0.1
+    _, w = o.route_from_scores(s, 8, bias, 8, 4, 2, True, 2.5)
+    np.testing.assert_allclose(w.sum(axis=1), 2.5, rtol=1e-14)
+
+
+def test_grouped_reduces_to_plain_when_one_group():
+    rng = np.random.default_rng(5)
+    s = rng.random((20, 32))
+    a, _ = o.route_from_scores(s, 4, n_group=1)
+    b, _ = o.route_from_scores(s, 4, n_group=4, topk_group=4, group_topn=2)
+    assert (a == b).all()
+
+
+# ------------------------------------------------------------------ permutation
+@pytest.mark.parametrize("block_m", [1, 4, 128])
+def test_permute_invariants_and_bruteforce(block_m):
+    rng = np.random.default_rng(block_m)
+    T, K, E = 37, 3, 9
+    ids = np.stack([rng.choice(E, size=K, replace=False) for _ in range(T)])
+    counts, offs, rop, por = o.permute(ids, E, block_m)
+    assert counts.sum() == T * K
+    assert (counts == np.bincount(ids.ravel(), minlength=E)).all()
+    assert (offs % block_m == 0).all() and offs[0] == 0
+    assert (np.diff(offs) >= counts).all() and (np.diff(offs) < counts + block_m).all()
+    flat = ids.ravel()
+    for p in range(T * K):
+        e = flat[p]
+        assert rop[p] == offs[e] + sum(1 for q in range(p) if flat[q] == e)
+        assert por[rop[p]] == p
+    assert (por == -1).sum() == offs[E] - T * K
+
+
+# ------------------------------------------------------------------ FFN and combine
+def _torch_swiglu(x, wg, wu, wd):
+    x, wg, wu, wd = (torch.from_numpy(np.asarray(a, np.float64)) for a in (x, wg, wu, wd))
+    return F.linear(F.silu(F.linear(x, wg)) * F.linear(x, wu), wd).numpy()
+
+
+def test_single_expert_layer_is_dense_swiglu():
+    # E = 1, K = 1, renormalised: every token goes to the one expert with weight 1, so
+    # the layer is the dense SwiGLU FFN (computed here with torch's linear and silu).
+    rng = np.random.default_rng(6)
+    T, H, I = 11, 16, 24
+    x = rng.normal(size=(T, H))
+    wg, wu, wd = rng.normal(size=(I, H)) * .2, rng.normal(size=(I, H)) * .2, rng.normal(size=(H, I)) * .2
+    ids = np.zeros((T, 1), dtype=np.int32)
+    w = np.ones((T, 1))
+    out = o.forward_given_routing(x, ids, w, lambda e: (wg, wu, wd), 1, block_m=4)
+    np.testing.assert_allclose(out, _torch_swiglu(x, wg, wu, wd), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(o.swiglu_ffn(x, wg, wu, wd), _torch_swiglu(x, wg, wu, wd), rtol=1e-12)
+
+
+def test_combine_of_identity_experts_returns_x():
+    rng = np.random.default_rng(7)
+    T, H, E, K = 13, 8, 5, 3
+    x = rng.normal(size=(T, H))
+    s = scipy.special.softmax(rng.normal(size=(T, E)), axis=1)
+    ids, w = o.route_from_scores(s, K, renormalize=True)
+    counts, offs, rop, por = o.permute(ids, E, 4)
+    y_perm = np.zeros((offs[E], H))
+    real = por >= 0
+    y_perm[real] = x[por[real] // K]          # identity expert: y = x
+    np.testing.assert_allclose(o.combine(y_perm, rop, w), x, rtol=1e-13, atol=1e-14)
+
+
+def _loop_swiglu(xt, wg, wu, wd):
+    I, H = wg.shape
+    h = []
+    for i in range(I):
+        g = sum(wg[i, j] * xt[j] for j in range(H))
+        u = sum(wu[i, j] * xt[j] for j in range(H))
+        h.append(g / (1 + np.exp(-g)) * u)
+    return np.array([sum(wd[j, i] * h[i] for i in range(I)) for j in range(H)])
+
+
+@pytest.mark.parametrize("case", ["softmax_plain", "sigmoid_grouped_bias_shared"])
+def test_layer_equals_dense_mixture_masked_to_topk(case):
+    # Dense all-experts mixture (every expert run on every token, routing page §二),
+    # masked to the chosen top-K with their renormalised weights, in plain Python
+    # loops; must equal the oracle's sparse dispatch -> grouped FFN -> combine path.
+    rng = np.random.default_rng(8)
+    T, H, I, E, K = 6, 8, 6, 8, 2
+    x = rng.normal(size=(T, H))
+    w_r = rng.normal(size=(E, H)) * 0.5
+    Wg, Wu = rng.normal(size=(E, I, H)) * .3, rng.normal(size=(E, I, H)) * .3
+    Wd = rng.normal(size=(E, H, I)) * .3
+    from types import SimpleNamespace as NS
+    if case == "softmax_plain":
+        wl = NS(E=E, K=K, score_fn=0, n_group=1, topk_group=1, group_topn=1, renormalize=True,
+                routed_scale=1.0, dtype=0)
+        bias, shared = None, None
+    else:
+        wl = NS(E=E, K=K, score_fn=1, n_group=4, topk_group=2, group_topn=2, renormalize=True,
+                routed_scale=2.5, dtype=0)
+        bias = rng.normal(size=E) * 0.1
+        shared = (rng.normal(size=(4, H)) * .3, rng.normal(size=(4, H)) * .3, rng.normal(size=(H, 4)) * .3)
+    out, ids, w, s = o.layer_forward(x, w_r, bias, lambda e: (Wg[e], Wu[e], Wd[e]), wl, shared)
+    for t in range(T):
+        dense = np.zeros(H)
+        for e in range(E):
+            p = 0.0
+            if e in ids[t]:
+                k = list(ids[t]).index(e)
+                p = w[t, k]
+            dense += p * _loop_swiglu(x[t], Wg[e], Wu[e], Wd[e])
+        if shared is not None:
+            dense += _loop_swiglu(x[t], *shared)
+        np.testing.assert_allclose(out[t], dense, rtol=1e-10, atol=1e-12)
+
+
+# ------------------------------------------------------------------ e4m3
+def test_e4m3_decode_table_matches_torch_and_spot_values():
+    codes = np.arange(256, dtype=np.uint8)
+    mine = o.decode_e4m3(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    nan = np.isnan(ref)
+    assert (np.isnan(mine) == nan).all() and nan.sum() == 2
+    np.testing.assert_array_equal(mine[~nan], ref[~nan])
+    assert mine[0x7E] == 448.0 and mine[0x01] == 2.0 ** -9 and mine[0x08] == 2.0 ** -6
+    assert mine[0x38] == 1.0 and mine[0xB8] == -1.0 and mine[0x07] == 7 * 2.0 ** -9
+
+
+def test_e4m3_quantize_is_nearest_even_by_search():
+    grid_codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+    grid = o.decode_e4m3(grid_codes)
+    rng = np.random.default_rng(9)
+    pos = np.sort(np.unique(np.abs(grid)))
+    mids = (pos[1:] + pos[:-1]) / 2
+    v = np.concatenate([rng.normal(size=2000) * 50, mids, -mids, [0.0, 448.0, 470, 1e6, -1e6, 2.0 ** -11]])
+    q = o.quantize_e4m3(v)
+    for vi, qi in zip(v, q):
+        if abs(vi) >= 448:
+            assert qi == np.copysign(448.0, vi)
+            continue
+        d = np.abs(grid - vi)
+        cand = grid_codes[d == d.min()]
+        cand_vals = o.decode_e4m3(cand)
+        if len(set(cand_vals.tolist())) > 1:   # a true midpoint: pick the even code
+            cand = cand[(cand & 1) == 0]
+        assert qi == o.decode_e4m3(cand[:1])[0] or (qi == 0 and vi == 0)
+    inr = np.abs(v) < 448
+    tq = torch.from_numpy(v[inr]).to(torch.float32).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal(np.abs(q[inr]), np.abs(tq))
+
+
+def test_pow2_scale_definition():
+    rng = np.random.default_rng(10)
+    amax = np.concatenate([rng.random(500) * 10.0 ** rng.integers(-6, 6, 500), [448.0, 896.0, 224.0, 0.0]])
+    s = o.pow2_scale(amax)
+    for a, si in zip(amax, s):
+        if a == 0:
+            assert si == 1.0
+            continue
+        assert np.log2(si) == np.round(np.log2(si))
+        assert a / si <= 448.0 < a / (si / 2)
+
+
+def test_rowwise_requant_error_bound():
+    rng = np.random.default_rng(11)
+    h = rng.normal(size=(5, 256)) * np.exp(rng.normal(size=(5, 1)))
+    q = o.quantize_rows_1x128(h)
+    b = h.reshape(5, 2, 128)
+    s = o.pow2_scale(np.abs(b).max(axis=2))[:, :, None]
+    err = np.abs(q.reshape(5, 2, 128) - b)
+    # half a unit in the last place of e4m3 (3 mantissa bits), or of the subnormal step
+    bound = np.maximum(np.abs(b) * 2.0 ** -4, s * 2.0 ** -10)
+    assert (err <= bound + 1e-300).all()
