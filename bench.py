@@ -1,0 +1,369 @@
+"""Benchmark of the MoE FFN layer forward on B200 (one JSON line on stdout).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one moe_layer_forward over the whole workload (route, permute, gate/up GEMM
+with SwiGLU, down GEMM, shared expert if any, combine) with inputs resident in HBM.
+L2 is flushed (a 512 MiB write) before every timed step, outside the timed events.
+With N > 1 (torchrun, one process per GPU) every rank runs an independent replica of
+the layer on its own inputs (the layer has no cross-GPU exchange on one node's data
+path): the reported value is all ranks' tokens over the slowest rank's time.
+
+`value` is tokens/s; the line also carries the grouped-GEMM TFLOP/s, an end-to-end
+number through moe_layer_forward_host (host activations copied in and the output
+copied back inside the timed region), the roofline of the dominant kernel from CUDA
+events recorded around its launches, the SM clocks sampled during the timed region,
+and the fp64 CPU oracle timed on a bounded sample of the same workload.
+`--impl reference` times that oracle alone, per step, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mixture_experts_ffn_08_b200 import binding as B  # noqa: E402
+from mixture_experts_ffn_08_b200 import inputs, workloads as W  # noqa: E402
+
+METRIC = "MoE layer tokens/s and grouped-GEMM TFLOP/s (or HBM GB/s) vs B200 roofline"
+FLUSH_BYTES = 512 << 20
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d["bf16_tflops"], d["hbm_gbs"], "measured"
+    return 1590.0, 6650.0, "fallback"
+
+
+def _describe(wl):
+    s = (f"T={wl.T} H={wl.H} I={wl.I} E={wl.E} K={wl.K} "
+         f"{'softmax' if wl.score_fn == 0 else 'sigmoid'}")
+    if wl.n_group > 1:
+        s += f" groups={wl.n_group}/keep{wl.topk_group}/top{wl.group_topn}"
+    if wl.has_bias:
+        s += " bias"
+    s += f" renorm x{wl.routed_scale:g}" if wl.renormalize else f" x{wl.routed_scale:g}"
+    if wl.I_shared:
+        s += f" +shared I={wl.I_shared}"
+    return s + (" fp8" if wl.dtype else " bf16")
+
+
+def _dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.proc = None
+        self.uuid = str(torch.cuda.get_device_properties(device).uuid)
+        if not self.uuid.startswith("GPU-"):
+            self.uuid = "GPU-" + self.uuid
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.uuid, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.3)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8]
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip() == "Active"})
+        loaded = [v for v in sm if smax and v > 0.5 * max(smax)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ CPU oracle leg
+def _oracle_sample(wl, d, n_tokens, seed=0):
+    """Oracle forward (route + experts + combine) of a seeded token sample; returns
+    (tokens, seconds, threads)."""
+    from oracle import moe_oracle as o
+    from threadpoolctl import threadpool_info
+    rng = np.random.default_rng(seed)
+    toks = np.sort(rng.choice(wl.T, size=min(n_tokens, wl.T), replace=False))
+    idx = torch.as_tensor(toks, device=d["w_r"].device)
+    # host copies of the inputs are not part of the timed oracle work
+    if wl.dtype == W.DTYPE_FP8:
+        xq, xs = d["x_q"][idx].cpu().numpy(), d["x_scale"][idx].cpu().numpy()
+        x_of = lambda: o.dequant_blocks(xq, xs, 1)  # noqa: E731
+    else:
+        xh = d["x"][idx].cpu().to(torch.float64).numpy()
+        x_of = lambda: xh  # noqa: E731
+    w_r = d["w_r"].cpu().to(torch.float64).numpy()
+    bias = d["bias"].cpu().to(torch.float64).numpy() if d["bias"] is not None else None
+    host_w = {}
+
+    def fetch(e):
+        if e not in host_w:
+            if wl.dtype == W.DTYPE_FP8:
+                host_w[e] = tuple((d[n + "_q"][e].cpu().numpy(), d[n + "_s"][e].cpu().numpy())
+                                  for n in ("w_gate", "w_up", "w_down"))
+            else:
+                host_w[e] = tuple(d[n][e].cpu() for n in ("w_gate", "w_up", "w_down"))
+        return host_w[e]
+
+    # routing decides which experts the sample needs; fetch them before the clock starts
+    x0 = x_of()
+    ids0, _, _ = o.route(x0, w_r, bias, wl)
+    for e in np.unique(ids0):
+        fetch(int(e))
+    shared = None
+    if wl.I_shared:
+        sh = [d[n].cpu() for n in ("ws_gate", "ws_up", "ws_down")]
+
+    def expert_weights(e):
+        if wl.dtype == W.DTYPE_FP8:
+            return tuple(o.dequant_blocks(q, s, 128) for q, s in fetch(e))
+        return tuple(t.to(torch.float64).numpy() for t in fetch(e))
+
+    t0 = time.perf_counter()
+    x = x_of()
+    if wl.I_shared:
+        shared = tuple(t.to(torch.float64).numpy() for t in sh)
+    o.layer_forward(x, w_r, bias, expert_weights, wl, shared)
+    dt = time.perf_counter() - t0
+    threads = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    return len(toks), dt, threads
+
+
+def _cpu_sample_tokens(wl):
+    # about 10-30 s of fp64 work on a few host cores
+    per_token_flops = 6 * wl.K * wl.H * wl.I + 6 * wl.H * wl.I_shared
+    return int(max(4, min(wl.T, 2.0e11 / max(per_token_flops, 1) / 4)))
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args):
+    world, rank, local = _dist()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    wl = W.ALL[args.workload]
+    p = B.params(wl)
+    d = inputs.make_inputs(wl, seed=rank, device="cuda")
+    fp8 = wl.dtype == W.DTYPE_FP8
+    a = dict(x=d["x_q"] if fp8 else d["x"], x_scale=d.get("x_scale"))
+    wts = [d["w_gate_q"] if fp8 else d["w_gate"], d["w_up_q"] if fp8 else d["w_up"],
+           d["w_down_q"] if fp8 else d["w_down"], d.get("w_gate_s"), d.get("w_up_s"), d.get("w_down_s"),
+           d.get("ws_gate"), d.get("ws_up"), d.get("ws_down")]
+    ws_bytes = B.moe_workspace_size_host(p)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    out = torch.empty((wl.T, wl.H), dtype=torch.bfloat16, device="cuda")
+    ids = torch.empty((wl.T, wl.K), dtype=torch.int32, device="cuda")
+    wgt = torch.empty((wl.T, wl.K), dtype=torch.float32, device="cuda")
+    counts = torch.empty((wl.E,), dtype=torch.int32, device="cuda")
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    B.check(B.moe_clear_device_status(ws))
+
+    def step():
+        B.check(B.moe_layer_forward(p, a["x"], a["x_scale"], d["w_r"], d["bias"], *wts, out, ids, wgt,
+                                    counts, ws, ws_bytes), "moe_layer_forward")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    # ---------------- timed region: device-resident inputs
+    clocks = ClockSampler(local) if rank == 0 else None
+    if clocks:
+        clocks.start()
+    dominant = B.K_GATEUP
+    B.check(B.moe_trace_enable(1 << dominant, 4 * args.steps))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    barrier()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    barrier()
+    step_ms = [s.elapsed_time(e) for s, e in ev]
+    traced = B.moe_trace_collect()
+    B.moe_trace_disable()
+    clk = clocks.stop() if clocks else None
+    status = B.moe_get_device_status(ws)
+    if status != 0:
+        raise B.MoEError(f"device status {status:#x} after the timed steps")
+
+    counts_h = counts.cpu().numpy()
+    P = wl.T * wl.K
+    ms_total = float(sum(step_ms))
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms_total], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    tokens_per_s = wl.T * world / (ms_step / 1e3)
+
+    # algorithmic work (unpadded rows)
+    flops_gateup = 4.0 * P * wl.H * wl.I
+    flops_down = 2.0 * P * wl.I * wl.H
+    flops_shared = 6.0 * wl.T * wl.H * wl.I_shared
+    gemm_flops = flops_gateup + flops_down + flops_shared
+    bf16_peak, hbm_peak, peak_kind = _peaks()
+    dom_ms = [ms for k, ms in traced if k == dominant]
+    dom_avg = statistics.mean(dom_ms) if dom_ms else None
+    achieved = flops_gateup / (dom_avg / 1e3) / 1e12 if dom_avg else None
+    roofline = {"kernel": "gateup_swiglu (grouped GEMM, fused SwiGLU)", "bound": "tensor",
+                "achieved": achieved, "peak": bf16_peak, "unit": "TFLOP/s",
+                "frac": achieved / bf16_peak if achieved else None, "traffic": None,
+                "peak_kind": f"{peak_kind} bf16 burst", "launches_timed": len(dom_ms),
+                "avg_ms": dom_avg, "algorithmic_flops_per_launch": flops_gateup}
+
+    # ---------------- end to end: host activations in, host output out
+    x_host = (d["x_q"] if fp8 else d["x"]).cpu().pin_memory()
+    out_host = torch.empty((wl.T, wl.H), dtype=torch.bfloat16).pin_memory()
+    e2e_ms = None
+    if not fp8:
+        def e2e_step():
+            B.check(B.moe_layer_forward_host(p, x_host, None, d["w_r"], d["bias"], *wts, out_host, ws,
+                                             ws_bytes), "moe_layer_forward_host")
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        barrier()
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            ev2[i][0].record(stream)
+            e2e_step()
+            ev2[i][1].record(stream)
+        barrier()
+        e2e_ms = sum(s.elapsed_time(e) for s, e in ev2)
+        if world > 1:
+            import torch.distributed as dist
+            t = torch.tensor([e2e_ms], device="cuda", dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e_ms /= args.steps
+    xbytes = wl.T * wl.H * (1 if fp8 else 2)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n, dt, threads = _oracle_sample(wl, d, _cpu_sample_tokens(wl))
+        cpu = {"value": n / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "sample": f"{n} seeded tokens of {wl.name} through the fp64 oracle "
+                         f"(route, experts, combine); {dt:.1f} s"}
+
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp8" if fp8 else "bf16",
+        "data": "synthetic (seeded Gaussian activations and random-init weights)",
+        "config": {"workload": f"{wl.name}: {_describe(wl)}", "global_batch": wl.T * world,
+                   "seq_len": 1, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "flushed before every timed step (512 MiB write, outside the events)"},
+        "grouped_gemm_tflops": gemm_flops / (ms_step / 1e3) / 1e12 * world,
+        "e2e": {"value": wl.T * world / (e2e_ms / 1e3) if e2e_ms else None, "unit": "tokens/s",
+                "h2d_bytes_per_step": xbytes, "d2h_bytes_per_step": wl.T * wl.H * 2},
+        "roofline": roofline,
+        "clocks": clk,
+        "gpu_launches": B.moe_layer_launch_count(p) * args.steps,
+        "cpu_baseline": cpu,
+        "expert_load": {"max": int(counts_h.max()), "min": int(counts_h.min()),
+                        "mean": P / wl.E},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args):
+    world, rank, _ = _dist()
+    if rank != 0:
+        return
+    wl = W.ALL[args.workload]
+    d = inputs.make_inputs(wl, seed=0, device="cpu" if not torch.cuda.is_available() else "cuda")
+    n = max(2, _cpu_sample_tokens(wl) // 8)
+    times, toks, threads = [], 0, 1
+    for i in range(args.warmup + args.steps):
+        k, dt, threads = _oracle_sample(wl, d, n, seed=i)
+        if i >= args.warmup:
+            times.append(dt)
+            toks += k
+    value = toks / sum(times)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded Gaussian activations and random-init weights)",
+        "config": {"workload": f"{wl.name}: {_describe(wl)}", "global_batch": wl.T, "seq_len": 1,
+                   "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{n} seeded tokens per step through the fp64 oracle"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="mixtral_prefill", choices=sorted(W.ALL))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

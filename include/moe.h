@@ -1,0 +1,227 @@
+/*
+ * moe.h — C ABI of the B200 (sm_100a) MoE FFN layer forward.
+ *
+ * The layer (one GPU, forward only), as the pages define it:
+ *   router logits  z = x @ W_r^T                       "MoE" chapter index (llm-infra-atlas),
+ *                                                      §0 data-path diagram; routing primer §三
+ *   scores         s = softmax(z_t) | sigmoid(z)       "MoE 路由入门：从 Dense FFN 到 GroupedTopK" §三
+ *   selection      top-K of c = s + bias (bias only    "MoE" §0 ("+bias, only for selection"), §2.2;
+ *                  chooses), optionally group-limited  routing primer §六, §七, §九, §十
+ *   weights        s of the chosen experts, renormal-  routing primer §四
+ *                  ised, times routed_scale
+ *   dispatch       P = T*K pairs bucketed by expert    routing primer §5.1
+ *   expert FFN     W_down (SiLU(W_gate x) * W_up x)    routing primer §一, §5.2; MoE optimisation
+ *                                                      blog ("MoE 优化的探索…") §1
+ *   combine        out_t = sum_k w_tk y_tk (+ shared)  routing primer §5.3; "MoE" §0
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller, row-major, unless a
+ *     function says HOST.  The library never allocates device memory: scratch comes from
+ *     the caller's workspace `ws` of at least moe_workspace_size() bytes, 256-byte aligned.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*; NULL is the
+ *     legacy default stream) and does no host synchronisation, except where stated.
+ *   - Argument errors are returned synchronously as a moe_status_t and nothing is
+ *     launched.  Errors found by a kernel (an expert id out of range, a pipeline wait that
+ *     timed out) are OR-ed into a status word inside `ws`; read it with
+ *     moe_get_device_status().  No kernel traps.
+ *   - Base pointers of bf16 / e4m3 matrices must be 16-byte aligned; H and I must be
+ *     multiples of 128.
+ *   - Weight layout is [out_features, in_features] (nn.Linear): W_r [E,H];
+ *     W_gate, W_up [E,I,H]; W_down [E,H,I]; shared expert Ws_gate, Ws_up [I_shared,H],
+ *     Ws_down [H,I_shared].
+ *   - dtype MOE_DTYPE_BF16: x, weights, outputs bf16; fp32 accumulation.
+ *     dtype MOE_DTYPE_FP8_E4M3: x is e4m3 [T,H] with fp32 power-of-two scales
+ *     x_scale [T,H/128] (one per token and 128 channels); expert weights are e4m3 with
+ *     fp32 scales per 128x128 block ([E,I/128,H/128] for gate/up, [E,H/128,I/128] for
+ *     down); W_r stays bf16; the output is bf16.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_ABI_VERSION 1
+
+typedef enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned pointer, small workspace */
+  MOE_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. H not a multiple of 128)   */
+  MOE_ERR_CUDA = 3,         /* a CUDA runtime call failed (launch, attribute, copy)        */
+  MOE_ERR_TIMEOUT = 4,      /* device: a bounded pipeline wait gave up                     */
+  MOE_ERR_DEVICE = 5        /* device: bad input found by a kernel (expert id out of range) */
+} moe_status_t;
+
+/* Bits of the device status word (moe_get_device_status). */
+#define MOE_DEV_BAD_EXPERT_ID 0x1   /* a topk id outside [0,E): the pair was skipped      */
+#define MOE_DEV_TIMEOUT 0x2         /* a GEMM pipeline wait exceeded its limit and exited */
+
+enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 };
+enum { MOE_DTYPE_BF16 = 0, MOE_DTYPE_FP8_E4M3 = 1 };
+
+typedef struct moe_params {
+  int32_t T;            /* tokens                                                        */
+  int32_t H;            /* hidden size (multiple of 128)                                 */
+  int32_t I;            /* intermediate size of a routed expert (multiple of 128)        */
+  int32_t E;            /* routed experts, 1..1024                                       */
+  int32_t K;            /* experts per token, 1..min(E,32)                               */
+  int32_t n_group;      /* expert groups for group-limited top-k (1 = plain top-k)       */
+  int32_t topk_group;   /* groups kept                                                   */
+  int32_t group_topn;   /* group score = sum of the group_topn largest selection scores  */
+  int32_t score_fn;     /* MOE_SCORE_SOFTMAX or MOE_SCORE_SIGMOID                        */
+  int32_t renormalize;  /* 1: divide the chosen weights by their sum                     */
+  float routed_scale;   /* factor applied to the (renormalised) weights                  */
+  int32_t I_shared;     /* intermediate size of the shared expert, 0 = none              */
+  int32_t dtype;        /* MOE_DTYPE_BF16 or MOE_DTYPE_FP8_E4M3                          */
+  int32_t block_m;      /* row alignment of each expert's bucket; 0 = default (128).     */
+                        /* Only 128 is accepted by this build.                           */
+} moe_params_t;
+
+/* ---------------------------------------------------------------------------------- */
+/* Sizes                                                                               */
+/* ---------------------------------------------------------------------------------- */
+
+/* Bytes of workspace a moe_layer_forward() call needs (the per-stage calls need at most
+ * this much).  0 if the parameters are invalid. */
+size_t moe_workspace_size(const moe_params_t* p);
+
+/* Bytes of workspace moe_layer_forward_host() needs: moe_workspace_size() plus device
+ * staging for the copied activations and output.  0 if the parameters are invalid. */
+size_t moe_workspace_size_host(const moe_params_t* p);
+
+/* Upper bound on the padded row count P + E*(block_m-1): the row capacity that
+ * pair_of_row, x_perm and y_perm must have.  -1 if the parameters are invalid. */
+int64_t moe_max_padded_rows(const moe_params_t* p);
+
+/* ---------------------------------------------------------------------------------- */
+/* Stage 1 — routing.  Routing primer §三 (router, scores), §四 (top-k, renormalise),   */
+/* §六-§十 (group-limited top-k); "MoE" §0 (selection-only bias).                      */
+/*   x        [T,H] bf16, or e4m3 codes with x_scale [T,H/128] (FP8 dtype)              */
+/*   w_r      [E,H] bf16;  bias [E] fp32 or NULL                                        */
+/*   topk_ids [T,K] int32 out: experts in descending selection score (ties: lower id)   */
+/*   topk_w   [T,K] fp32 out: weights from the unbiased scores                          */
+/* Uses ws for the logits (and, for FP8, a bf16 copy of x).                            */
+/* ---------------------------------------------------------------------------------- */
+moe_status_t moe_route(const moe_params_t* p, const void* x, const float* x_scale,
+                       const void* w_r, const float* bias, int32_t* topk_ids, float* topk_w,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------- */
+/* Stage 2 — dispatch (routing primer §5.1).  Buckets the pairs p = t*K + k by expert,  */
+/* stably in p, each bucket starting at a multiple of block_m.                          */
+/*   topk_ids       [T,K] int32 in                                                      */
+/*   counts         [E] int32 out: pairs per expert                                     */
+/*   offsets_padded [E+1] int32 out: first row of each bucket; offsets_padded[E] = rows */
+/*   row_of_pair    [T*K] int32 out                                                     */
+/*   pair_of_row    [moe_max_padded_rows] int32 out: pair of each row, -1 on pad rows   */
+/*   x_perm         [moe_max_padded_rows, H] out: x[t] copied to each pair's row, pad   */
+/*                  rows zero (bf16, or e4m3 codes + x_perm_scale [rows, H/128] fp32)   */
+/* An id outside [0,E) sets MOE_DEV_BAD_EXPERT_ID and that pair is left out.            */
+/* ---------------------------------------------------------------------------------- */
+moe_status_t moe_permute(const moe_params_t* p, const int32_t* topk_ids, const void* x,
+                         const float* x_scale, int32_t* counts, int32_t* offsets_padded,
+                         int32_t* row_of_pair, int32_t* pair_of_row, void* x_perm,
+                         float* x_perm_scale, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------- */
+/* Stage 3 — expert FFN on the bucketed rows (routing primer §5.2; M-grouped GEMM as    */
+/* in the "MoE" chapter index §1, grouped GEMM entry).                                  */
+/*   y_perm[r] = W_down[e] (SiLU(W_gate[e] x_perm[r]) * W_up[e] x_perm[r])              */
+/* for every row r of expert e's bucket (pad rows included; their result is unused).    */
+/*   offsets_padded [E+1], counts [E] as written by moe_permute (read on the device     */
+/*                  only); counts may be NULL, then pad rows are computed and stored too */
+/*   y_perm [moe_max_padded_rows, H] fp32 out; rows past counts[e] in a bucket are not   */
+/*                  written when counts is given                                        */
+/* The SwiGLU intermediate h (bf16) lives in ws.  y_perm stays fp32 because it feeds    */
+/* the output directly: the final bf16 rounding already uses most of the error budget. */
+/* ---------------------------------------------------------------------------------- */
+moe_status_t moe_expert_ffn(const moe_params_t* p, const void* x_perm, const float* x_perm_scale,
+                            const int32_t* offsets_padded, const int32_t* counts,
+                            const void* w_gate, const void* w_up, const void* w_down,
+                            const float* w_gate_scale, const float* w_up_scale,
+                            const float* w_down_scale, float* y_perm, void* ws, size_t ws_bytes,
+                            void* stream);
+
+/* Dense SwiGLU FFN of the always-active shared expert on all T tokens ("MoE" §0, §2.1):
+ *   y_shared [T,H] fp32 = Ws_down (SiLU(Ws_gate x) * Ws_up x).   bf16 dtype only. */
+moe_status_t moe_shared_expert_ffn(const moe_params_t* p, const void* x, const void* ws_gate,
+                                   const void* ws_up, const void* ws_down, float* y_shared,
+                                   void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------- */
+/* Stage 4 — combine (routing primer §5.3): out[t] = sum_k w[t,k] y_perm[row_of_pair[   */
+/* t*K+k]] (+ y_shared[t]), fp32 accumulation in fixed k order, one rounding to bf16.   */
+/* y_perm [rows,H] and y_shared [T,H] (may be NULL) are fp32; out [T,H] bf16.  Pairs    */
+/* with row_of_pair = -1 are left out.  No atomics: bitwise reproducible.               */
+/* ---------------------------------------------------------------------------------- */
+moe_status_t moe_combine(const moe_params_t* p, const float* y_perm, const int32_t* row_of_pair,
+                         const float* topk_w, const float* y_shared, void* out, void* stream);
+
+/* ---------------------------------------------------------------------------------- */
+/* The whole layer: route -> permute -> expert FFN -> [shared expert] -> combine, all   */
+/* on `stream`, with no host synchronisation.  out [T,H] bf16.                          */
+/* topk_ids_out [T,K], topk_w_out [T,K], counts_out [E] are optional copies of the      */
+/* routing decision (NULL: kept in ws only).  ws_gate/ws_up/ws_down are the shared      */
+/* expert's weights (required iff I_shared > 0).                                        */
+/* ---------------------------------------------------------------------------------- */
+moe_status_t moe_layer_forward(const moe_params_t* p, const void* x, const float* x_scale,
+                               const void* w_r, const float* bias, const void* w_gate,
+                               const void* w_up, const void* w_down, const float* w_gate_scale,
+                               const float* w_up_scale, const float* w_down_scale,
+                               const void* ws_gate, const void* ws_up, const void* ws_down,
+                               void* out, int32_t* topk_ids_out, float* topk_w_out,
+                               int32_t* counts_out, void* ws, size_t ws_bytes, void* stream);
+
+/* Same layer with HOST activations: x_host (and x_scale_host for FP8) are copied to the
+ * device inside the call and the result is copied back to out_host, all enqueued on
+ * `stream`.  Weights stay device pointers.  Host buffers should be pinned; they must
+ * stay valid until the stream has passed this call (cudaStreamSynchronize). */
+moe_status_t moe_layer_forward_host(const moe_params_t* p, const void* x_host,
+                                    const float* x_scale_host, const void* w_r,
+                                    const float* bias, const void* w_gate, const void* w_up,
+                                    const void* w_down, const float* w_gate_scale,
+                                    const float* w_up_scale, const float* w_down_scale,
+                                    const void* ws_gate, const void* ws_up,
+                                    const void* ws_down, void* out_host, void* ws,
+                                    size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------- */
+/* Status, tracing                                                                      */
+/* ---------------------------------------------------------------------------------- */
+
+/* Synchronises `stream`, copies the device status word of `ws` into *host_status. */
+moe_status_t moe_get_device_status(const void* ws, void* stream, int32_t* host_status);
+/* Clears the device status word of `ws` (asynchronous on `stream`). */
+moe_status_t moe_clear_device_status(void* ws, void* stream);
+
+const char* moe_status_string(moe_status_t s);
+int32_t moe_abi_version(void);
+
+/* Kernel ids for tracing. */
+enum {
+  MOE_K_ROUTER_GEMM = 0, MOE_K_TOPK = 1, MOE_K_PERM_COUNT = 2, MOE_K_PERM_SCAN = 3,
+  MOE_K_PERM_RANK = 4, MOE_K_PERM_GATHER = 5, MOE_K_GATEUP = 6, MOE_K_DOWN = 7,
+  MOE_K_SHARED_GATEUP = 8, MOE_K_SHARED_DOWN = 9, MOE_K_COMBINE = 10, MOE_K_DEQUANT_X = 11,
+  MOE_K_COUNT = 12
+};
+
+/* Tracing: while enabled, every launch of a kernel whose bit (1u << id) is in
+ * kernel_mask is bracketed by two CUDA events on its stream (at most `capacity` launches
+ * are kept).  moe_trace_collect() synchronises on the recorded events, writes each
+ * launch's kernel id and duration in milliseconds, returns the number written and
+ * clears the record.  Process-wide, not thread-safe. */
+moe_status_t moe_trace_enable(uint32_t kernel_mask, int32_t capacity);
+moe_status_t moe_trace_disable(void);
+int32_t moe_trace_collect(int32_t* kernel_ids, float* ms, int32_t max_out);
+
+/* Number of kernels the library launches for one moe_layer_forward with these params. */
+int32_t moe_layer_launch_count(const moe_params_t* p);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

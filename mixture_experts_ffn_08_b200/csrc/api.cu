@@ -1,0 +1,440 @@
+// C ABI of the MoE layer forward (declared in include/moe.h): argument validation,
+// workspace layout, stage orchestration on one stream, device status word and tracing.
+#include <cuda_runtime.h>
+
+#include <mutex>
+#include <vector>
+
+#include "../../include/moe.h"
+#include "internal.h"
+
+namespace moe {
+
+// ------------------------------------------------------------------ device properties
+int num_sms() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+// ------------------------------------------------------------------ tracing
+namespace {
+struct Trace {
+  bool on = false;
+  uint32_t mask = 0;
+  int cap = 0;
+  int n = 0;
+  bool open = false;
+  std::vector<cudaEvent_t> ev;
+  std::vector<int> kid;
+};
+Trace g_trace;
+}  // namespace
+
+void trace_before(int kid, cudaStream_t st) {
+  Trace& t = g_trace;
+  t.open = false;
+  if (!t.on || !((t.mask >> kid) & 1u) || t.n >= t.cap) return;
+  if (cudaEventRecord(t.ev[2 * t.n], st) == cudaSuccess) t.open = true;
+}
+
+void trace_after(int kid, cudaStream_t st) {
+  Trace& t = g_trace;
+  if (!t.open) return;
+  t.open = false;
+  if (cudaEventRecord(t.ev[2 * t.n + 1], st) == cudaSuccess) {
+    t.kid[t.n] = kid;
+    ++t.n;
+  }
+}
+
+// ------------------------------------------------------------------ workspace layout
+namespace {
+
+constexpr size_t kAlign = 256;
+size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+struct Layout {
+  size_t status, logits, xb, ids, w, counts, offsets, row_of_pair, pair_of_row, chunk_counts;
+  size_t x_perm, x_perm_scale, h, y_perm, h_sh, y_sh, total;
+  size_t x_stage, x_scale_stage, out_stage, total_host;
+  long long max_rows;
+};
+
+bool is_fp8(const moe_params_t* p) { return p->dtype == MOE_DTYPE_FP8_E4M3; }
+
+Layout layout(const moe_params_t* p) {
+  Layout L{};
+  const long long T = p->T, H = p->H, I = p->I, E = p->E, K = p->K;
+  const long long P = T * K;
+  const long long rows = P + E * (kBlockM - 1);
+  const long long nchunks = (P + kPermChunk - 1) / kPermChunk;
+  const size_t xelem = is_fp8(p) ? 1 : 2;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t at = o; o += up(bytes); return at; };
+  L.max_rows = rows;
+  L.status = take(256);
+  L.logits = take(T * E * 4);
+  L.xb = take(is_fp8(p) ? T * H * 2 : 0);
+  L.ids = take(P * 4);
+  L.w = take(P * 4);
+  L.counts = take(E * 4);
+  L.offsets = take((E + 1) * 4);
+  L.row_of_pair = take(P * 4);
+  L.pair_of_row = take(rows * 4);
+  L.chunk_counts = take((nchunks > 0 ? nchunks : 1) * E * 4);
+  L.x_perm = take(rows * H * xelem);
+  L.x_perm_scale = take(is_fp8(p) ? rows * (H / 128) * 4 : 0);
+  L.h = take(rows * I * 2);
+  L.y_perm = take(rows * H * 4);
+  L.h_sh = take(T * static_cast<long long>(p->I_shared) * 2);
+  L.y_sh = take(p->I_shared > 0 ? T * H * 4 : 0);
+  L.total = o;
+  L.x_stage = take(T * H * xelem);
+  L.x_scale_stage = take(is_fp8(p) ? T * (H / 128) * 4 : 0);
+  L.out_stage = take(T * H * 2);
+  L.total_host = o;
+  return L;
+}
+
+template <class Tp>
+Tp* at(void* ws, size_t off) {
+  return reinterpret_cast<Tp*>(static_cast<uint8_t*>(ws) + off);
+}
+
+moe_status_t validate(const moe_params_t* p) {
+  if (p == nullptr) return MOE_ERR_INVALID_ARG;
+  if (p->T < 0 || p->H <= 0 || p->I <= 0 || p->E <= 0 || p->K <= 0) return MOE_ERR_INVALID_ARG;
+  if (p->E > kMaxExperts || p->K > kMaxTopK || p->K > p->E) return MOE_ERR_INVALID_ARG;
+  if (p->score_fn != MOE_SCORE_SOFTMAX && p->score_fn != MOE_SCORE_SIGMOID) return MOE_ERR_INVALID_ARG;
+  if (p->dtype != MOE_DTYPE_BF16 && p->dtype != MOE_DTYPE_FP8_E4M3) return MOE_ERR_INVALID_ARG;
+  if (p->n_group < 1 || p->n_group > 32 || p->E % p->n_group != 0) return MOE_ERR_INVALID_ARG;
+  if (p->n_group > 1) {
+    const int gs = p->E / p->n_group;
+    if (p->topk_group < 1 || p->topk_group > p->n_group) return MOE_ERR_INVALID_ARG;
+    if (p->group_topn < 1 || p->group_topn > gs) return MOE_ERR_INVALID_ARG;
+    if (p->topk_group * gs < p->K) return MOE_ERR_INVALID_ARG;
+  }
+  if (p->I_shared < 0) return MOE_ERR_INVALID_ARG;
+  if (p->H % 128 != 0 || p->I % 128 != 0 || p->I_shared % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  if (p->block_m != 0 && p->block_m != kBlockM) return MOE_ERR_UNSUPPORTED;
+  const long long rows = static_cast<long long>(p->T) * p->K + static_cast<long long>(p->E) * (kBlockM - 1);
+  if (rows >= (1LL << 31) / 2) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+moe_status_t check_ws(const moe_params_t* p, const void* ws, size_t ws_bytes, bool host) {
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return MOE_ERR_INVALID_ARG;
+  const Layout L = layout(p);
+  if (ws_bytes < (host ? L.total_host : L.total)) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+#define MOE_TRY(expr)                          \
+  do {                                         \
+    const moe_status_t s_ = (expr);            \
+    if (s_ != MOE_OK) return s_;               \
+  } while (0)
+
+#define MOE_CUDA(expr) MOE_TRY(cuda_status(expr))
+
+// ---------------------------------------------------------------- stages (no validation)
+moe_status_t do_route(const moe_params_t* p, const void* x, const float* x_scale, const void* w_r,
+                      const float* bias, int32_t* ids, float* w, void* ws, cudaStream_t st) {
+  const Layout L = layout(p);
+  int32_t* status = at<int32_t>(ws, L.status);
+  const void* xb = x;
+  if (is_fp8(p)) {
+    MOE_CUDA(launch_dequant_x(static_cast<const uint8_t*>(x), x_scale, p->T, p->H, at<void>(ws, L.xb), st));
+    xb = at<void>(ws, L.xb);
+  }
+  float* logits = at<float>(ws, L.logits);
+  MOE_CUDA(gemm_router(xb, w_r, p->T, p->H, p->E, logits, status, st));
+  MOE_CUDA(launch_topk(logits, *p, bias, ids, w, st));
+  return MOE_OK;
+}
+
+moe_status_t do_permute(const moe_params_t* p, const int32_t* ids, const void* x, const float* x_scale,
+                        int32_t* counts, int32_t* offsets, int32_t* rop, int32_t* por, void* x_perm,
+                        float* x_perm_scale, void* ws, cudaStream_t st) {
+  const Layout L = layout(p);
+  return cuda_status(launch_permute(*p, ids, x, x_scale, counts, offsets, rop, por, x_perm, x_perm_scale,
+                                    at<int32_t>(ws, L.chunk_counts), at<int32_t>(ws, L.status), st));
+}
+
+moe_status_t do_expert_ffn(const moe_params_t* p, const void* x_perm, const int32_t* offsets,
+                           const int32_t* counts, const void* w_gate, const void* w_up,
+                           const void* w_down, float* y_perm, void* ws, cudaStream_t st) {
+  if (is_fp8(p)) return MOE_ERR_UNSUPPORTED;
+  const Layout L = layout(p);
+  int32_t* status = at<int32_t>(ws, L.status);
+  void* h = at<void>(ws, L.h);
+  MOE_CUDA(gemm_gateup_swiglu(x_perm, L.max_rows, offsets, counts, p->E, 0, w_gate, w_up, p->I, p->H,
+                              h, status, MOE_K_GATEUP, st));
+  MOE_CUDA(gemm_down(h, L.max_rows, offsets, counts, p->E, 0, w_down, p->H, p->I, y_perm, status,
+                     MOE_K_DOWN, st));
+  return MOE_OK;
+}
+
+moe_status_t do_shared(const moe_params_t* p, const void* x, const void* wsg, const void* wsu,
+                       const void* wsd, float* y_sh, void* ws, cudaStream_t st) {
+  const Layout L = layout(p);
+  int32_t* status = at<int32_t>(ws, L.status);
+  void* h = at<void>(ws, L.h_sh);
+  MOE_CUDA(gemm_gateup_swiglu(x, p->T, nullptr, nullptr, 1, p->T, wsg, wsu, p->I_shared, p->H, h,
+                              status, MOE_K_SHARED_GATEUP, st));
+  MOE_CUDA(gemm_down(h, p->T, nullptr, nullptr, 1, p->T, wsd, p->H, p->I_shared, y_sh, status,
+                     MOE_K_SHARED_DOWN, st));
+  return MOE_OK;
+}
+
+moe_status_t do_layer(const moe_params_t* p, const void* x, const float* x_scale, const void* w_r,
+                      const float* bias, const void* w_gate, const void* w_up, const void* w_down,
+                      const void* wsg, const void* wsu, const void* wsd, void* out, int32_t* ids_out,
+                      float* w_out, int32_t* counts_out, void* ws, cudaStream_t st) {
+  const Layout L = layout(p);
+  if (p->T == 0) return MOE_OK;
+  int32_t* ids = ids_out ? ids_out : at<int32_t>(ws, L.ids);
+  float* w = w_out ? w_out : at<float>(ws, L.w);
+  int32_t* counts = counts_out ? counts_out : at<int32_t>(ws, L.counts);
+  int32_t* offsets = at<int32_t>(ws, L.offsets);
+  int32_t* rop = at<int32_t>(ws, L.row_of_pair);
+  float* y_perm = at<float>(ws, L.y_perm);
+  MOE_TRY(do_route(p, x, x_scale, w_r, bias, ids, w, ws, st));
+  MOE_TRY(do_permute(p, ids, x, x_scale, counts, offsets, rop, at<int32_t>(ws, L.pair_of_row),
+                     at<void>(ws, L.x_perm), at<float>(ws, L.x_perm_scale), ws, st));
+  MOE_TRY(do_expert_ffn(p, at<void>(ws, L.x_perm), offsets, counts, w_gate, w_up, w_down, y_perm, ws, st));
+  float* y_sh = nullptr;
+  if (p->I_shared > 0) {
+    y_sh = at<float>(ws, L.y_sh);
+    MOE_TRY(do_shared(p, x, wsg, wsu, wsd, y_sh, ws, st));
+  }
+  return cuda_status(launch_combine(*p, y_perm, rop, w, y_sh, out, st));
+}
+
+moe_status_t check_layer_args(const moe_params_t* p, const void* x, const float* x_scale, const void* w_r,
+                              const void* w_gate, const void* w_up, const void* w_down, const void* wsg,
+                              const void* wsu, const void* wsd, const void* out) {
+  if (!x || !w_r || !w_gate || !w_up || !w_down || !out) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_r) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down) ||
+      !aligned16(out))
+    return MOE_ERR_INVALID_ARG;
+  if (is_fp8(p) && !x_scale) return MOE_ERR_INVALID_ARG;
+  if (p->I_shared > 0) {
+    if (!wsg || !wsu || !wsd) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(wsg) || !aligned16(wsu) || !aligned16(wsd)) return MOE_ERR_INVALID_ARG;
+  }
+  return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+size_t moe_workspace_size(const moe_params_t* p) {
+  if (validate(p) != MOE_OK) return 0;
+  return layout(p).total;
+}
+
+size_t moe_workspace_size_host(const moe_params_t* p) {
+  if (validate(p) != MOE_OK) return 0;
+  return layout(p).total_host;
+}
+
+int64_t moe_max_padded_rows(const moe_params_t* p) {
+  if (validate(p) != MOE_OK) return -1;
+  return layout(p).max_rows;
+}
+
+moe_status_t moe_route(const moe_params_t* p, const void* x, const float* x_scale, const void* w_r,
+                       const float* bias, int32_t* topk_ids, float* topk_w, void* ws, size_t ws_bytes,
+                       void* stream) {
+  MOE_TRY(validate(p));
+  MOE_TRY(check_ws(p, ws, ws_bytes, false));
+  if (!x || !w_r || !topk_ids || !topk_w || !aligned16(x) || !aligned16(w_r)) return MOE_ERR_INVALID_ARG;
+  if (is_fp8(p) && !x_scale) return MOE_ERR_INVALID_ARG;
+  if (p->T == 0) return MOE_OK;
+  return do_route(p, x, x_scale, w_r, bias, topk_ids, topk_w, ws, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_permute(const moe_params_t* p, const int32_t* topk_ids, const void* x, const float* x_scale,
+                         int32_t* counts, int32_t* offsets_padded, int32_t* row_of_pair, int32_t* pair_of_row,
+                         void* x_perm, float* x_perm_scale, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(validate(p));
+  MOE_TRY(check_ws(p, ws, ws_bytes, false));
+  if (!topk_ids || !x || !counts || !offsets_padded || !row_of_pair || !pair_of_row || !x_perm)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(x_perm)) return MOE_ERR_INVALID_ARG;
+  if (is_fp8(p) && (!x_scale || !x_perm_scale)) return MOE_ERR_INVALID_ARG;
+  return do_permute(p, topk_ids, x, x_scale, counts, offsets_padded, row_of_pair, pair_of_row, x_perm,
+                    x_perm_scale, ws, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_expert_ffn(const moe_params_t* p, const void* x_perm, const float* x_perm_scale,
+                            const int32_t* offsets_padded, const int32_t* counts, const void* w_gate,
+                            const void* w_up, const void* w_down, const float* w_gate_scale,
+                            const float* w_up_scale, const float* w_down_scale, float* y_perm,
+                            void* ws, size_t ws_bytes, void* stream) {
+  (void)x_perm_scale; (void)w_gate_scale; (void)w_up_scale; (void)w_down_scale;
+  MOE_TRY(validate(p));
+  MOE_TRY(check_ws(p, ws, ws_bytes, false));
+  if (!x_perm || !offsets_padded || !w_gate || !w_up || !w_down || !y_perm) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x_perm) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down) || !aligned16(y_perm))
+    return MOE_ERR_INVALID_ARG;
+  if (p->T == 0) return MOE_OK;
+  return do_expert_ffn(p, x_perm, offsets_padded, counts, w_gate, w_up, w_down, y_perm, ws,
+                       static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_shared_expert_ffn(const moe_params_t* p, const void* x, const void* ws_gate,
+                                   const void* ws_up, const void* ws_down, float* y_shared, void* ws,
+                                   size_t ws_bytes, void* stream) {
+  MOE_TRY(validate(p));
+  MOE_TRY(check_ws(p, ws, ws_bytes, false));
+  if (p->I_shared <= 0 || is_fp8(p)) return MOE_ERR_UNSUPPORTED;
+  if (!x || !ws_gate || !ws_up || !ws_down || !y_shared) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(ws_gate) || !aligned16(ws_up) || !aligned16(ws_down) || !aligned16(y_shared))
+    return MOE_ERR_INVALID_ARG;
+  if (p->T == 0) return MOE_OK;
+  return do_shared(p, x, ws_gate, ws_up, ws_down, y_shared, ws, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_combine(const moe_params_t* p, const float* y_perm, const int32_t* row_of_pair,
+                         const float* topk_w, const float* y_shared, void* out, void* stream) {
+  MOE_TRY(validate(p));
+  if (!y_perm || !row_of_pair || !topk_w || !out) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y_perm) || !aligned16(out) || (y_shared && !aligned16(y_shared))) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_combine(*p, y_perm, row_of_pair, topk_w, y_shared, out,
+                                    static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_layer_forward(const moe_params_t* p, const void* x, const float* x_scale, const void* w_r,
+                               const float* bias, const void* w_gate, const void* w_up, const void* w_down,
+                               const float* w_gate_scale, const float* w_up_scale, const float* w_down_scale,
+                               const void* ws_gate, const void* ws_up, const void* ws_down, void* out,
+                               int32_t* topk_ids_out, float* topk_w_out, int32_t* counts_out, void* ws,
+                               size_t ws_bytes, void* stream) {
+  (void)w_gate_scale; (void)w_up_scale; (void)w_down_scale;
+  MOE_TRY(validate(p));
+  MOE_TRY(check_ws(p, ws, ws_bytes, false));
+  MOE_TRY(check_layer_args(p, x, x_scale, w_r, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, out));
+  if (is_fp8(p)) return MOE_ERR_UNSUPPORTED;
+  return do_layer(p, x, x_scale, w_r, bias, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, out, topk_ids_out,
+                  topk_w_out, counts_out, ws, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_layer_forward_host(const moe_params_t* p, const void* x_host, const float* x_scale_host,
+                                    const void* w_r, const float* bias, const void* w_gate, const void* w_up,
+                                    const void* w_down, const float* w_gate_scale, const float* w_up_scale,
+                                    const float* w_down_scale, const void* ws_gate, const void* ws_up,
+                                    const void* ws_down, void* out_host, void* ws, size_t ws_bytes,
+                                    void* stream) {
+  (void)w_gate_scale; (void)w_up_scale; (void)w_down_scale;
+  MOE_TRY(validate(p));
+  MOE_TRY(check_ws(p, ws, ws_bytes, true));
+  if (!x_host || !out_host) return MOE_ERR_INVALID_ARG;
+  if (is_fp8(p)) return MOE_ERR_UNSUPPORTED;
+  const Layout L = layout(p);
+  void* x_dev = at<void>(ws, L.x_stage);
+  void* out_dev = at<void>(ws, L.out_stage);
+  MOE_TRY(check_layer_args(p, x_dev, nullptr, w_r, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, out_dev));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t xbytes = static_cast<size_t>(p->T) * p->H * 2;
+  if (p->T == 0) return MOE_OK;
+  MOE_CUDA(cudaMemcpyAsync(x_dev, x_host, xbytes, cudaMemcpyHostToDevice, st));
+  MOE_TRY(do_layer(p, x_dev, nullptr, w_r, bias, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, out_dev,
+                   nullptr, nullptr, nullptr, ws, st));
+  MOE_CUDA(cudaMemcpyAsync(out_host, out_dev, static_cast<size_t>(p->T) * p->H * 2, cudaMemcpyDeviceToHost, st));
+  return MOE_OK;
+}
+
+moe_status_t moe_get_device_status(const void* ws, void* stream, int32_t* host_status) {
+  if (!ws || !host_status) return MOE_ERR_INVALID_ARG;
+  MOE_CUDA(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  MOE_CUDA(cudaMemcpy(host_status, ws, sizeof(int32_t), cudaMemcpyDeviceToHost));
+  return MOE_OK;
+}
+
+moe_status_t moe_clear_device_status(void* ws, void* stream) {
+  if (!ws) return MOE_ERR_INVALID_ARG;
+  return cuda_status(cudaMemsetAsync(ws, 0, 256, static_cast<cudaStream_t>(stream)));
+}
+
+const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MOE_ERR_CUDA: return "CUDA runtime error";
+    case MOE_ERR_TIMEOUT: return "device pipeline wait timed out";
+    case MOE_ERR_DEVICE: return "device detected bad input";
+  }
+  return "unknown status";
+}
+
+int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+moe_status_t moe_trace_enable(uint32_t kernel_mask, int32_t capacity) {
+  if (capacity <= 0 || capacity > (1 << 20)) return MOE_ERR_INVALID_ARG;
+  Trace& t = g_trace;
+  if (static_cast<int>(t.kid.size()) < capacity) {
+    const size_t have = t.ev.size();
+    t.ev.resize(2 * static_cast<size_t>(capacity));
+    for (size_t i = have; i < t.ev.size(); ++i)
+      if (cudaEventCreate(&t.ev[i]) != cudaSuccess) return MOE_ERR_CUDA;
+    t.kid.resize(capacity);
+  }
+  t.cap = capacity;
+  t.mask = kernel_mask;
+  t.n = 0;
+  t.on = true;
+  return MOE_OK;
+}
+
+moe_status_t moe_trace_disable(void) {
+  g_trace.on = false;
+  return MOE_OK;
+}
+
+int32_t moe_trace_collect(int32_t* kernel_ids, float* ms, int32_t max_out) {
+  Trace& t = g_trace;
+  int32_t n = 0;
+  for (int i = 0; i < t.n && n < max_out; ++i) {
+    if (cudaEventSynchronize(t.ev[2 * i + 1]) != cudaSuccess) break;
+    float v = 0.f;
+    if (cudaEventElapsedTime(&v, t.ev[2 * i], t.ev[2 * i + 1]) != cudaSuccess) break;
+    if (kernel_ids) kernel_ids[n] = t.kid[i];
+    if (ms) ms[n] = v;
+    ++n;
+  }
+  t.n = 0;
+  return n;
+}
+
+int32_t moe_layer_launch_count(const moe_params_t* p) {
+  if (validate(p) != MOE_OK) return -1;
+  if (p->T == 0) return 0;
+  int n = 2;                                 // router GEMM, top-k
+  if (is_fp8(p)) n += 1;                     // dequantise x for the router
+  n += (p->T * p->K > 0) ? 4 : 2;            // count, scan, rank, gather
+  n += 2;                                    // gate/up, down
+  if (p->I_shared > 0) n += 2;               // shared gate/up, down
+  n += 1;                                    // combine
+  return n;
+}
+
+}  // extern "C"

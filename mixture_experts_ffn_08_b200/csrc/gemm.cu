@@ -1,0 +1,155 @@
+// Host side of the tcgen05 GEMMs: TMA tensor maps and the launch configurations used
+// for the router logits, the gate/up projection with fused SwiGLU and the down
+// projection.
+#include <cudaTypedefs.h>
+
+#include "internal.h"
+#include "tc_gemm.cuh"
+
+namespace moe {
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// Row-major bf16 matrix [rows, cols], box of 64 columns (128 bytes) x box_rows rows,
+// 128-byte swizzle; out-of-range rows read as zero.
+bool make_tmap_bf16(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols,
+                    uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <class Cfg>
+cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                   const GemmParams& gp, long long max_items, int kid, cudaStream_t st) {
+  auto kern = tc_gemm_kernel<Cfg>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Cfg::SMEM_BYTES);
+  if (err != cudaSuccess) return err;
+  const long long sms = num_sms();
+  const int grid = static_cast<int>(max_items < sms ? (max_items > 0 ? max_items : 1) : sms);
+  trace_before(kid, st);
+  kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, st>>>(a, b0, b1, gp);
+  trace_after(kid, st);
+  return cudaGetLastError();
+}
+
+long long ceil_div(long long a, long long b) { return (a + b - 1) / b; }
+
+}  // namespace
+
+cudaError_t gemm_router(const void* x, const void* w_r, int T, int H, int E, float* logits,
+                        int32_t* status, cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  const int bn = E >= 256 ? 256 : ((E + 15) / 16) * 16;
+  CUtensorMap ta, tb;
+  if (!make_tmap_bf16(&ta, x, T, H, 128) || !make_tmap_bf16(&tb, w_r, E, H, bn))
+    return cudaErrorInvalidValue;
+  GemmParams gp{};
+  gp.offsets = nullptr;
+  gp.counts = nullptr;
+  gp.G = 1;
+  gp.dense_rows = T;
+  gp.K = H;
+  gp.N = E;
+  gp.b_rows_per_group = E;
+  gp.out = logits;
+  gp.ldo = E;
+  gp.status = status;
+  const long long items = ceil_div(T, 128) * ceil_div(E, bn);
+#define MOE_ROUTER_CASE(BN, ST) \
+  return launch<GemmCfg<BN, EPI_F32, ST>>(ta, tb, tb, gp, items, MOE_K_ROUTER_GEMM, st)
+  switch (bn) {
+    case 16: MOE_ROUTER_CASE(16, 8);
+    case 32: MOE_ROUTER_CASE(32, 8);
+    case 48: MOE_ROUTER_CASE(48, 8);
+    case 64: MOE_ROUTER_CASE(64, 8);
+    case 80: MOE_ROUTER_CASE(80, 6);
+    case 96: MOE_ROUTER_CASE(96, 6);
+    case 112: MOE_ROUTER_CASE(112, 6);
+    case 128: MOE_ROUTER_CASE(128, 6);
+    case 144: MOE_ROUTER_CASE(144, 5);
+    case 160: MOE_ROUTER_CASE(160, 5);
+    case 176: MOE_ROUTER_CASE(176, 5);
+    case 192: MOE_ROUTER_CASE(192, 5);
+    case 208: MOE_ROUTER_CASE(208, 4);
+    case 224: MOE_ROUTER_CASE(224, 4);
+    case 240: MOE_ROUTER_CASE(240, 4);
+    default: MOE_ROUTER_CASE(256, 4);
+  }
+#undef MOE_ROUTER_CASE
+}
+
+cudaError_t gemm_gateup_swiglu(const void* A, int64_t a_rows, const int32_t* offsets,
+                               const int32_t* counts, int G, int dense_rows, const void* w_gate,
+                               const void* w_up, int N, int K, void* h, int32_t* status, int kid,
+                               cudaStream_t st) {
+  using Cfg = GemmCfg<256, EPI_SWIGLU, 4>;
+  CUtensorMap ta, tg, tu;
+  if (!make_tmap_bf16(&ta, A, a_rows, K, 128) ||
+      !make_tmap_bf16(&tg, w_gate, static_cast<uint64_t>(G) * N, K, 128) ||
+      !make_tmap_bf16(&tu, w_up, static_cast<uint64_t>(G) * N, K, 128))
+    return cudaErrorInvalidValue;
+  GemmParams gp{};
+  gp.offsets = offsets;
+  gp.counts = counts;
+  gp.G = G;
+  gp.dense_rows = dense_rows;
+  gp.K = K;
+  gp.N = N;
+  gp.b_rows_per_group = N;
+  gp.out = h;
+  gp.ldo = N;
+  gp.status = status;
+  const long long items = ceil_div(a_rows, 128) * ceil_div(N, Cfg::OUT_COLS);
+  return launch<Cfg>(ta, tg, tu, gp, items, kid, st);
+}
+
+cudaError_t gemm_down(const void* A, int64_t a_rows, const int32_t* offsets,
+                      const int32_t* counts, int G, int dense_rows, const void* w, int N, int K,
+                      float* y, int32_t* status, int kid, cudaStream_t st) {
+  CUtensorMap ta, tb;
+  const bool wide = N % 256 == 0;
+  if (!make_tmap_bf16(&ta, A, a_rows, K, 128) ||
+      !make_tmap_bf16(&tb, w, static_cast<uint64_t>(G) * N, K, wide ? 256 : 128))
+    return cudaErrorInvalidValue;
+  GemmParams gp{};
+  gp.offsets = offsets;
+  gp.counts = counts;
+  gp.G = G;
+  gp.dense_rows = dense_rows;
+  gp.K = K;
+  gp.N = N;
+  gp.b_rows_per_group = N;
+  gp.out = y;
+  gp.ldo = N;
+  gp.status = status;
+  if (wide) {
+    using Cfg = GemmCfg<256, EPI_F32, 4>;
+    return launch<Cfg>(ta, tb, tb, gp, ceil_div(a_rows, 128) * ceil_div(N, 256), kid, st);
+  }
+  using Cfg = GemmCfg<128, EPI_F32, 6>;
+  return launch<Cfg>(ta, tb, tb, gp, ceil_div(a_rows, 128) * ceil_div(N, 128), kid, st);
+}
+
+}  // namespace moe

@@ -1,0 +1,55 @@
+// Internal launchers shared between the translation units of the library.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+constexpr int kBlockM = 128;    // M-tile of the grouped GEMM = row alignment of buckets
+constexpr int kMaxExperts = 1024;
+constexpr int kMaxTopK = 32;
+constexpr int kPermChunk = 256;  // pairs per chunk of the stable bucket ranking
+
+// Tracing (api.cu): brackets a launch of kernel `kid` with events when enabled.
+void trace_before(int kid, cudaStream_t st);
+void trace_after(int kid, cudaStream_t st);
+int num_sms();
+
+// ---------------------------------------------------------------- routing (kernels.cu)
+cudaError_t launch_dequant_x(const uint8_t* xq, const float* xs, int T, int H, void* x_bf16,
+                             cudaStream_t st);
+cudaError_t launch_topk(const float* logits, const moe_params_t& p, const float* bias,
+                        int32_t* ids, float* w, cudaStream_t st);
+
+// ---------------------------------------------------------------- dispatch (kernels.cu)
+cudaError_t launch_permute(const moe_params_t& p, const int32_t* ids, const void* x,
+                           const float* x_scale, int32_t* counts, int32_t* offsets,
+                           int32_t* row_of_pair, int32_t* pair_of_row, void* x_perm,
+                           float* x_perm_scale, int32_t* chunk_counts, int32_t* status,
+                           cudaStream_t st);
+
+// ---------------------------------------------------------------- combine (kernels.cu)
+cudaError_t launch_combine(const moe_params_t& p, const float* y_perm, const int32_t* row_of_pair,
+                           const float* w, const float* y_shared, void* out, cudaStream_t st);
+
+// ---------------------------------------------------------------- GEMMs (gemm.cu)
+// Router logits [T, E] fp32 = x [T,H] bf16 @ W_r[E,H]^T.
+cudaError_t gemm_router(const void* x, const void* w_r, int T, int H, int E, float* logits,
+                        int32_t* status, cudaStream_t st);
+// h [rows, N] bf16 = SiLU(A Wg^T) * (A Wu^T), grouped by offsets (or dense when null);
+// with counts, pad rows of each group are not stored.
+cudaError_t gemm_gateup_swiglu(const void* A, int64_t a_rows, const int32_t* offsets,
+                               const int32_t* counts, int G, int dense_rows, const void* w_gate,
+                               const void* w_up, int N, int K, void* h, int32_t* status, int kid,
+                               cudaStream_t st);
+// y [rows, N] fp32 = A W^T, grouped by offsets (or dense when null); with counts, pad
+// rows of each group are not stored.
+cudaError_t gemm_down(const void* A, int64_t a_rows, const int32_t* offsets,
+                      const int32_t* counts, int G, int dense_rows, const void* w, int N, int K,
+                      float* y, int32_t* status, int kid, cudaStream_t st);
+
+}  // namespace moe

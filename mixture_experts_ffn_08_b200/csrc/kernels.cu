@@ -1,0 +1,443 @@
+// Routing, dispatch and combine kernels of the MoE layer (sm_100a).
+//
+//   topk_kernel        warp per token: scores, selection bias, group-limited top-k,
+//                      renormalised weights (routing primer "MoE 路由入门" §三, §四,
+//                      §六-§十; "MoE" chapter index §0 "+bias only for selection")
+//   perm_*_kernel      pairs bucketed by expert, stably, each bucket padded to the GEMM
+//                      M-tile (routing primer §5.1): per-chunk histogram -> one-block scan
+//                      -> stable in-chunk ranks with warp match -> row gather of x
+//   combine_kernel     out_t = sum_k w_tk y_tk (+ shared), fixed k order (routing primer
+//                      §5.3), vectorised, no atomics
+#include <cuda_fp8.h>
+#include <math_constants.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+// ================================================================== FP8 x -> bf16 (router)
+// Each e4m3 value times its power-of-two scale is exactly representable in bf16.
+__global__ void dequant_x_kernel(const uint8_t* __restrict__ xq, const float* __restrict__ xs,
+                                 int T, int H, __nv_bfloat16* __restrict__ xb) {
+  const long long n16 = static_cast<long long>(T) * H / 16;
+  for (long long v = blockIdx.x * (long long)blockDim.x + threadIdx.x; v < n16;
+       v += (long long)gridDim.x * blockDim.x) {
+    const long long e0 = v * 16;
+    const int t = static_cast<int>(e0 / H), h = static_cast<int>(e0 % H);
+    const float s = __ldg(xs + static_cast<long long>(t) * (H / 128) + h / 128);
+    const uint4 q = __ldg(reinterpret_cast<const uint4*>(xq) + v);
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const __nv_fp8x2_storage_t pair = static_cast<__nv_fp8x2_storage_t>(w[i] >> (16 * half));
+        const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+        o[2 * i + half] = pack_bf16x2(f.x * s, f.y * s);
+      }
+    }
+    uint4* dst = reinterpret_cast<uint4*>(xb) + v * 2;
+    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
+
+cudaError_t launch_dequant_x(const uint8_t* xq, const float* xs, int T, int H, void* x_bf16,
+                             cudaStream_t st) {
+  const long long n16 = static_cast<long long>(T) * H / 16;
+  const int grid = static_cast<int>(n16 / 256 + 1 < num_sms() * 8 ? n16 / 256 + 1 : num_sms() * 8);
+  trace_before(MOE_K_DEQUANT_X, st);
+  dequant_x_kernel<<<grid, 256, 0, st>>>(xq, xs, T, H, static_cast<__nv_bfloat16*>(x_bf16));
+  trace_after(MOE_K_DEQUANT_X, st);
+  return cudaGetLastError();
+}
+
+// ================================================================== top-k
+// (value, index) order: larger value first, equal values -> lower index first.
+MOE_DEVINL bool better(float v, int i, float v2, int i2) { return v > v2 || (v == v2 && i < i2); }
+
+MOE_DEVINL void warp_argmax(float& v, int& i) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float v2 = __shfl_xor_sync(kFull, v, o);
+    const int i2 = __shfl_xor_sync(kFull, i, o);
+    if (better(v2, i2, v, i)) { v = v2; i = i2; }
+  }
+}
+
+MOE_DEVINL float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+  return v;
+}
+
+MOE_DEVINL float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
+  return v;
+}
+
+// Lane l holds experts l, l+32, l+64, ... (EPL of them): E <= 32 * EPL.
+template <int EPL>
+__global__ void __launch_bounds__(128) topk_kernel(
+    const float* __restrict__ logits, int T, int E, int K, int n_group, int topk_group,
+    int group_topn, int score_fn, int renorm, float scale, const float* __restrict__ bias,
+    int32_t* __restrict__ ids, float* __restrict__ wout) {
+  const int token = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (token >= T) return;  // warp-uniform
+  const float* z = logits + static_cast<long long>(token) * E;
+
+  float s[EPL], c[EPL];
+#pragma unroll
+  for (int j = 0; j < EPL; ++j) {
+    const int e = j * 32 + lane;
+    s[j] = e < E ? __ldg(z + e) : -CUDART_INF_F;
+  }
+  if (score_fn == MOE_SCORE_SOFTMAX) {
+    float m = -CUDART_INF_F;
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) m = fmaxf(m, s[j]);
+    m = warp_max(m);
+    float sum = 0.f;
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) {
+      s[j] = (j * 32 + lane < E) ? expf(s[j] - m) : 0.f;
+      sum += s[j];
+    }
+    sum = warp_sum(sum);
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) s[j] = s[j] / sum;
+  } else {
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) s[j] = (j * 32 + lane < E) ? 1.f / (1.f + expf(-s[j])) : 0.f;
+  }
+#pragma unroll
+  for (int j = 0; j < EPL; ++j) {
+    const int e = j * 32 + lane;
+    c[j] = e < E ? s[j] + (bias ? __ldg(bias + e) : 0.f) : -CUDART_INF_F;
+  }
+
+  if (n_group > 1) {
+    const int gs = E / n_group;
+    float my_gscore = -CUDART_INF_F;  // lane g keeps the score of group g
+    for (int g = 0; g < n_group; ++g) {
+      uint32_t taken = 0;
+      float acc = 0.f;
+      for (int r = 0; r < group_topn; ++r) {
+        float bv = -CUDART_INF_F;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) {
+          const int e = j * 32 + lane;
+          if (e < E && e / gs == g && !((taken >> j) & 1u) && better(c[j], e, bv, bi)) {
+            bv = c[j];
+            bi = e;
+          }
+        }
+        warp_argmax(bv, bi);
+        acc += bv;
+        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+      }
+      if (lane == g) my_gscore = acc;
+    }
+    uint32_t keep = 0;
+    float cand = lane < n_group ? my_gscore : -CUDART_INF_F;
+    for (int r = 0; r < topk_group; ++r) {
+      float bv = cand;
+      int bi = lane;
+      warp_argmax(bv, bi);
+      keep |= 1u << bi;
+      if (lane == bi) cand = -CUDART_INF_F;
+    }
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) {
+      const int e = j * 32 + lane;
+      if (e < E && !((keep >> (e / gs)) & 1u)) c[j] = -CUDART_INF_F;
+    }
+  }
+
+  int my_id = -1;
+  float my_w = 0.f;
+  for (int k = 0; k < K; ++k) {
+    float bv = -CUDART_INF_F;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) {
+      const int e = j * 32 + lane;
+      if (e < E && better(c[j], e, bv, bi)) { bv = c[j]; bi = e; }
+    }
+    warp_argmax(bv, bi);
+    const int owner = bi & 31, jj = bi >> 5;
+    float sv = 0.f;
+#pragma unroll
+    for (int j = 0; j < EPL; ++j)
+      if (j == jj) sv = s[j];
+    sv = __shfl_sync(kFull, sv, owner);
+    if (lane == owner) {
+#pragma unroll
+      for (int j = 0; j < EPL; ++j)
+        if (j == jj) c[j] = -CUDART_INF_F;
+    }
+    if (lane == k) { my_id = bi; my_w = sv; }
+  }
+  const float wsum = warp_sum(my_w);
+  if (renorm) my_w = my_w / wsum;
+  my_w *= scale;
+  if (lane < K) {
+    ids[static_cast<long long>(token) * K + lane] = my_id;
+    wout[static_cast<long long>(token) * K + lane] = my_w;
+  }
+}
+
+cudaError_t launch_topk(const float* logits, const moe_params_t& p, const float* bias,
+                        int32_t* ids, float* w, cudaStream_t st) {
+  const int grid = (p.T + 3) / 4;
+  if (grid == 0) return cudaSuccess;
+  const int epl = (p.E + 31) / 32;
+  trace_before(MOE_K_TOPK, st);
+#define MOE_TOPK_CASE(N)                                                                   \
+  topk_kernel<N><<<grid, 128, 0, st>>>(logits, p.T, p.E, p.K, p.n_group, p.topk_group,    \
+                                       p.group_topn, p.score_fn, p.renormalize,            \
+                                       p.routed_scale, bias, ids, w)
+  if (epl <= 1) MOE_TOPK_CASE(1);
+  else if (epl <= 2) MOE_TOPK_CASE(2);
+  else if (epl <= 4) MOE_TOPK_CASE(4);
+  else if (epl <= 8) MOE_TOPK_CASE(8);
+  else if (epl <= 16) MOE_TOPK_CASE(16);
+  else MOE_TOPK_CASE(32);
+#undef MOE_TOPK_CASE
+  trace_after(MOE_K_TOPK, st);
+  return cudaGetLastError();
+}
+
+// ================================================================== permute
+// 1) per-chunk expert histogram
+__global__ void __launch_bounds__(kPermChunk) perm_count_kernel(
+    const int32_t* __restrict__ ids, int P, int E, int32_t* __restrict__ chunk_counts,
+    int32_t* status) {
+  extern __shared__ int hist[];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int p = blockIdx.x * kPermChunk + threadIdx.x;
+  if (p < P) {
+    const int e = __ldg(ids + p);
+    if (e >= 0 && e < E) atomicAdd(&hist[e], 1);
+    else set_status(status, MOE_DEV_BAD_EXPERT_ID);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    chunk_counts[static_cast<long long>(blockIdx.x) * E + e] = hist[e];
+}
+
+// 2) one block: expert totals, padded exclusive scan -> offsets, and per-chunk bases
+//    (chunk_counts is overwritten with the first row of each (chunk, expert) run).
+__global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t* __restrict__ chunk_counts,
+                                                         int nchunks, int E, int block_m,
+                                                         int32_t* __restrict__ counts,
+                                                         int32_t* __restrict__ offsets) {
+  __shared__ int warp_tot[32];
+  const int e = threadIdx.x, lane = e & 31, w = e >> 5;
+  int total = 0;
+  if (e < E)
+    for (int c = 0; c < nchunks; ++c) total += chunk_counts[static_cast<long long>(c) * E + e];
+  const int padded = e < E ? (total + block_m - 1) / block_m * block_m : 0;
+  // inclusive scan of `padded` across the block
+  int v = padded;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(kFull, v, o);
+    if (lane >= o) v += n;
+  }
+  if (lane == 31) warp_tot[w] = v;
+  __syncthreads();
+  if (w == 0) {
+    int t = warp_tot[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(kFull, t, o);
+      if (lane >= o) t += n;
+    }
+    warp_tot[lane] = t;  // inclusive totals of warps 0..lane
+  }
+  __syncthreads();
+  const int incl = v + (w > 0 ? warp_tot[w - 1] : 0);
+  const int excl = incl - padded;
+  if (e < E) {
+    counts[e] = total;
+    offsets[e] = excl;
+    int run = excl;
+    for (int c = 0; c < nchunks; ++c) {
+      const long long idx = static_cast<long long>(c) * E + e;
+      const int n = chunk_counts[idx];
+      chunk_counts[idx] = run;
+      run += n;
+    }
+  }
+  if (e == E - 1) offsets[E] = incl;
+}
+
+// 3) stable rank inside each chunk: one warp per chunk walks its pairs in order,
+//    32 at a time; lanes with the same expert are ranked by lane (warp match).
+constexpr int kRankWarps = 4;
+__global__ void __launch_bounds__(32 * kRankWarps) perm_rank_kernel(
+    const int32_t* __restrict__ ids, int P, int E, const int32_t* __restrict__ chunk_base,
+    int32_t* __restrict__ row_of_pair, int32_t* __restrict__ pair_of_row) {
+  extern __shared__ int run_cnt[];  // [kRankWarps][E]
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int* my = run_cnt + w * E;
+  for (int e = lane; e < E; e += 32) my[e] = 0;
+  __syncwarp();
+  const int chunk = blockIdx.x * kRankWarps + w;
+  if (chunk * kPermChunk >= P) return;  // warp-uniform
+  const int32_t* base = chunk_base + static_cast<long long>(chunk) * E;
+  for (int it = 0; it < kPermChunk / 32; ++it) {
+    const int p = chunk * kPermChunk + it * 32 + lane;
+    const int e = p < P ? __ldg(ids + p) : -1;
+    const bool ok = p < P && e >= 0 && e < E;
+    const int key = ok ? e : -1 - lane;  // invalid lanes match nobody
+    const unsigned peers = __match_any_sync(kFull, key);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    const int run = ok ? my[e] : 0;
+    __syncwarp();
+    if (ok) {
+      const int row = __ldg(base + e) + run + rank;
+      row_of_pair[p] = row;
+      pair_of_row[row] = p;
+      if (rank == 0) my[e] = run + __popc(peers);
+    } else if (p < P) {
+      row_of_pair[p] = -1;
+    }
+    __syncwarp();
+  }
+}
+
+// 4) row gather: x_perm[r] = x[pair_of_row[r] / K]; pad rows -> zero, pair -1.
+template <bool FP8>
+__global__ void __launch_bounds__(256) perm_gather_kernel(
+    const void* __restrict__ x, const float* __restrict__ x_scale, int H, int K, int E,
+    const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets,
+    int32_t* __restrict__ pair_of_row, void* __restrict__ x_perm,
+    float* __restrict__ x_perm_scale) {
+  const int total = __ldg(offsets + E);
+  const int row_bytes = FP8 ? H : 2 * H;
+  const int nvec = row_bytes / 16;
+  const int nsc = H / 128;
+  for (int r = blockIdx.x; r < total; r += gridDim.x) {
+    int lo = 0, hi = E - 1;  // expert owning row r: smallest e with offsets[e+1] > r
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (__ldg(offsets + mid + 1) > r) hi = mid; else lo = mid + 1;
+    }
+    const bool pad = r - __ldg(offsets + lo) >= __ldg(counts + lo);
+    const long long t = pad ? 0 : pair_of_row[r] / K;
+    if (pad && threadIdx.x == 0) pair_of_row[r] = -1;
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(x_perm) + static_cast<long long>(r) * row_bytes);
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(x) + t * row_bytes);
+    for (int v = threadIdx.x; v < nvec; v += blockDim.x)
+      dst[v] = pad ? make_uint4(0, 0, 0, 0) : __ldg(src + v);
+    if (FP8) {
+      for (int j = threadIdx.x; j < nsc; j += blockDim.x)
+        x_perm_scale[static_cast<long long>(r) * nsc + j] = pad ? 1.0f : __ldg(x_scale + t * nsc + j);
+    }
+  }
+}
+
+cudaError_t launch_permute(const moe_params_t& p, const int32_t* ids, const void* x,
+                           const float* x_scale, int32_t* counts, int32_t* offsets,
+                           int32_t* row_of_pair, int32_t* pair_of_row, void* x_perm,
+                           float* x_perm_scale, int32_t* chunk_counts, int32_t* status,
+                           cudaStream_t st) {
+  const int P = p.T * p.K;
+  const int nchunks = (P + kPermChunk - 1) / kPermChunk;
+  const int bm = kBlockM;
+  cudaError_t err;
+  if (nchunks > 0) {
+    trace_before(MOE_K_PERM_COUNT, st);
+    perm_count_kernel<<<nchunks, kPermChunk, p.E * sizeof(int), st>>>(ids, P, p.E, chunk_counts, status);
+    trace_after(MOE_K_PERM_COUNT, st);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  }
+  trace_before(MOE_K_PERM_SCAN, st);
+  perm_scan_kernel<<<1, 1024, 0, st>>>(chunk_counts, nchunks, p.E, bm, counts, offsets);
+  trace_after(MOE_K_PERM_SCAN, st);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  if (nchunks > 0) {
+    trace_before(MOE_K_PERM_RANK, st);
+    const int blocks = (nchunks + kRankWarps - 1) / kRankWarps;
+    perm_rank_kernel<<<blocks, 32 * kRankWarps, kRankWarps * p.E * sizeof(int), st>>>(
+        ids, P, p.E, chunk_counts, row_of_pair, pair_of_row);
+    trace_after(MOE_K_PERM_RANK, st);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  }
+  const long long max_rows = static_cast<long long>(P) + static_cast<long long>(p.E) * (bm - 1);
+  const int grid = static_cast<int>(max_rows < num_sms() * 16LL ? (max_rows > 0 ? max_rows : 1) : num_sms() * 16LL);
+  trace_before(MOE_K_PERM_GATHER, st);
+  if (p.dtype == MOE_DTYPE_FP8_E4M3)
+    perm_gather_kernel<true><<<grid, 256, 0, st>>>(x, x_scale, p.H, p.K, p.E, counts, offsets,
+                                                   pair_of_row, x_perm, x_perm_scale);
+  else
+    perm_gather_kernel<false><<<grid, 256, 0, st>>>(x, x_scale, p.H, p.K, p.E, counts, offsets,
+                                                    pair_of_row, x_perm, x_perm_scale);
+  trace_after(MOE_K_PERM_GATHER, st);
+  return cudaGetLastError();
+}
+
+// ================================================================== combine
+__global__ void __launch_bounds__(128) combine_kernel(
+    const float* __restrict__ y_perm, const int32_t* __restrict__ row_of_pair,
+    const float* __restrict__ w, const float* __restrict__ y_sh,
+    __nv_bfloat16* __restrict__ out, int T, int H, int K) {
+  __shared__ int rows[kMaxTopK];
+  __shared__ float wk[kMaxTopK];
+  const int nvec = H / 8;  // 8 outputs (two float4 loads, one 16-byte store) per thread step
+  for (int t = blockIdx.x; t < T; t += gridDim.x) {
+    __syncthreads();
+    if (threadIdx.x < K) {
+      rows[threadIdx.x] = __ldg(row_of_pair + static_cast<long long>(t) * K + threadIdx.x);
+      wk[threadIdx.x] = __ldg(w + static_cast<long long>(t) * K + threadIdx.x);
+    }
+    __syncthreads();
+    for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      for (int k = 0; k < K; ++k) {
+        const int r = rows[k];
+        if (r < 0) continue;
+        const float4* src = reinterpret_cast<const float4*>(y_perm + static_cast<long long>(r) * H) + 2 * v;
+        const float4 a = __ldg(src), b = __ldg(src + 1);
+        const float wv = wk[k];
+        acc[0] = fmaf(wv, a.x, acc[0]); acc[1] = fmaf(wv, a.y, acc[1]);
+        acc[2] = fmaf(wv, a.z, acc[2]); acc[3] = fmaf(wv, a.w, acc[3]);
+        acc[4] = fmaf(wv, b.x, acc[4]); acc[5] = fmaf(wv, b.y, acc[5]);
+        acc[6] = fmaf(wv, b.z, acc[6]); acc[7] = fmaf(wv, b.w, acc[7]);
+      }
+      if (y_sh) {
+        const float4* src = reinterpret_cast<const float4*>(y_sh + static_cast<long long>(t) * H) + 2 * v;
+        const float4 a = __ldg(src), b = __ldg(src + 1);
+        acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+        acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+      }
+      reinterpret_cast<uint4*>(out + static_cast<long long>(t) * H)[v] =
+          make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                     pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+    }
+  }
+}
+
+cudaError_t launch_combine(const moe_params_t& p, const float* y_perm, const int32_t* row_of_pair,
+                           const float* w, const float* y_shared, void* out, cudaStream_t st) {
+  if (p.T == 0) return cudaSuccess;
+  const int grid = p.T < num_sms() * 16 ? p.T : num_sms() * 16;
+  trace_before(MOE_K_COMBINE, st);
+  combine_kernel<<<grid, 128, 0, st>>>(y_perm, row_of_pair, w, y_shared,
+                                       static_cast<__nv_bfloat16*>(out), p.T, p.H, p.K);
+  trace_after(MOE_K_COMBINE, st);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

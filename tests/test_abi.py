@@ -1,0 +1,100 @@
+"""The C-ABI library without a GPU: it loads, exports every function include/moe.h
+declares, sizes workspaces and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from mixture_experts_ffn_08_b200 import binding as B
+from mixture_experts_ffn_08_b200 import workloads as W
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if not h.endswith(".h"):
+            continue
+        src = open(os.path.join(ROOT, "include", h), encoding="utf-8").read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names |= set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", src))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(B._LIB_PATH):
+        from mixture_experts_ffn_08_b200 import build
+        build.build()
+    return B.lib(require_gpu=False)
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = _declared_functions()
+    assert {"moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward"} <= declared
+    raw = ctypes.CDLL(B._LIB_PATH)
+    for name in declared:
+        assert hasattr(raw, name), name
+    assert declared == set(B.EXPORTED), declared ^ set(B.EXPORTED)
+    assert lib.moe_abi_version() == 1
+
+
+def test_params_struct_matches_header():
+    src = open(os.path.join(ROOT, "include", "moe.h"), encoding="utf-8").read()
+    body = re.search(r"typedef struct moe_params \{(.*?)\} moe_params_t;", src, re.S).group(1)
+    fields = re.findall(r"(?:int32_t|float)\s+(\w+);", re.sub(r"/\*.*?\*/", "", body, flags=re.S))
+    assert fields == [f[0] for f in B.MoeParams._fields_]
+    assert ctypes.sizeof(B.MoeParams) == 4 * len(fields)
+
+
+def test_sizes(lib):
+    for wl in W.ALL.values():
+        p = B.params(wl)
+        rows = B.moe_max_padded_rows(p)
+        assert rows == wl.T * wl.K + wl.E * (B.BLOCK_M - 1)
+        ws = B.moe_workspace_size(p)
+        assert ws >= rows * wl.H * (1 if wl.dtype else 2) * 2
+        assert B.moe_workspace_size_host(p) > ws
+        assert B.moe_layer_launch_count(p) == 9 + (2 if wl.I_shared else 0) + (1 if wl.dtype else 0)
+
+
+@pytest.mark.parametrize("change", [dict(H=100), dict(I=200), dict(K=0), dict(E=2000),
+                                    dict(K=40), dict(n_group=3), dict(topk_group=9),
+                                    dict(group_topn=40), dict(score_fn=5), dict(dtype=7),
+                                    dict(I_shared=100), dict(T=-1)])
+def test_invalid_params_give_no_workspace(lib, change):
+    wl = W.DSV3_PREFILL.with_(**change)
+    p = B.params(wl)
+    assert B.moe_workspace_size(p) == 0
+    assert B.moe_max_padded_rows(p) == -1
+
+
+def test_invalid_args_rejected_on_host(lib):
+    p = B.params(W.TINY)
+    size = B.moe_workspace_size(p)
+    # a null pointer, a misaligned workspace and a short workspace all fail before any launch
+    assert lib.moe_route(ctypes.byref(p), None, None, None, None, None, None, 256, size, None) == 1
+    assert lib.moe_route(ctypes.byref(p), 256, None, 256, None, 256, 256, 260, size, None) == 1
+    assert lib.moe_route(ctypes.byref(p), 256, None, 256, None, 256, 256, 256, 100, None) == 1
+    assert lib.moe_combine(ctypes.byref(p), None, None, None, None, None, None) == 1
+    bad = B.params(W.TINY.with_(H=100))
+    assert lib.moe_layer_forward(ctypes.byref(bad), *([256] * 18), size, None) == 2
+    assert B.moe_status_string(2) == "unsupported configuration"
+
+
+def test_product_path_refuses_to_run_without_cuda(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    with pytest.raises(B.MoEError):
+        B.moe_route(B.params(W.TINY), None, None, None, None, None, None, None, 0, 0)
+
+
+def test_binding_argument_counts_match_header(lib):
+    src = open(os.path.join(ROOT, "include", "moe.h"), encoding="utf-8").read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    for name, params in re.findall(r"\b(moe_[a-z0-9_]+)\s*\(([^)]*)\)\s*;", src):
+        n = 0 if params.strip() in ("", "void") else params.count(",") + 1
+        assert len(B._SIGS[name][1]) == n, (name, n, len(B._SIGS[name][1]))

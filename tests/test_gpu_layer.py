@@ -1,0 +1,102 @@
+"""Whole-layer parity: moe_layer_forward through the C ABI against the fp64 oracle.
+
+Small workloads keep the shapes' features (routing rules, several M/N/K tiles, ragged
+buckets) at sizes the oracle finishes in seconds and are compared on every element.
+The full workloads run in the configuration the benchmark times and are compared on the
+whole routing decision and permutation, plus sampled output rows.
+"""
+import numpy as np
+import pytest
+import torch
+
+from mixture_experts_ffn_08_b200 import binding as B
+from mixture_experts_ffn_08_b200 import inputs, workloads as W
+from oracle import moe_oracle as o
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    "tiny": W.TINY,
+    "mixtral_small": W.MIXTRAL_PREFILL.with_(name="mixtral_small", T=1000, H=512, I=384),
+    "dsv3_small": W.DSV3_PREFILL.with_(name="dsv3_small", T=200, H=512, I=256, E=32, I_shared=256),
+    "dsv3_decode_small": W.DSV3_DECODE.with_(name="dsv3_decode_small", T=16, H=512, I=256, E=32,
+                                             I_shared=256),
+    "one_token": W.MIXTRAL_PREFILL.with_(name="one_token", T=1, H=256, I=128, E=4, K=2),
+    "dense_like": W.TINY.with_(name="dense_like", T=300, E=1, K=1),
+}
+
+
+def _oracle_full(d, wl, gpu_ids):
+    x = P.x_f64(d, wl)
+    s = o.scores(o.router_logits(x, P.f64(d["w_r"])), wl.score_fn)
+    bias = P.f64(d["bias"]) if d["bias"] is not None else None
+    return x, s, bias
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_layer_small_all_elements(name):
+    wl = SMALL[name]
+    d = inputs.make_inputs(wl, seed=0, device="cuda")
+    r = P.run_layer(wl, d)
+    assert B.moe_get_device_status(r["ws"]) == 0
+    gpu_ids = r["ids"].cpu().numpy()
+    x, s, bias = _oracle_full(d, wl, gpu_ids)
+    _, w_or = P.check_routing(gpu_ids, r["w"].cpu().numpy(), s, bias, wl)
+    np.testing.assert_array_equal(r["counts"].cpu().numpy(), np.bincount(gpu_ids.ravel(), minlength=wl.E))
+    ref = o.forward_given_routing(x, gpu_ids, w_or, P.expert_weights_fn(d, wl), wl.E,
+                                  P.shared_weights(d, wl), quantize_h=wl.dtype == W.DTYPE_FP8)
+    P.check_close(P.f64(r["out"]), ref, P.BF16_MAX_TOL, name)
+
+
+def test_layer_is_deterministic():
+    wl = SMALL["dsv3_small"]
+    d = inputs.make_inputs(wl, seed=1, device="cuda")
+    first = P.run_layer(wl, d)
+    for _ in range(5):
+        again = P.run_layer(wl, d, ws=first["ws"])
+        assert torch.equal(again["out"], first["out"])
+        assert torch.equal(again["ids"], first["ids"])
+
+
+FULL = ["mixtral_prefill", "dsv3_prefill", "dsv3_decode"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_layer_full_size_sampled(name):
+    wl = W.ALL[name]
+    d = inputs.make_inputs(wl, seed=0, device="cuda")
+    r = P.run_layer(wl, d)
+    assert B.moe_get_device_status(r["ws"]) == 0
+    gpu_ids = r["ids"].cpu().numpy()
+    x, s, bias = _oracle_full(d, wl, gpu_ids)
+    n_mism, w_or = P.check_routing(gpu_ids, r["w"].cpu().numpy(), s, bias, wl)
+    assert n_mism <= max(2, wl.T // 1000), f"{n_mism} near-tie tokens"
+    counts = r["counts"].cpu().numpy()
+    assert counts.sum() == wl.T * wl.K
+    np.testing.assert_array_equal(counts, np.bincount(gpu_ids.ravel(), minlength=wl.E))
+    rng = np.random.default_rng(0)
+    n_sample = 12 if wl.E <= 8 else 4
+    toks = np.sort(rng.choice(wl.T, size=n_sample, replace=False))
+    ref = o.forward_given_routing(x[toks], gpu_ids[toks], w_or[toks], P.expert_weights_fn(d, wl),
+                                  wl.E, P.shared_weights(d, wl) if wl.I_shared else None)
+    got = P.f64(r["out"][torch.as_tensor(toks, device="cuda")])
+    P.check_close(got, ref, P.BF16_MAX_TOL, name)
+    del d, r
+    torch.cuda.empty_cache()
+
+
+def test_host_entry_point_matches_device_entry_point():
+    wl = SMALL["dsv3_small"]
+    d = inputs.make_inputs(wl, seed=2, device="cuda")
+    r = P.run_layer(wl, d)
+    p = B.params(wl)
+    a = P.device_inputs_ptrs(d, wl)
+    x_host = d["x"].cpu().pin_memory()
+    out_host = torch.empty((wl.T, wl.H), dtype=torch.bfloat16).pin_memory()
+    ws = r["ws"]
+    B.check(B.moe_layer_forward_host(p, x_host, None, a["w_r"], a["bias"], a["w_gate"], a["w_up"],
+                                     a["w_down"], None, None, None, a["ws_gate"], a["ws_up"],
+                                     a["ws_down"], out_host, ws, ws.numel()))
+    torch.cuda.synchronize()
+    assert torch.equal(out_host, r["out"].cpu())
