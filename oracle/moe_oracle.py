@@ -33,11 +33,13 @@ Readings where the pages are silent (each also listed in the design notes):
   - Each expert's rows start at a multiple of `block_m`; pad rows carry no pair.
   - Renormalise first, then multiply by routed_scale; the shared expert is added with
     weight 1.
+  - The SwiGLU output h is an activation and is stored in the workload's activation
+    format before the down projection, as the Mega MoE pipeline does with its
+    "SwiGLU / FP8 Cast" stage (MoE optimisation blog, §5.1): bf16 (round to nearest
+    even) for the bf16 workloads, whose weights and activations are bf16; e4m3 with
+    one power-of-two scale per row and 128 columns for the FP8 workload.
   - FP8 workload: e4m3 (max 448, round to nearest even, saturating); one
-    power-of-two scale per 1x128 activation block and per 128x128 weight block;
-    the SwiGLU output h is re-quantised per row and 128 columns before the down
-    projection ("SwiGLU / FP8 Cast" stage of the Mega MoE pipeline on the MoE
-    optimisation blog, §5.1).
+    power-of-two scale per 1x128 activation block and per 128x128 weight block.
   - No residual is added; the layer returns routed + shared only.
 
 Parity status: routed_scale and group_topn = 2 are not fixed by any worked example on
@@ -113,6 +115,25 @@ def quantize_rows_1x128(h) -> np.ndarray:
     b = h.reshape(R, C // QBLOCK, QBLOCK)
     s = pow2_scale(np.abs(b).max(axis=2))
     return (quantize_e4m3(b / s[:, :, None]) * s[:, :, None]).reshape(R, C)
+
+
+def round_bf16(v) -> np.ndarray:
+    """Nearest bfloat16 value (8 significant bits, ties to even) of each element, as
+    float64.  Values here stay far inside bf16's normal range."""
+    v = np.asarray(v, np.float64)
+    m, e = np.frexp(v)                         # v = m * 2^e, |m| in [0.5, 1)
+    return np.ldexp(np.round(np.ldexp(m, 8)), e - 8)   # np.round: half to even
+
+
+def store_activation(h, h_format):
+    """h in the activation format of the layer: None (exact), "bf16" or "e4m3"."""
+    if h_format is None:
+        return np.asarray(h, np.float64)
+    if h_format == "bf16":
+        return round_bf16(h)
+    if h_format == "e4m3":
+        return quantize_rows_1x128(h)
+    raise ValueError(h_format)
 
 
 # ----------------------------------------------------------------------------------
@@ -220,18 +241,17 @@ def silu(g):
     return g / (1.0 + np.exp(-g))
 
 
-def swiglu_ffn(xr, wg, wu, wd, quantize_h: bool = False):
-    """W_down (SiLU(W_gate x) * W_up x) for each row of xr [n, H]; weights [out, in]."""
+def swiglu_ffn(xr, wg, wu, wd, h_format=None):
+    """W_down (SiLU(W_gate x) * W_up x) for each row of xr [n, H]; weights [out, in].
+    h_format: format h is stored in between the two projections (see store_activation)."""
     xr = np.asarray(xr, np.float64)
     g = xr @ np.asarray(wg, np.float64).T
     u = xr @ np.asarray(wu, np.float64).T
-    h = silu(g) * u
-    if quantize_h:
-        h = quantize_rows_1x128(h)
+    h = store_activation(silu(g) * u, h_format)
     return h @ np.asarray(wd, np.float64).T
 
 
-def expert_outputs(x, ids, expert_weights, E: int, block_m: int, quantize_h: bool = False):
+def expert_outputs(x, ids, expert_weights, E: int, block_m: int, h_format=None):
     """y_perm [P_pad, H]: the output of every pair's expert on its token, laid out in
     the bucketed row order of `permute` (pad rows are zero).  `expert_weights(e)`
     returns (W_gate[e], W_up[e], W_down[e]) as arrays [I,H], [I,H], [H,I]."""
@@ -246,7 +266,7 @@ def expert_outputs(x, ids, expert_weights, E: int, block_m: int, quantize_h: boo
         rows = np.arange(offsets[e], offsets[e] + n)
         toks = pair_of_row[rows] // K
         wg, wu, wd = expert_weights(e)
-        y[rows] = swiglu_ffn(x[toks], wg, wu, wd, quantize_h)
+        y[rows] = swiglu_ffn(x[toks], wg, wu, wd, h_format)
     return y, row_of_pair
 
 
@@ -265,17 +285,24 @@ def combine(y_perm, row_of_pair, w, y_shared=None) -> np.ndarray:
 
 
 def forward_given_routing(x, ids, w, expert_weights, E: int, shared=None,
-                          quantize_h: bool = False, block_m: int = 1):
+                          h_format=None, block_m: int = 1):
     """Layer output [T, H] for a given routing decision (ids, w).  `shared` is
     (W_gate, W_up, W_down) of the shared expert or None."""
-    y_perm, row_of_pair = expert_outputs(x, ids, expert_weights, E, block_m, quantize_h)
-    y_sh = swiglu_ffn(x, *shared) if shared is not None else None
+    y_perm, row_of_pair = expert_outputs(x, ids, expert_weights, E, block_m, h_format)
+    y_sh = swiglu_ffn(x, *shared, h_format=h_format) if shared is not None else None
     return combine(y_perm, row_of_pair, w, y_sh)
 
 
-def layer_forward(x, w_r, bias, expert_weights, wl, shared=None):
-    """Route, then run the chosen experts and combine.  Returns (out, ids, w, s)."""
+def activation_format(dtype: int):
+    """Storage format of h for a workload dtype (0 = bf16, 1 = FP8 e4m3)."""
+    return "e4m3" if dtype == 1 else "bf16"
+
+
+def layer_forward(x, w_r, bias, expert_weights, wl, shared=None, h_format="auto"):
+    """Route, then run the chosen experts and combine.  Returns (out, ids, w, s).
+    h_format "auto" stores h in the workload's activation format."""
     ids, w, s = route(x, w_r, bias, wl)
-    out = forward_given_routing(x, ids, w, expert_weights, wl.E, shared,
-                                quantize_h=(wl.dtype == 1))
+    if h_format == "auto":
+        h_format = activation_format(wl.dtype)
+    out = forward_given_routing(x, ids, w, expert_weights, wl.E, shared, h_format=h_format)
     return out, ids, w, s

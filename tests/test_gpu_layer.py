@@ -45,7 +45,7 @@ def test_layer_small_all_elements(name):
     _, w_or = P.check_routing(gpu_ids, r["w"].cpu().numpy(), s, bias, wl)
     np.testing.assert_array_equal(r["counts"].cpu().numpy(), np.bincount(gpu_ids.ravel(), minlength=wl.E))
     ref = o.forward_given_routing(x, gpu_ids, w_or, P.expert_weights_fn(d, wl), wl.E,
-                                  P.shared_weights(d, wl), quantize_h=wl.dtype == W.DTYPE_FP8)
+                                  P.shared_weights(d, wl), h_format=o.activation_format(wl.dtype))
     P.check_close(P.f64(r["out"]), ref, P.BF16_MAX_TOL, name)
 
 
@@ -79,7 +79,8 @@ def test_layer_full_size_sampled(name):
     n_sample = 12 if wl.E <= 8 else 4
     toks = np.sort(rng.choice(wl.T, size=n_sample, replace=False))
     ref = o.forward_given_routing(x[toks], gpu_ids[toks], w_or[toks], P.expert_weights_fn(d, wl),
-                                  wl.E, P.shared_weights(d, wl) if wl.I_shared else None)
+                                  wl.E, P.shared_weights(d, wl) if wl.I_shared else None,
+                                  h_format=o.activation_format(wl.dtype))
     got = P.f64(r["out"][torch.as_tensor(toks, device="cuda")])
     P.check_close(got, ref, P.BF16_MAX_TOL, name)
     del d, r

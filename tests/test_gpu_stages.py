@@ -165,7 +165,7 @@ def test_expert_ffn_grouped_gemm(E, K, T, H, I):
     rows = B.moe_max_padded_rows(p)
     offs = torch.as_tensor(r["offs"], device="cuda")
     counts = torch.as_tensor(r["counts"], device="cuda")
-    ref, _ = o.expert_outputs(P.f64(d["x"]), ids, P.expert_weights_fn(d, wl), E, BM)
+    ref, _ = o.expert_outputs(P.f64(d["x"]), ids, P.expert_weights_fn(d, wl), E, BM, h_format="bf16")
     total = r["offs"][E]
     real = r["por"][:total] >= 0
     # with counts: pad rows are left untouched; without: they are computed (zero input -> 0)
@@ -191,7 +191,7 @@ def test_shared_expert_dense_ffn_ragged_T():
     y = torch.empty((wl.T, wl.H), dtype=torch.float32, device="cuda")
     B.check(B.moe_shared_expert_ffn(p, d["x"], d["ws_gate"], d["ws_up"], d["ws_down"], y, ws, ws.numel()))
     torch.cuda.synchronize()
-    ref = o.swiglu_ffn(P.f64(d["x"]), *P.shared_weights(d, wl))
+    ref = o.swiglu_ffn(P.f64(d["x"]), *P.shared_weights(d, wl), h_format="bf16")
     P.check_close(P.f64(y), ref, P.BF16_MAX_TOL, "shared")
 
 

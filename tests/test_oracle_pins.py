@@ -257,7 +257,8 @@ def test_layer_equals_dense_mixture_masked_to_topk(case):
                 routed_scale=2.5, dtype=0)
         bias = rng.normal(size=E) * 0.1
         shared = (rng.normal(size=(4, H)) * .3, rng.normal(size=(4, H)) * .3, rng.normal(size=(H, 4)) * .3)
-    out, ids, w, s = o.layer_forward(x, w_r, bias, lambda e: (Wg[e], Wu[e], Wd[e]), wl, shared)
+    out, ids, w, s = o.layer_forward(x, w_r, bias, lambda e: (Wg[e], Wu[e], Wd[e]), wl, shared,
+                                     h_format=None)
     for t in range(T):
         dense = np.zeros(H)
         for e in range(E):
@@ -328,3 +329,49 @@ def test_rowwise_requant_error_bound():
     # half a unit in the last place of e4m3 (3 mantissa bits), or of the subnormal step
     bound = np.maximum(np.abs(b) * 2.0 ** -4, s * 2.0 ** -10)
     assert (err <= bound + 1e-300).all()
+
+
+# ------------------------------------------------------------------ bf16 activations
+def test_round_bf16_matches_torch_on_fp32_values():
+    rng = np.random.default_rng(12)
+    v = (rng.normal(size=200000) * np.exp(rng.normal(size=200000) * 3)).astype(np.float32)
+    ref = torch.from_numpy(v).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(o.round_bf16(v.astype(np.float64)), ref)
+
+
+def test_round_bf16_nearest_even_by_grid():
+    rng = np.random.default_rng(13)
+    v = np.abs(rng.normal(size=3000)) * 10.0 ** rng.integers(-3, 4, 3000)
+    for vi, qi in zip(v, o.round_bf16(v)):
+        k = np.floor(np.log2(vi))
+        ulp = 2.0 ** (k - 7)                      # 8 significant bits
+        lo = np.floor(vi / ulp) * ulp
+        hi = lo + ulp
+        if vi - lo < hi - vi:
+            want = lo
+        elif vi - lo > hi - vi:
+            want = hi
+        else:
+            want = lo if int(round(lo / ulp)) % 2 == 0 else hi
+        assert qi == want, (vi, qi, want)
+    # exact midpoints between neighbours go to the even neighbour
+    assert o.round_bf16(1.0 + 2.0 ** -8) == 1.0
+    assert o.round_bf16(1.0 + 3 * 2.0 ** -8) == 1.0 + 2.0 ** -6
+    assert o.round_bf16(-(1.0 + 2.0 ** -8)) == -1.0
+
+
+def test_store_activation_formats():
+    h = np.random.default_rng(14).normal(size=(3, 256))
+    np.testing.assert_array_equal(o.store_activation(h, None), h)
+    np.testing.assert_array_equal(o.store_activation(h, "bf16"), o.round_bf16(h))
+    np.testing.assert_array_equal(o.store_activation(h, "e4m3"), o.quantize_rows_1x128(h))
+    # SwiGLU with h stored in bf16 equals torch's pieces with an explicit bf16 round trip
+    rng = np.random.default_rng(15)
+    x, wg, wu, wd = rng.normal(size=(4, 16)), rng.normal(size=(8, 16)) * .3, rng.normal(size=(8, 16)) * .3, rng.normal(size=(16, 8)) * .3
+    g = torch.from_numpy(x) @ torch.from_numpy(wg).T
+    u = torch.from_numpy(x) @ torch.from_numpy(wu).T
+    h = (F.silu(g) * u).float().to(torch.bfloat16).double()
+    want = (h @ torch.from_numpy(wd).T).numpy()
+    got = o.swiglu_ffn(x, wg, wu, wd, h_format="bf16")
+    # torch rounds through fp32 first; both are within one bf16 rounding of each other
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
