@@ -39,6 +39,29 @@ METRIC = "MoE layer tokens/s and grouped-GEMM TFLOP/s (or HBM GB/s) vs B200 roof
 FLUSH_BYTES = 512 << 20
 
 
+GEMM_SOURCES = ("csrc/tc_gemm.cuh", "csrc/common.cuh", "csrc/gemm.cu")
+
+
+def _profiled_traffic(workload):
+    """DRAM bytes per launch of the gate/up kernel from the committed ncu summary of this
+    workload, or None if there is none or the kernel sources changed since it was taken."""
+    import hashlib
+    import re
+    path = os.path.join(ROOT, "profiles", f"gateup_swiglu_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    txt = open(path, encoding="utf-8").read()
+    m_t = re.search(r"^traffic_bytes_per_launch:\s*(\d+)", txt, re.M)
+    m_h = re.search(r"^kernel_source_sha256:\s*([0-9a-f]+)", txt, re.M)
+    if not (m_t and m_h):
+        return None
+    h = hashlib.sha256()
+    for f in GEMM_SOURCES:
+        with open(os.path.join(ROOT, "mixture_experts_ffn_08_b200", f), "rb") as fh:
+            h.update(fh.read())
+    return int(m_t.group(1)) if h.hexdigest() == m_h.group(1) else None
+
+
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -252,7 +275,8 @@ def run_ours(args):
     achieved = flops_gateup / (dom_avg / 1e3) / 1e12 if dom_avg else None
     roofline = {"kernel": "gateup_swiglu (grouped GEMM, fused SwiGLU)", "bound": "tensor",
                 "achieved": achieved, "peak": bf16_peak, "unit": "TFLOP/s",
-                "frac": achieved / bf16_peak if achieved else None, "traffic": None,
+                "frac": achieved / bf16_peak if achieved else None,
+                "traffic": _profiled_traffic(wl.name),
                 "peak_kind": f"{peak_kind} bf16 burst", "launches_timed": len(dom_ms),
                 "avg_ms": dom_avg, "algorithmic_flops_per_launch": flops_gateup}
 
@@ -351,7 +375,7 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="mixtral_prefill", choices=sorted(W.ALL))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
