@@ -127,6 +127,26 @@ moe_status_t moe_permute(const moe_params_t* p, const int32_t* topk_ids, const v
                          int32_t* row_of_pair, int32_t* pair_of_row, void* x_perm,
                          float* x_perm_scale, void* ws, size_t ws_bytes, void* stream);
 
+/* Allocation-free variant of moe_permute.  The pages have no counterpart: this entry
+ * point exists for callers that cannot give the library device memory of its own
+ * (plug-ins inside a host framework that owns all device memory and offers no scratch
+ * hook; serving loops where a cudaMalloc or allocator round trip is not allowed).  It
+ * takes the same inputs and outputs as moe_permute but no workspace: the per-chunk
+ * expert histogram lives in a fixed 1 MiB file-scope device array that every GPU using
+ * the library holds until the process exits.
+ *   - Limit: ceil(T*K/256) * E <= 262144, else MOE_ERR_UNSUPPORTED (nothing launched).
+ *   - device_status: optional device int32 the caller has zeroed; MOE_DEV_BAD_EXPERT_ID
+ *     is OR-ed into it (NULL: not reported; bad pairs still get row_of_pair = -1).
+ *   - All calls share the one array: calls that overlap on the GPU (other streams,
+ *     other host threads on the same device) race.  Serialise them on one stream.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress with that device current); make that first call before
+ *     any stream capture.  No call allocates or frees device memory. */
+moe_status_t moe_permute_noalloc(const moe_params_t* p, const int32_t* topk_ids, const void* x,
+                                 const float* x_scale, int32_t* counts, int32_t* offsets_padded,
+                                 int32_t* row_of_pair, int32_t* pair_of_row, void* x_perm,
+                                 float* x_perm_scale, int32_t* device_status, void* stream);
+
 /* ---------------------------------------------------------------------------------- */
 /* Stage 3 — expert FFN on the bucketed rows (routing primer §5.2; M-grouped GEMM as    */
 /* in the "MoE" chapter index §1, grouped GEMM entry).                                  */

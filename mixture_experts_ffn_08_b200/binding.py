@@ -58,6 +58,7 @@ _SIGS = {
     "moe_max_padded_rows": (ctypes.c_int64, [_PP]),
     "moe_route": (ctypes.c_int, [_PP, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_permute": (ctypes.c_int, [_PP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_permute_noalloc": (ctypes.c_int, [_PP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_expert_ffn": (ctypes.c_int, [_PP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                       ctypes.c_size_t, _P]),
     "moe_shared_expert_ffn": (ctypes.c_int, [_PP, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
@@ -147,6 +148,16 @@ def moe_permute(p, topk_ids, x, x_scale, counts, offsets_padded, row_of_pair, pa
     return lib().moe_permute(ctypes.byref(p), _ptr(topk_ids), _ptr(x), _ptr(x_scale), _ptr(counts),
                              _ptr(offsets_padded), _ptr(row_of_pair), _ptr(pair_of_row),
                              _ptr(x_perm), _ptr(x_perm_scale), _ptr(ws), ws_bytes, _stream(stream))
+
+
+def moe_permute_noalloc(p, topk_ids, x, x_scale, counts, offsets_padded, row_of_pair,
+                        pair_of_row, x_perm, x_perm_scale, device_status, stream=None) -> int:
+    """moe_permute without a workspace, for callers that cannot allocate device memory
+    for the library; its scratch is a fixed device array inside the library."""
+    return lib().moe_permute_noalloc(ctypes.byref(p), _ptr(topk_ids), _ptr(x), _ptr(x_scale),
+                                     _ptr(counts), _ptr(offsets_padded), _ptr(row_of_pair),
+                                     _ptr(pair_of_row), _ptr(x_perm), _ptr(x_perm_scale),
+                                     _ptr(device_status), _stream(stream))
 
 
 def moe_expert_ffn(p, x_perm, x_perm_scale, offsets_padded, counts, w_gate, w_up, w_down,
