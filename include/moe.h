@@ -226,7 +226,7 @@ enum {
   MOE_K_ROUTER_GEMM = 0, MOE_K_TOPK = 1, MOE_K_PERM_COUNT = 2, MOE_K_PERM_SCAN = 3,
   MOE_K_PERM_RANK = 4, MOE_K_PERM_GATHER = 5, MOE_K_GATEUP = 6, MOE_K_DOWN = 7,
   MOE_K_SHARED_GATEUP = 8, MOE_K_SHARED_DOWN = 9, MOE_K_COMBINE = 10, MOE_K_DEQUANT_X = 11,
-  MOE_K_COUNT = 12
+  MOE_K_SCALE_ATOMS = 12, MOE_K_COUNT = 13
 };
 
 /* Tracing: while enabled, every launch of a kernel whose bit (1u << id) is in

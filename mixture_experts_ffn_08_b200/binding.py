@@ -27,8 +27,10 @@ BLOCK_M = 128
 # Kernel ids for tracing (include/moe.h).
 K_ROUTER_GEMM, K_TOPK, K_PERM_COUNT, K_PERM_SCAN, K_PERM_RANK, K_PERM_GATHER = range(6)
 K_GATEUP, K_DOWN, K_SHARED_GATEUP, K_SHARED_DOWN, K_COMBINE, K_DEQUANT_X = range(6, 12)
+K_SCALE_ATOMS = 12
 KERNEL_NAMES = ["router_gemm", "topk", "perm_count", "perm_scan", "perm_rank", "perm_gather",
-                "gateup_swiglu", "down", "shared_gateup", "shared_down", "combine", "dequant_x"]
+                "gateup_swiglu", "down", "shared_gateup", "shared_down", "combine", "dequant_x",
+                "scale_atoms"]
 
 
 class MoEError(RuntimeError):

@@ -64,6 +64,7 @@ size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 struct Layout {
   size_t status, logits, xb, ids, w, counts, offsets, row_of_pair, pair_of_row, chunk_counts;
   size_t x_perm, x_perm_scale, h, y_perm, h_sh, y_sh, total;
+  size_t x_atoms, h_atoms, wg_atoms, wu_atoms, wd_atoms;
   size_t x_stage, x_scale_stage, out_stage, total_host;
   long long max_rows;
 };
@@ -75,6 +76,7 @@ Layout layout(const moe_params_t* p) {
   const long long T = p->T, H = p->H, I = p->I, E = p->E, K = p->K;
   const long long P = T * K;
   const long long rows = P + E * (kBlockM - 1);
+  const long long rows_t = (rows + kBlockM - 1) / kBlockM * kBlockM;  // whole M-tiles
   const long long nchunks = (P + kPermChunk - 1) / kPermChunk;
   const size_t xelem = is_fp8(p) ? 1 : 2;
   size_t o = 0;
@@ -92,10 +94,16 @@ Layout layout(const moe_params_t* p) {
   L.chunk_counts = take((nchunks > 0 ? nchunks : 1) * E * 4);
   L.x_perm = take(rows * H * xelem);
   L.x_perm_scale = take(is_fp8(p) ? rows * (H / 128) * 4 : 0);
-  L.h = take(rows * I * 2);
+  L.h = take(rows_t * I * 2);
   L.y_perm = take(rows * H * 4);
   L.h_sh = take(T * static_cast<long long>(p->I_shared) * 2);
   L.y_sh = take(p->I_shared > 0 ? T * H * 4 : 0);
+  const bool f8 = is_fp8(p);
+  L.x_atoms = take(f8 ? rows_t * (H / 128) * 4 : 0);
+  L.h_atoms = take(f8 ? rows_t * (I / 128) * 4 : 0);
+  L.wg_atoms = take(f8 ? E * (I / 128) * (H / 128) * 512 : 0);
+  L.wu_atoms = take(f8 ? E * (I / 128) * (H / 128) * 512 : 0);
+  L.wd_atoms = take(f8 ? E * (H / 128) * (I / 128) * 512 : 0);
   L.total = o;
   L.x_stage = take(T * H * xelem);
   L.x_scale_stage = take(is_fp8(p) ? T * (H / 128) * 4 : 0);
@@ -125,6 +133,7 @@ moe_status_t validate(const moe_params_t* p) {
   if (p->I_shared < 0) return MOE_ERR_INVALID_ARG;
   if (p->H % 128 != 0 || p->I % 128 != 0 || p->I_shared % 128 != 0) return MOE_ERR_UNSUPPORTED;
   if (p->block_m != 0 && p->block_m != kBlockM) return MOE_ERR_UNSUPPORTED;
+  if (p->dtype == MOE_DTYPE_FP8_E4M3 && p->I_shared > 0) return MOE_ERR_UNSUPPORTED;
   const long long rows = static_cast<long long>(p->T) * p->K + static_cast<long long>(p->E) * (kBlockM - 1);
   if (rows >= (1LL << 31) / 2) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
@@ -173,10 +182,31 @@ moe_status_t do_permute(const moe_params_t* p, const int32_t* ids, const void* x
                                     at<int32_t>(ws, L.chunk_counts), at<int32_t>(ws, L.status), st));
 }
 
+moe_status_t do_expert_ffn_fp8(const moe_params_t* p, const void* x_perm, const float* x_perm_scale,
+                               const int32_t* offsets, const int32_t* counts, const void* w_gate,
+                               const void* w_up, const void* w_down, const float* wgs,
+                               const float* wus, const float* wds, float* y_perm, void* ws,
+                               cudaStream_t st) {
+  const Layout L = layout(p);
+  int32_t* status = at<int32_t>(ws, L.status);
+  const long long nb_gu = static_cast<long long>(p->E) * (p->I / 128) * (p->H / 128);
+  MOE_CUDA(launch_sf_blocks_to_atoms(wgs, nb_gu, at<uint8_t>(ws, L.wg_atoms), st));
+  MOE_CUDA(launch_sf_blocks_to_atoms(wus, nb_gu, at<uint8_t>(ws, L.wu_atoms), st));
+  MOE_CUDA(launch_sf_blocks_to_atoms(wds, nb_gu, at<uint8_t>(ws, L.wd_atoms), st));
+  MOE_CUDA(launch_sf_rows_to_atoms(x_perm_scale, p->H / 128, offsets, p->E, L.max_rows,
+                                   at<uint8_t>(ws, L.x_atoms), st));
+  void* h = at<void>(ws, L.h);
+  MOE_CUDA(gemm_gateup_swiglu_fp8(x_perm, at<uint8_t>(ws, L.x_atoms), L.max_rows, offsets, counts, p->E,
+                                  w_gate, w_up, at<uint8_t>(ws, L.wg_atoms), at<uint8_t>(ws, L.wu_atoms),
+                                  p->I, p->H, h, at<uint8_t>(ws, L.h_atoms), status, st));
+  MOE_CUDA(gemm_down_fp8(h, at<uint8_t>(ws, L.h_atoms), L.max_rows, offsets, counts, p->E, w_down,
+                         at<uint8_t>(ws, L.wd_atoms), p->H, p->I, y_perm, status, st));
+  return MOE_OK;
+}
+
 moe_status_t do_expert_ffn(const moe_params_t* p, const void* x_perm, const int32_t* offsets,
                            const int32_t* counts, const void* w_gate, const void* w_up,
                            const void* w_down, float* y_perm, void* ws, cudaStream_t st) {
-  if (is_fp8(p)) return MOE_ERR_UNSUPPORTED;
   const Layout L = layout(p);
   int32_t* status = at<int32_t>(ws, L.status);
   void* h = at<void>(ws, L.h);
@@ -201,8 +231,9 @@ moe_status_t do_shared(const moe_params_t* p, const void* x, const void* wsg, co
 
 moe_status_t do_layer(const moe_params_t* p, const void* x, const float* x_scale, const void* w_r,
                       const float* bias, const void* w_gate, const void* w_up, const void* w_down,
-                      const void* wsg, const void* wsu, const void* wsd, void* out, int32_t* ids_out,
-                      float* w_out, int32_t* counts_out, void* ws, cudaStream_t st) {
+                      const float* wgs, const float* wus, const float* wds, const void* wsg,
+                      const void* wsu, const void* wsd, void* out, int32_t* ids_out, float* w_out,
+                      int32_t* counts_out, void* ws, cudaStream_t st) {
   const Layout L = layout(p);
   if (p->T == 0) return MOE_OK;
   int32_t* ids = ids_out ? ids_out : at<int32_t>(ws, L.ids);
@@ -214,7 +245,11 @@ moe_status_t do_layer(const moe_params_t* p, const void* x, const float* x_scale
   MOE_TRY(do_route(p, x, x_scale, w_r, bias, ids, w, ws, st));
   MOE_TRY(do_permute(p, ids, x, x_scale, counts, offsets, rop, at<int32_t>(ws, L.pair_of_row),
                      at<void>(ws, L.x_perm), at<float>(ws, L.x_perm_scale), ws, st));
-  MOE_TRY(do_expert_ffn(p, at<void>(ws, L.x_perm), offsets, counts, w_gate, w_up, w_down, y_perm, ws, st));
+  if (is_fp8(p))
+    MOE_TRY(do_expert_ffn_fp8(p, at<void>(ws, L.x_perm), at<float>(ws, L.x_perm_scale), offsets, counts,
+                              w_gate, w_up, w_down, wgs, wus, wds, y_perm, ws, st));
+  else
+    MOE_TRY(do_expert_ffn(p, at<void>(ws, L.x_perm), offsets, counts, w_gate, w_up, w_down, y_perm, ws, st));
   float* y_sh = nullptr;
   if (p->I_shared > 0) {
     y_sh = at<float>(ws, L.y_sh);
@@ -289,13 +324,18 @@ moe_status_t moe_expert_ffn(const moe_params_t* p, const void* x_perm, const flo
                             const void* w_up, const void* w_down, const float* w_gate_scale,
                             const float* w_up_scale, const float* w_down_scale, float* y_perm,
                             void* ws, size_t ws_bytes, void* stream) {
-  (void)x_perm_scale; (void)w_gate_scale; (void)w_up_scale; (void)w_down_scale;
   MOE_TRY(validate(p));
   MOE_TRY(check_ws(p, ws, ws_bytes, false));
   if (!x_perm || !offsets_padded || !w_gate || !w_up || !w_down || !y_perm) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x_perm) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down) || !aligned16(y_perm))
     return MOE_ERR_INVALID_ARG;
+  if (is_fp8(p) && (!x_perm_scale || !w_gate_scale || !w_up_scale || !w_down_scale))
+    return MOE_ERR_INVALID_ARG;
   if (p->T == 0) return MOE_OK;
+  if (is_fp8(p))
+    return do_expert_ffn_fp8(p, x_perm, x_perm_scale, offsets_padded, counts, w_gate, w_up, w_down,
+                             w_gate_scale, w_up_scale, w_down_scale, y_perm, ws,
+                             static_cast<cudaStream_t>(stream));
   return do_expert_ffn(p, x_perm, offsets_padded, counts, w_gate, w_up, w_down, y_perm, ws,
                        static_cast<cudaStream_t>(stream));
 }
@@ -328,12 +368,12 @@ moe_status_t moe_layer_forward(const moe_params_t* p, const void* x, const float
                                const void* ws_gate, const void* ws_up, const void* ws_down, void* out,
                                int32_t* topk_ids_out, float* topk_w_out, int32_t* counts_out, void* ws,
                                size_t ws_bytes, void* stream) {
-  (void)w_gate_scale; (void)w_up_scale; (void)w_down_scale;
   MOE_TRY(validate(p));
   MOE_TRY(check_ws(p, ws, ws_bytes, false));
   MOE_TRY(check_layer_args(p, x, x_scale, w_r, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, out));
-  if (is_fp8(p)) return MOE_ERR_UNSUPPORTED;
-  return do_layer(p, x, x_scale, w_r, bias, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, out, topk_ids_out,
+  if (is_fp8(p) && (!w_gate_scale || !w_up_scale || !w_down_scale)) return MOE_ERR_INVALID_ARG;
+  return do_layer(p, x, x_scale, w_r, bias, w_gate, w_up, w_down, w_gate_scale, w_up_scale, w_down_scale,
+                  ws_gate, ws_up, ws_down, out, topk_ids_out,
                   topk_w_out, counts_out, ws, static_cast<cudaStream_t>(stream));
 }
 
@@ -356,7 +396,8 @@ moe_status_t moe_layer_forward_host(const moe_params_t* p, const void* x_host, c
   const size_t xbytes = static_cast<size_t>(p->T) * p->H * 2;
   if (p->T == 0) return MOE_OK;
   MOE_CUDA(cudaMemcpyAsync(x_dev, x_host, xbytes, cudaMemcpyHostToDevice, st));
-  MOE_TRY(do_layer(p, x_dev, nullptr, w_r, bias, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, out_dev,
+  MOE_TRY(do_layer(p, x_dev, nullptr, w_r, bias, w_gate, w_up, w_down, nullptr, nullptr, nullptr, ws_gate,
+                   ws_up, ws_down, out_dev,
                    nullptr, nullptr, nullptr, ws, st));
   MOE_CUDA(cudaMemcpyAsync(out_host, out_dev, static_cast<size_t>(p->T) * p->H * 2, cudaMemcpyDeviceToHost, st));
   return MOE_OK;
@@ -429,7 +470,7 @@ int32_t moe_layer_launch_count(const moe_params_t* p) {
   if (validate(p) != MOE_OK) return -1;
   if (p->T == 0) return 0;
   int n = 2;                                 // router GEMM, top-k
-  if (is_fp8(p)) n += 1;                     // dequantise x for the router
+  if (is_fp8(p)) n += 5;                     // dequantise x for the router, 4 scale-atom passes
   n += (p->T * p->K > 0) ? 4 : 2;            // count, scan, rank, gather
   n += 2;                                    // gate/up, down
   if (p->I_shared > 0) n += 2;               // shared gate/up, down

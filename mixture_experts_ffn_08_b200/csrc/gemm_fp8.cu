@@ -1,0 +1,158 @@
+// Host side of the block-scaled FP8 expert GEMMs, and the kernels that turn the layer's
+// fp32 power-of-two block scales into the 512-byte UE8M0 scale atoms the tensor core
+// reads (layout described in tc_gemm_fp8.cuh).
+#include <cudaTypedefs.h>
+
+#include "internal.h"
+#include "tc_gemm_fp8.cuh"
+
+namespace moe {
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn8() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// Row-major byte matrix [rows, cols], box of 128 columns (128 bytes) x box_rows rows,
+// 128-byte swizzle; out-of-range rows read as zero.
+bool make_tmap_u8(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  auto fn = encode_fn8();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <class Cfg>
+cudaError_t launch8(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                    const Fp8Params& fp, long long max_items, int kid, cudaStream_t st) {
+  auto kern = tc_gemm_fp8_kernel<Cfg>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
+  if (err != cudaSuccess) return err;
+  const long long sms = num_sms();
+  const int grid = static_cast<int>(max_items < sms ? (max_items > 0 ? max_items : 1) : sms);
+  trace_before(kid, st);
+  kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, st>>>(a, b0, b1, fp);
+  trace_after(kid, st);
+  return cudaGetLastError();
+}
+
+// UE8M0 byte of a power-of-two fp32 scale: its biased exponent field.
+__device__ __forceinline__ uint32_t ue8m0_of(float s) { return (__float_as_uint(s) >> 23) & 0xFFu; }
+
+// Per-row scales [rows, nk] (one per 128 columns) -> atoms [rows/128][nk][512], for the
+// rows of the buckets (offsets[G] of them).
+__global__ void sf_rows_to_atoms_kernel(const float* __restrict__ scales, int nk,
+                                        const int32_t* __restrict__ offsets, int G,
+                                        uint8_t* __restrict__ atoms) {
+  const long long n = static_cast<long long>(__ldg(offsets + G)) * nk;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long r = i / nk;
+    const int kb = static_cast<int>(i % nk);
+    const uint32_t word = ue8m0_of(__ldg(scales + i)) * 0x01010101u;
+    uint8_t* atom = atoms + ((r >> 7) * nk + kb) * 512;
+    *reinterpret_cast<uint32_t*>(atom + sf_atom_offset(static_cast<int>(r & 127))) = word;
+  }
+}
+
+// One scale per 128x128 weight block -> one atom (512 equal bytes) per block.
+__global__ void sf_blocks_to_atoms_kernel(const float* __restrict__ scales, long long nblocks,
+                                          uint8_t* __restrict__ atoms) {
+  const long long n = nblocks * 32;  // 32 x 16 bytes per atom
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x) {
+    const uint32_t w = ue8m0_of(__ldg(scales + (i >> 5))) * 0x01010101u;
+    reinterpret_cast<uint4*>(atoms)[i] = make_uint4(w, w, w, w);
+  }
+}
+
+long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
+
+}  // namespace
+
+cudaError_t launch_sf_rows_to_atoms(const float* scales, int nk, const int32_t* offsets, int G,
+                                    long long max_rows, uint8_t* atoms, cudaStream_t st) {
+  const long long n = max_rows * nk;
+  const int grid = static_cast<int>(cdiv(n, 256) < num_sms() * 8LL ? cdiv(n, 256) : num_sms() * 8LL);
+  trace_before(MOE_K_SCALE_ATOMS, st);
+  sf_rows_to_atoms_kernel<<<grid > 0 ? grid : 1, 256, 0, st>>>(scales, nk, offsets, G, atoms);
+  trace_after(MOE_K_SCALE_ATOMS, st);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sf_blocks_to_atoms(const float* scales, long long nblocks, uint8_t* atoms,
+                                      cudaStream_t st) {
+  const long long n = nblocks * 32;
+  const int grid = static_cast<int>(cdiv(n, 256) < num_sms() * 8LL ? cdiv(n, 256) : num_sms() * 8LL);
+  trace_before(MOE_K_SCALE_ATOMS, st);
+  sf_blocks_to_atoms_kernel<<<grid > 0 ? grid : 1, 256, 0, st>>>(scales, nblocks, atoms);
+  trace_after(MOE_K_SCALE_ATOMS, st);
+  return cudaGetLastError();
+}
+
+cudaError_t gemm_gateup_swiglu_fp8(const void* A, const uint8_t* a_atoms, int64_t a_rows,
+                                   const int32_t* offsets, const int32_t* counts, int G,
+                                   const void* w_gate, const void* w_up, const uint8_t* gate_atoms,
+                                   const uint8_t* up_atoms, int N, int K, void* h, uint8_t* h_atoms,
+                                   int32_t* status, cudaStream_t st) {
+  using Cfg = Fp8Cfg<256, EPI8_SWIGLU_Q, 4>;
+  CUtensorMap ta, tg, tu;
+  if (!make_tmap_u8(&ta, A, a_rows, K, 128) ||
+      !make_tmap_u8(&tg, w_gate, static_cast<uint64_t>(G) * N, K, 128) ||
+      !make_tmap_u8(&tu, w_up, static_cast<uint64_t>(G) * N, K, 128))
+    return cudaErrorInvalidValue;
+  Fp8Params fp{};
+  fp.offsets = offsets;
+  fp.counts = counts;
+  fp.G = G;
+  fp.K = K;
+  fp.N = N;
+  fp.sfa = a_atoms;
+  fp.sfb0 = gate_atoms;
+  fp.sfb1 = up_atoms;
+  fp.out = h;
+  fp.ldo = N;
+  fp.out_sf = h_atoms;
+  fp.status = status;
+  return launch8<Cfg>(ta, tg, tu, fp, cdiv(a_rows, 128) * cdiv(N, 128), MOE_K_GATEUP, st);
+}
+
+cudaError_t gemm_down_fp8(const void* A, const uint8_t* a_atoms, int64_t a_rows,
+                          const int32_t* offsets, const int32_t* counts, int G, const void* w,
+                          const uint8_t* w_atoms, int N, int K, float* y, int32_t* status,
+                          cudaStream_t st) {
+  using Cfg = Fp8Cfg<128, EPI8_F32, 5>;
+  CUtensorMap ta, tb;
+  if (!make_tmap_u8(&ta, A, a_rows, K, 128) || !make_tmap_u8(&tb, w, static_cast<uint64_t>(G) * N, K, 128))
+    return cudaErrorInvalidValue;
+  Fp8Params fp{};
+  fp.offsets = offsets;
+  fp.counts = counts;
+  fp.G = G;
+  fp.K = K;
+  fp.N = N;
+  fp.sfa = a_atoms;
+  fp.sfb0 = w_atoms;
+  fp.sfb1 = nullptr;
+  fp.out = y;
+  fp.ldo = N;
+  fp.out_sf = nullptr;
+  fp.status = status;
+  return launch8<Cfg>(ta, tb, tb, fp, cdiv(a_rows, 128) * cdiv(N, 128), MOE_K_DOWN, st);
+}
+
+}  // namespace moe

@@ -52,4 +52,22 @@ cudaError_t gemm_down(const void* A, int64_t a_rows, const int32_t* offsets,
                       const int32_t* counts, int G, int dense_rows, const void* w, int N, int K,
                       float* y, int32_t* status, int kid, cudaStream_t st);
 
+// ---------------------------------------------------------------- FP8 GEMMs (gemm_fp8.cu)
+// fp32 power-of-two scales -> 512-byte UE8M0 scale atoms (see tc_gemm_fp8.cuh).
+cudaError_t launch_sf_rows_to_atoms(const float* scales, int nk, const int32_t* offsets, int G,
+                                    long long max_rows, uint8_t* atoms, cudaStream_t st);
+cudaError_t launch_sf_blocks_to_atoms(const float* scales, long long nblocks, uint8_t* atoms,
+                                      cudaStream_t st);
+// h (e4m3 [rows, N] + scale atoms) = quant(SiLU(A Wg^T) * (A Wu^T)), block-scaled e4m3 GEMM.
+cudaError_t gemm_gateup_swiglu_fp8(const void* A, const uint8_t* a_atoms, int64_t a_rows,
+                                   const int32_t* offsets, const int32_t* counts, int G,
+                                   const void* w_gate, const void* w_up, const uint8_t* gate_atoms,
+                                   const uint8_t* up_atoms, int N, int K, void* h, uint8_t* h_atoms,
+                                   int32_t* status, cudaStream_t st);
+// y [rows, N] fp32 = A W^T, block-scaled e4m3 GEMM.
+cudaError_t gemm_down_fp8(const void* A, const uint8_t* a_atoms, int64_t a_rows,
+                          const int32_t* offsets, const int32_t* counts, int G, const void* w,
+                          const uint8_t* w_atoms, int N, int K, float* y, int32_t* status,
+                          cudaStream_t st);
+
 }  // namespace moe
