@@ -57,7 +57,7 @@ def test_sizes(lib):
         ws = B.moe_workspace_size(p)
         assert ws >= rows * wl.H * (1 if wl.dtype else 2) * 2
         assert B.moe_workspace_size_host(p) > ws
-        assert B.moe_layer_launch_count(p) == 9 + (2 if wl.I_shared else 0) + (1 if wl.dtype else 0)
+        assert B.moe_layer_launch_count(p) == 9 + (2 if wl.I_shared else 0) + (5 if wl.dtype else 0)
 
 
 @pytest.mark.parametrize("change", [dict(H=100), dict(I=200), dict(K=0), dict(E=2000),
