@@ -255,6 +255,18 @@ def run_ours(args):
     if status != 0:
         raise B.MoEError(f"device status {status:#x} after the timed steps")
 
+    # per-kernel breakdown: a few more steps, every kernel of the library bracketed by
+    # events (outside the timed region, so the events do not perturb the headline)
+    B.check(B.moe_trace_enable((1 << 13) - 1, 64 * 8))
+    for _ in range(3):
+        flush.fill_(0)
+        step()
+    breakdown = {}
+    for k, ms in B.moe_trace_collect():
+        breakdown.setdefault(B.KERNEL_NAMES[k], []).append(ms)
+    B.moe_trace_disable()
+    kernel_ms = {k: round(sum(v) / 3, 4) for k, v in breakdown.items()}
+
     counts_h = counts.cpu().numpy()
     P = wl.T * wl.K
     ms_total = float(sum(step_ms))
@@ -355,6 +367,7 @@ def run_ours(args):
         "clocks": clk,
         "gpu_launches": B.moe_layer_launch_count(p) * args.steps,
         "cpu_baseline": cpu,
+        "kernel_ms_per_step": kernel_ms,
         "expert_load": {"max": int(counts_h.max()), "min": int(counts_h.min()),
                         "mean": P / wl.E},
     }
