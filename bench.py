@@ -63,12 +63,16 @@ def _profiled_traffic(workload):
 
 
 def _peaks():
+    """(bf16 burst TFLOP/s, bf16 sustained TFLOP/s, HBM GB/s, kind)."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
         with open(path) as f:
             d = json.load(f)
-        return d["bf16_tflops"], d["hbm_gbs"], "measured"
-    return 1590.0, 6650.0, "fallback"
+        return d["bf16_tflops"], d.get("bf16_tflops_sustained", d["bf16_tflops"]), d["hbm_gbs"], "measured"
+    return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+FP8_OVER_BF16 = 2.0   # nominal dense e4m3 / bf16 tensor throughput (4.5 / 2.25 PFLOP/s)
 
 
 def _describe(wl):
@@ -288,20 +292,30 @@ def run_ours(args):
     bytes_gateup = (active * 2 * wl.I * wl.H * wbytes + P * wl.H * wbytes + P * wl.I * wbytes)
     layer_bytes = (active * 3 * wl.I * wl.H * wbytes + 3 * wl.I_shared * wl.H * 2 + wl.E * wl.H * 2
                    + wl.T * wl.H * (wbytes + 2))
-    bf16_peak, hbm_peak, peak_kind = _peaks()
+    burst, sustained, hbm_peak, peak_kind = _peaks()
+    # a kernel timed inside a long, power-capped run is held to the sustained figure
+    capped = bool(clk and ("sw_power_cap" in clk.get("reasons", []) or
+                           (clk.get("sm_mhz") and clk.get("sm_max_mhz") and
+                            clk["sm_mhz"] < 0.9 * clk["sm_max_mhz"])))
+    ratio = FP8_OVER_BF16 if fp8 else 1.0
+    tensor_peak = (sustained if capped else burst) * ratio
+    dt_name = "e4m3" if fp8 else "bf16"
     dom_ms = [ms for k, ms in traced if k == dominant]
     dom_avg = statistics.mean(dom_ms) if dom_ms else None
-    ridge = bf16_peak * 1e12 / (hbm_peak * 1e9)
+    ridge = tensor_peak * 1e12 / (hbm_peak * 1e9)
     if flops_gateup / bytes_gateup >= ridge:
         achieved = flops_gateup / (dom_avg / 1e3) / 1e12 if dom_avg else None
-        roofline = {"bound": "tensor", "achieved": achieved, "peak": bf16_peak, "unit": "TFLOP/s",
-                    "peak_kind": f"{peak_kind} bf16 burst"}
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": tensor_peak, "unit": "TFLOP/s",
+                    "peak_kind": (f"{peak_kind} bf16 {'sustained' if capped else 'burst'}"
+                                  + (" x2 (e4m3/bf16 nominal ratio)" if fp8 else "")),
+                    "frac_of_burst": achieved / (burst * ratio) if achieved else None,
+                    "frac_of_sustained": achieved / (sustained * ratio) if achieved else None}
     else:
         achieved = bytes_gateup / (dom_avg / 1e3) / 1e9 if dom_avg else None
         roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                     "peak_kind": f"{peak_kind} HBM copy"}
     roofline.update({
-        "kernel": "gateup_swiglu (grouped GEMM, fused SwiGLU)",
+        "kernel": f"gateup_swiglu (grouped GEMM, fused SwiGLU, {dt_name})",
         "frac": achieved / roofline["peak"] if achieved else None,
         "traffic": _profiled_traffic(wl.name), "launches_timed": len(dom_ms), "avg_ms": dom_avg,
         "algorithmic_flops_per_launch": flops_gateup, "algorithmic_bytes_per_launch": bytes_gateup,
@@ -359,6 +373,11 @@ def run_ours(args):
                    "seq_len": 1, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "flushed before every timed step (512 MiB write, outside the events)"},
         "grouped_gemm_tflops": gemm_flops / (ms_step / 1e3) / 1e12 * world,
+        "gemm_kernel_tflops": {k: f / (kernel_ms[k] / 1e3) / 1e12 for k, f in
+                               (("gateup_swiglu", flops_gateup), ("down", flops_down),
+                                ("shared_gateup", 4.0 * wl.T * wl.H * wl.I_shared),
+                                ("shared_down", 2.0 * wl.T * wl.H * wl.I_shared))
+                               if kernel_ms.get(k)},
         "layer_hbm_gbs": layer_bytes / (ms_step / 1e3) / 1e9 * world,
         "active_experts": active,
         "e2e": {"value": wl.T * world / (e2e_ms / 1e3) if e2e_ms else None, "unit": "tokens/s",
@@ -403,6 +422,33 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_micro_grouped_topk(args):
+    """GroupedTopK alone at the routing primer's KernelSwift shape (§十): 83 tokens, 256
+    experts in 8 groups of 32, keep 4 groups, top-8, softmax, renormalised."""
+    wl = W.Workload("grouped_topk_kernelswift", T=83, H=7168, I=128, E=256, K=8, n_group=8,
+                    topk_group=4, group_topn=1)
+    p = B.params(wl)
+    g = torch.Generator(device="cuda").manual_seed(0)
+    logits = torch.randn((wl.T, wl.E), generator=g, device="cuda")
+    ids = torch.empty((wl.T, wl.K), dtype=torch.int32, device="cuda")
+    w = torch.empty((wl.T, wl.K), dtype=torch.float32, device="cuda")
+    for _ in range(args.warmup):
+        B.check(B.moe_grouped_topk(p, logits, None, ids, w))
+    n = max(args.steps, 100)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    s.record()
+    for _ in range(n):
+        B.check(B.moe_grouped_topk(p, logits, None, ids, w))
+    e.record()
+    torch.cuda.synchronize()
+    us = s.elapsed_time(e) * 1e3 / n
+    print(json.dumps({"metric": "GroupedTopK latency (83 tokens, 256 experts, 8x32 groups, keep 4, top-8)",
+                      "value": us, "unit": "us/call", "higher_is_better": False, "steps": n,
+                      "warmup": args.warmup, "n_gpus": 1, "dtype": "f32",
+                      "config": {"workload": wl.name}, "gpu_launches": n}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -411,10 +457,14 @@ def main():
     ap.add_argument("--workload", default="mixtral_prefill", choices=sorted(W.ALL))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--micro", choices=["grouped_topk"], default=None,
+                    help="time one stage alone instead of the layer")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    if args.impl == "reference":
+    if args.micro == "grouped_topk":
+        run_micro_grouped_topk(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

@@ -110,6 +110,19 @@ moe_status_t moe_route(const moe_params_t* p, const void* x, const float* x_scal
                        const void* w_r, const float* bias, int32_t* topk_ids, float* topk_w,
                        void* ws, size_t ws_bytes, void* stream);
 
+/* GroupedTopK on given router logits [T,E] fp32 (routing primer §九, §十: the op takes
+ * the logits and returns K weights and ids per token; x is not read).  Same scoring,
+ * selection and weighting as moe_route; no workspace. */
+moe_status_t moe_grouped_topk(const moe_params_t* p, const float* logits, const float* bias,
+                              int32_t* topk_ids, float* topk_w, void* stream);
+
+/* Auxiliary-loss-free balancing bias, one update from the per-expert loads ("MoE"
+ * chapter index §2.2): bias[e] += gamma * sign(mean_e'(counts) - counts[e]).  counts [E]
+ * int32 (e.g. the counts moe_permute writes), bias [E] fp32 updated in place.  The
+ * bias only steers selection (moe_route); the weights never see it. */
+moe_status_t moe_aux_free_bias_update(const int32_t* counts, int32_t E, float gamma,
+                                      float* bias, void* stream);
+
 /* ---------------------------------------------------------------------------------- */
 /* Stage 2 — dispatch (routing primer §5.1).  Buckets the pairs p = t*K + k by expert,  */
 /* stably in p, each bucket starting at a multiple of block_m.                          */

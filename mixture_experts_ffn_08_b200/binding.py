@@ -60,6 +60,8 @@ _SIGS = {
     "moe_max_padded_rows": (ctypes.c_int64, [_PP]),
     "moe_route": (ctypes.c_int, [_PP, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_permute": (ctypes.c_int, [_PP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "moe_grouped_topk": (ctypes.c_int, [_PP, _P, _P, _P, _P, _P]),
+    "moe_aux_free_bias_update": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.c_float, _P, _P]),
     "moe_permute_noalloc": (ctypes.c_int, [_PP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     "moe_expert_ffn": (ctypes.c_int, [_PP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                       ctypes.c_size_t, _P]),
@@ -143,6 +145,15 @@ def moe_layer_launch_count(p: MoeParams) -> int:
 def moe_route(p, x, x_scale, w_r, bias, topk_ids, topk_w, ws, ws_bytes, stream=None) -> int:
     return lib().moe_route(ctypes.byref(p), _ptr(x), _ptr(x_scale), _ptr(w_r), _ptr(bias),
                            _ptr(topk_ids), _ptr(topk_w), _ptr(ws), ws_bytes, _stream(stream))
+
+
+def moe_grouped_topk(p, logits, bias, topk_ids, topk_w, stream=None) -> int:
+    return lib().moe_grouped_topk(ctypes.byref(p), _ptr(logits), _ptr(bias), _ptr(topk_ids),
+                                  _ptr(topk_w), _stream(stream))
+
+
+def moe_aux_free_bias_update(counts, E, gamma, bias, stream=None) -> int:
+    return lib().moe_aux_free_bias_update(_ptr(counts), E, gamma, _ptr(bias), _stream(stream))
 
 
 def moe_permute(p, topk_ids, x, x_scale, counts, offsets_padded, row_of_pair, pair_of_row,

@@ -306,6 +306,20 @@ moe_status_t moe_route(const moe_params_t* p, const void* x, const float* x_scal
   return do_route(p, x, x_scale, w_r, bias, topk_ids, topk_w, ws, static_cast<cudaStream_t>(stream));
 }
 
+moe_status_t moe_grouped_topk(const moe_params_t* p, const float* logits, const float* bias,
+                              int32_t* topk_ids, float* topk_w, void* stream) {
+  MOE_TRY(validate(p));
+  if (!logits || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
+  if (p->T == 0) return MOE_OK;
+  return cuda_status(launch_topk(logits, *p, bias, topk_ids, topk_w, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_aux_free_bias_update(const int32_t* counts, int32_t E, float gamma, float* bias,
+                                      void* stream) {
+  if (!counts || !bias || E <= 0 || E > kMaxExperts) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_bias_update(counts, E, gamma, bias, static_cast<cudaStream_t>(stream)));
+}
+
 moe_status_t moe_permute(const moe_params_t* p, const int32_t* topk_ids, const void* x, const float* x_scale,
                          int32_t* counts, int32_t* offsets_padded, int32_t* row_of_pair, int32_t* pair_of_row,
                          void* x_perm, float* x_perm_scale, void* ws, size_t ws_bytes, void* stream) {

@@ -25,6 +25,9 @@ cudaError_t launch_dequant_x(const uint8_t* xq, const float* xs, int T, int H, v
 cudaError_t launch_topk(const float* logits, const moe_params_t& p, const float* bias,
                         int32_t* ids, float* w, cudaStream_t st);
 
+// b_e += gamma * sign(mean load - load_e) (aux-free balancing bias).
+cudaError_t launch_bias_update(const int32_t* counts, int E, float gamma, float* bias, cudaStream_t st);
+
 // ---------------------------------------------------------------- dispatch (kernels.cu)
 cudaError_t launch_permute(const moe_params_t& p, const int32_t* ids, const void* x,
                            const float* x_scale, int32_t* counts, int32_t* offsets,

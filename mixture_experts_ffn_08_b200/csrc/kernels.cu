@@ -216,6 +216,32 @@ cudaError_t launch_topk(const float* logits, const moe_params_t& p, const float*
   return cudaGetLastError();
 }
 
+// ================================================================== aux-free bias
+// b_e += gamma * sign(mean_load - load_e), the sign taken exactly in integers as
+// sign(sum_j load_j - E * load_e).  One block.
+__global__ void __launch_bounds__(1024) bias_update_kernel(const int32_t* __restrict__ counts, int E,
+                                                           float gamma, float* __restrict__ bias) {
+  __shared__ long long warp_sum_sh[32];
+  long long local = 0;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) local += __ldg(counts + e);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) local += __shfl_xor_sync(kFull, local, o);
+  if ((threadIdx.x & 31) == 0) warp_sum_sh[threadIdx.x >> 5] = local;
+  __syncthreads();
+  long long total = 0;
+  for (int w = 0; w < (int)(blockDim.x + 31) / 32; ++w) total += warp_sum_sh[w];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const long long d = total - static_cast<long long>(E) * __ldg(counts + e);
+    const float sgn = d > 0 ? 1.f : (d < 0 ? -1.f : 0.f);
+    bias[e] = bias[e] + gamma * sgn;
+  }
+}
+
+cudaError_t launch_bias_update(const int32_t* counts, int E, float gamma, float* bias, cudaStream_t st) {
+  bias_update_kernel<<<1, 1024, 0, st>>>(counts, E, gamma, bias);
+  return cudaGetLastError();
+}
+
 // ================================================================== permute
 // 1) per-chunk expert histogram
 __global__ void __launch_bounds__(kPermChunk) perm_count_kernel(

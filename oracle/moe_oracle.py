@@ -205,6 +205,14 @@ def route(x, w_r, bias, wl):
     return ids, w, s
 
 
+def aux_free_bias_update(bias, counts, gamma: float) -> np.ndarray:
+    """One step of the auxiliary-loss-free balancing bias ("MoE" chapter index §2.2):
+    b_e <- b_e + gamma * sign(mean_load - load_e), with mean_load the average of the
+    per-expert loads (pair counts); an expert exactly at the mean is left unchanged."""
+    load = np.asarray(counts, np.float64)
+    return np.asarray(bias, np.float64) + gamma * np.sign(load.mean() - load)
+
+
 # ----------------------------------------------------------------------------------
 # Dispatch: pairs bucketed by expert
 # ----------------------------------------------------------------------------------

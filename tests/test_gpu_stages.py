@@ -240,3 +240,56 @@ def test_invalid_arguments_return_status_without_launch():
     bad = B.params(wl.with_(K=9))
     assert B.moe_route(bad, x, None, w_r, None, ids, w, ws, ws.numel()) == 1
     torch.cuda.synchronize()
+
+
+# ------------------------------------------------------------------ GroupedTopK, bias
+def _grouped_topk(wl, logits, bias=None):
+    ids = torch.empty((wl.T, wl.K), dtype=torch.int32, device="cuda")
+    w = torch.empty((wl.T, wl.K), dtype=torch.float32, device="cuda")
+    B.check(B.moe_grouped_topk(B.params(wl), logits, bias, ids, w))
+    torch.cuda.synchronize()
+    return ids.cpu().numpy(), w.cpu().numpy()
+
+
+def test_grouped_topk_page_example():
+    # routing primer §七: scores of 8 experts in 4 groups of 2, group score = max, keep 2;
+    # fed as logits log(score) through the softmax router (softmax keeps their order)
+    from tests.conftest import load_golden
+    g = load_golden("grouped_topk_example.txt")
+    z = torch.log(torch.tensor([g["scores"]], dtype=torch.float32, device="cuda"))
+    for K, want in ((3, g["grouped_top3"]), (4, g["grouped_top4"])):
+        wl = W.Workload("ex", T=1, H=128, I=128, E=8, K=K, n_group=g["n_group"],
+                        topk_group=g["topk_group"], group_topn=1)
+        ids, w = _grouped_topk(wl, z)
+        assert ids[0].tolist() == want
+        s = np.array(g["scores"])[want]
+        np.testing.assert_allclose(w[0], s / s.sum(), rtol=1e-6)
+
+
+def test_grouped_topk_kernelswift_shape():
+    # routing primer §十: 83 tokens, 256 experts in 8 groups of 32, keep 4 groups, top-8,
+    # softmax, renormalised
+    wl = W.Workload("ks", T=83, H=128, I=128, E=256, K=8, n_group=8, topk_group=4, group_topn=1)
+    z = torch.randn((wl.T, wl.E), generator=torch.Generator(device="cuda").manual_seed(7), device="cuda") * 2
+    ids, w = _grouped_topk(wl, z)
+    s = o.scores(P.f64(z), 0)
+    n_mism, _ = P.check_routing(ids, w, s, None, wl)
+    assert n_mism == 0
+
+
+def test_aux_free_bias_update_matches_oracle():
+    from tests.conftest import load_golden
+    g = load_golden("aux_free_bias_example.txt")
+    counts = torch.tensor(g["counts"], dtype=torch.int32, device="cuda")
+    bias = torch.tensor(g["bias"], dtype=torch.float32, device="cuda")
+    B.check(B.moe_aux_free_bias_update(counts, 4, g["gamma"], bias))
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(bias.cpu().numpy(), g["updated"], rtol=1e-6)
+    rng = np.random.default_rng(8)
+    c = rng.integers(0, 50, size=256).astype(np.int32)
+    b0 = rng.normal(size=256).astype(np.float32)
+    counts = torch.as_tensor(c, device="cuda")
+    bias = torch.as_tensor(b0, device="cuda")
+    B.check(B.moe_aux_free_bias_update(counts, 256, 0.01, bias))
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(bias.cpu().numpy(), o.aux_free_bias_update(b0, c, 0.01), rtol=1e-6, atol=1e-7)

@@ -375,3 +375,18 @@ def test_store_activation_formats():
     got = o.swiglu_ffn(x, wg, wu, wd, h_format="bf16")
     # torch rounds through fp32 first; both are within one bf16 rounding of each other
     np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------------------------ aux-free bias
+def test_aux_free_bias_update_example():
+    g = load_golden("aux_free_bias_example.txt")
+    got = o.aux_free_bias_update(g["bias"], g["counts"], g["gamma"])
+    np.testing.assert_allclose(got, g["updated"], rtol=0, atol=1e-15)
+
+
+def test_aux_free_bias_update_balanced_is_fixed_point():
+    b = np.array([0.3, -0.2, 0.1])
+    np.testing.assert_array_equal(o.aux_free_bias_update(b, [5, 5, 5], 0.01), b)
+    # only the sign of the imbalance matters, not its size
+    a = o.aux_free_bias_update(np.zeros(3), [1, 2, 100], 0.5)
+    np.testing.assert_array_equal(a, [0.5, 0.5, -0.5])
