@@ -204,7 +204,7 @@ def run_ours(args):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
-    wl = W.ALL[args.workload]
+    wl = {**W.ALL, **W.PROFILE}[args.workload]
     p = B.params(wl)
     d = inputs.make_inputs(wl, seed=rank, device="cuda")
     fp8 = wl.dtype == W.DTYPE_FP8
@@ -398,7 +398,7 @@ def run_reference(args):
     world, rank, _ = _dist()
     if rank != 0:
         return
-    wl = W.ALL[args.workload]
+    wl = {**W.ALL, **W.PROFILE}[args.workload]
     d = inputs.make_inputs(wl, seed=0, device="cpu" if not torch.cuda.is_available() else "cuda")
     n = max(2, _cpu_sample_tokens(wl) // 8)
     times, toks, threads = [], 0, 1
@@ -454,7 +454,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="mixtral_prefill", choices=sorted(W.ALL))
+    ap.add_argument("--workload", default="mixtral_prefill", choices=sorted(W.ALL) + sorted(W.PROFILE))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--micro", choices=["grouped_topk"], default=None,

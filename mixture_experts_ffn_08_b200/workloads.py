@@ -61,3 +61,11 @@ SKEWED_FP8 = Workload("skewed_fp8", T=16384, H=4096, I=1536, E=128, K=8,
                       dtype=DTYPE_FP8, skewed=True)
 
 ALL = {w.name: w for w in (TINY, MIXTRAL_PREFILL, DSV3_PREFILL, DSV3_DECODE, SKEWED_FP8)}
+
+# Stand-ins small enough for a full profiler capture (a few GB on the device) that keep
+# the tile structure of a full workload: DeepSeek-V3 expert shapes with 32 experts and
+# the same ~256 rows per expert as the 256-expert prefill.
+PROFILE = {w.name: w for w in (
+    DSV3_PREFILL.with_(name="dsv3_prefill_e32", T=1024, E=32),
+    SKEWED_FP8.with_(name="skewed_fp8_e32", T=4096, E=32),
+)}
