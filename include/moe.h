@@ -211,8 +211,9 @@ moe_status_t moe_layer_forward(const moe_params_t* p, const void* x, const float
 
 /* Same layer with HOST activations: x_host (and x_scale_host for FP8) are copied to the
  * device inside the call and the result is copied back to out_host, all enqueued on
- * `stream`.  Weights stay device pointers.  Host buffers should be pinned; they must
- * stay valid until the stream has passed this call (cudaStreamSynchronize). */
+ * `stream`.  Weights (and their FP8 scales) stay device pointers.  Host buffers should
+ * be pinned; they must stay valid until the stream has passed this call
+ * (cudaStreamSynchronize).  ws must hold moe_workspace_size_host() bytes. */
 moe_status_t moe_layer_forward_host(const moe_params_t* p, const void* x_host,
                                     const float* x_scale_host, const void* w_r,
                                     const float* bias, const void* w_gate, const void* w_up,

@@ -397,22 +397,24 @@ moe_status_t moe_layer_forward_host(const moe_params_t* p, const void* x_host, c
                                     const float* w_down_scale, const void* ws_gate, const void* ws_up,
                                     const void* ws_down, void* out_host, void* ws, size_t ws_bytes,
                                     void* stream) {
-  (void)w_gate_scale; (void)w_up_scale; (void)w_down_scale;
   MOE_TRY(validate(p));
   MOE_TRY(check_ws(p, ws, ws_bytes, true));
   if (!x_host || !out_host) return MOE_ERR_INVALID_ARG;
-  if (is_fp8(p)) return MOE_ERR_UNSUPPORTED;
+  if (is_fp8(p) && (!x_scale_host || !w_gate_scale || !w_up_scale || !w_down_scale)) return MOE_ERR_INVALID_ARG;
   const Layout L = layout(p);
   void* x_dev = at<void>(ws, L.x_stage);
+  float* xs_dev = is_fp8(p) ? at<float>(ws, L.x_scale_stage) : nullptr;
   void* out_dev = at<void>(ws, L.out_stage);
-  MOE_TRY(check_layer_args(p, x_dev, nullptr, w_r, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, out_dev));
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t xbytes = static_cast<size_t>(p->T) * p->H * 2;
+  MOE_TRY(check_layer_args(p, x_dev, xs_dev, w_r, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, out_dev));
   if (p->T == 0) return MOE_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t xbytes = static_cast<size_t>(p->T) * p->H * (is_fp8(p) ? 1 : 2);
   MOE_CUDA(cudaMemcpyAsync(x_dev, x_host, xbytes, cudaMemcpyHostToDevice, st));
-  MOE_TRY(do_layer(p, x_dev, nullptr, w_r, bias, w_gate, w_up, w_down, nullptr, nullptr, nullptr, ws_gate,
-                   ws_up, ws_down, out_dev,
-                   nullptr, nullptr, nullptr, ws, st));
+  if (is_fp8(p))
+    MOE_CUDA(cudaMemcpyAsync(xs_dev, x_scale_host, static_cast<size_t>(p->T) * (p->H / 128) * sizeof(float),
+                             cudaMemcpyHostToDevice, st));
+  MOE_TRY(do_layer(p, x_dev, xs_dev, w_r, bias, w_gate, w_up, w_down, w_gate_scale, w_up_scale, w_down_scale,
+                   ws_gate, ws_up, ws_down, out_dev, nullptr, nullptr, nullptr, ws, st));
   MOE_CUDA(cudaMemcpyAsync(out_host, out_dev, static_cast<size_t>(p->T) * p->H * 2, cudaMemcpyDeviceToHost, st));
   return MOE_OK;
 }

@@ -124,3 +124,18 @@ def test_fp8_layer_full_size_sampled():
                                   h_format="e4m3")
     got = P.f64(res["out"][torch.as_tensor(toks, device="cuda")])
     P.check_close(got, ref, P.FP8_MAX_TOL, wl.name)
+
+
+def test_fp8_host_entry_point_matches_device_entry_point():
+    wl = SMALL_FP8
+    d = inputs.make_inputs(wl, seed=2, device="cuda")
+    res = P.run_layer(wl, d)
+    p = B.params(wl)
+    a = P.device_inputs_ptrs(d, wl)
+    out_host = torch.empty((wl.T, wl.H), dtype=torch.bfloat16).pin_memory()
+    B.check(B.moe_layer_forward_host(p, d["x_q"].cpu().pin_memory(), d["x_scale"].cpu().pin_memory(),
+                                     a["w_r"], None, a["w_gate"], a["w_up"], a["w_down"], a["w_gate_scale"],
+                                     a["w_up_scale"], a["w_down_scale"], None, None, None, out_host,
+                                     res["ws"], res["ws"].numel()))
+    torch.cuda.synchronize()
+    assert torch.equal(out_host, res["out"].cpu())
