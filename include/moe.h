@@ -167,16 +167,18 @@ moe_status_t moe_permute_noalloc(const moe_params_t* p, const int32_t* topk_ids,
 /* for every row r of expert e's bucket (pad rows included; their result is unused).    */
 /*   offsets_padded [E+1], counts [E] as written by moe_permute (read on the device     */
 /*                  only); counts may be NULL, then pad rows are computed and stored too */
-/*   y_perm [moe_max_padded_rows, H] fp32 out; rows past counts[e] in a bucket are not   */
-/*                  written when counts is given                                        */
-/* The SwiGLU intermediate h (bf16) lives in ws.  y_perm stays fp32 because it feeds    */
-/* the output directly: the final bf16 rounding already uses most of the error budget. */
+/*   y_perm [moe_max_padded_rows, H] out, fp32 for MOE_DTYPE_BF16 and bf16 for FP8; rows */
+/*                  past counts[e] in a bucket are not written when counts is given     */
+/* The SwiGLU intermediate h (bf16, or e4m3 + scales) lives in ws.  For bf16 workloads  */
+/* y_perm stays fp32 because it feeds the output directly and the final bf16 rounding   */
+/* already uses most of the 2e-2 RMS error budget; the FP8 bound (6e-2) leaves room for */
+/* a bf16 y_perm, which halves its HBM round trip.                                      */
 /* ---------------------------------------------------------------------------------- */
 moe_status_t moe_expert_ffn(const moe_params_t* p, const void* x_perm, const float* x_perm_scale,
                             const int32_t* offsets_padded, const int32_t* counts,
                             const void* w_gate, const void* w_up, const void* w_down,
                             const float* w_gate_scale, const float* w_up_scale,
-                            const float* w_down_scale, float* y_perm, void* ws, size_t ws_bytes,
+                            const float* w_down_scale, void* y_perm, void* ws, size_t ws_bytes,
                             void* stream);
 
 /* Dense SwiGLU FFN of the always-active shared expert on all T tokens ("MoE" §0, §2.1):
@@ -188,10 +190,11 @@ moe_status_t moe_shared_expert_ffn(const moe_params_t* p, const void* x, const v
 /* ---------------------------------------------------------------------------------- */
 /* Stage 4 — combine (routing primer §5.3): out[t] = sum_k w[t,k] y_perm[row_of_pair[   */
 /* t*K+k]] (+ y_shared[t]), fp32 accumulation in fixed k order, one rounding to bf16.   */
-/* y_perm [rows,H] and y_shared [T,H] (may be NULL) are fp32; out [T,H] bf16.  Pairs    */
+/* y_perm [rows,H] as moe_expert_ffn writes it (fp32, or bf16 for FP8); y_shared [T,H]  */
+/* fp32 or NULL; out [T,H] bf16.  Pairs                                                 */
 /* with row_of_pair = -1 are left out.  No atomics: bitwise reproducible.               */
 /* ---------------------------------------------------------------------------------- */
-moe_status_t moe_combine(const moe_params_t* p, const float* y_perm, const int32_t* row_of_pair,
+moe_status_t moe_combine(const moe_params_t* p, const void* y_perm, const int32_t* row_of_pair,
                          const float* topk_w, const float* y_shared, void* out, void* stream);
 
 /* ---------------------------------------------------------------------------------- */

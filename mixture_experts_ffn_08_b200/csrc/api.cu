@@ -185,7 +185,7 @@ moe_status_t do_permute(const moe_params_t* p, const int32_t* ids, const void* x
 moe_status_t do_expert_ffn_fp8(const moe_params_t* p, const void* x_perm, const float* x_perm_scale,
                                const int32_t* offsets, const int32_t* counts, const void* w_gate,
                                const void* w_up, const void* w_down, const float* wgs,
-                               const float* wus, const float* wds, float* y_perm, void* ws,
+                               const float* wus, const float* wds, void* y_perm, void* ws,
                                cudaStream_t st) {
   const Layout L = layout(p);
   int32_t* status = at<int32_t>(ws, L.status);
@@ -336,7 +336,7 @@ moe_status_t moe_permute(const moe_params_t* p, const int32_t* topk_ids, const v
 moe_status_t moe_expert_ffn(const moe_params_t* p, const void* x_perm, const float* x_perm_scale,
                             const int32_t* offsets_padded, const int32_t* counts, const void* w_gate,
                             const void* w_up, const void* w_down, const float* w_gate_scale,
-                            const float* w_up_scale, const float* w_down_scale, float* y_perm,
+                            const float* w_up_scale, const float* w_down_scale, void* y_perm,
                             void* ws, size_t ws_bytes, void* stream) {
   MOE_TRY(validate(p));
   MOE_TRY(check_ws(p, ws, ws_bytes, false));
@@ -350,7 +350,7 @@ moe_status_t moe_expert_ffn(const moe_params_t* p, const void* x_perm, const flo
     return do_expert_ffn_fp8(p, x_perm, x_perm_scale, offsets_padded, counts, w_gate, w_up, w_down,
                              w_gate_scale, w_up_scale, w_down_scale, y_perm, ws,
                              static_cast<cudaStream_t>(stream));
-  return do_expert_ffn(p, x_perm, offsets_padded, counts, w_gate, w_up, w_down, y_perm, ws,
+  return do_expert_ffn(p, x_perm, offsets_padded, counts, w_gate, w_up, w_down, static_cast<float*>(y_perm), ws,
                        static_cast<cudaStream_t>(stream));
 }
 
@@ -367,7 +367,7 @@ moe_status_t moe_shared_expert_ffn(const moe_params_t* p, const void* x, const v
   return do_shared(p, x, ws_gate, ws_up, ws_down, y_shared, ws, static_cast<cudaStream_t>(stream));
 }
 
-moe_status_t moe_combine(const moe_params_t* p, const float* y_perm, const int32_t* row_of_pair,
+moe_status_t moe_combine(const moe_params_t* p, const void* y_perm, const int32_t* row_of_pair,
                          const float* topk_w, const float* y_shared, void* out, void* stream) {
   MOE_TRY(validate(p));
   if (!y_perm || !row_of_pair || !topk_w || !out) return MOE_ERR_INVALID_ARG;

@@ -133,9 +133,9 @@ cudaError_t gemm_gateup_swiglu_fp8(const void* A, const uint8_t* a_atoms, int64_
 
 cudaError_t gemm_down_fp8(const void* A, const uint8_t* a_atoms, int64_t a_rows,
                           const int32_t* offsets, const int32_t* counts, int G, const void* w,
-                          const uint8_t* w_atoms, int N, int K, float* y, int32_t* status,
+                          const uint8_t* w_atoms, int N, int K, void* y, int32_t* status,
                           cudaStream_t st) {
-  using Cfg = Fp8Cfg<128, EPI8_F32, 5>;
+  using Cfg = Fp8Cfg<128, EPI8_BF16, 5>;
   CUtensorMap ta, tb;
   if (!make_tmap_u8(&ta, A, a_rows, K, 128) || !make_tmap_u8(&tb, w, static_cast<uint64_t>(G) * N, K, 128))
     return cudaErrorInvalidValue;

@@ -36,7 +36,8 @@ cudaError_t launch_permute(const moe_params_t& p, const int32_t* ids, const void
                            cudaStream_t st);
 
 // ---------------------------------------------------------------- combine (kernels.cu)
-cudaError_t launch_combine(const moe_params_t& p, const float* y_perm, const int32_t* row_of_pair,
+// y_perm is fp32 for bf16 workloads and bf16 for FP8 workloads (p.dtype).
+cudaError_t launch_combine(const moe_params_t& p, const void* y_perm, const int32_t* row_of_pair,
                            const float* w, const float* y_shared, void* out, cudaStream_t st);
 
 // ---------------------------------------------------------------- GEMMs (gemm.cu)
@@ -67,10 +68,10 @@ cudaError_t gemm_gateup_swiglu_fp8(const void* A, const uint8_t* a_atoms, int64_
                                    const void* w_gate, const void* w_up, const uint8_t* gate_atoms,
                                    const uint8_t* up_atoms, int N, int K, void* h, uint8_t* h_atoms,
                                    int32_t* status, cudaStream_t st);
-// y [rows, N] fp32 = A W^T, block-scaled e4m3 GEMM.
+// y [rows, N] bf16 = A W^T, block-scaled e4m3 GEMM.
 cudaError_t gemm_down_fp8(const void* A, const uint8_t* a_atoms, int64_t a_rows,
                           const int32_t* offsets, const int32_t* counts, int G, const void* w,
-                          const uint8_t* w_atoms, int N, int K, float* y, int32_t* status,
+                          const uint8_t* w_atoms, int N, int K, void* y, int32_t* status,
                           cudaStream_t st);
 
 }  // namespace moe

@@ -415,13 +415,31 @@ cudaError_t launch_permute(const moe_params_t& p, const int32_t* ids, const void
 }
 
 // ================================================================== combine
+MOE_DEVINL void load8(const float* row, int v, float (&f)[8]) {
+  const float4* src = reinterpret_cast<const float4*>(row) + 2 * v;
+  const float4 a = __ldg(src), b = __ldg(src + 1);
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+
+MOE_DEVINL void load8(const __nv_bfloat16* row, int v, float (&f)[8]) {
+  const uint4 q = __ldg(reinterpret_cast<const uint4*>(row) + v);
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+// out[t] = sum_k w[t,k] y_perm[row_of_pair[t*K+k]] (+ y_sh[t]); YT = float or bf16.
+template <class YT>
 __global__ void __launch_bounds__(128) combine_kernel(
-    const float* __restrict__ y_perm, const int32_t* __restrict__ row_of_pair,
+    const YT* __restrict__ y_perm, const int32_t* __restrict__ row_of_pair,
     const float* __restrict__ w, const float* __restrict__ y_sh,
     __nv_bfloat16* __restrict__ out, int T, int H, int K) {
   __shared__ int rows[kMaxTopK];
   __shared__ float wk[kMaxTopK];
-  const int nvec = H / 8;  // 8 outputs (two float4 loads, one 16-byte store) per thread step
+  const int nvec = H / 8;  // 8 outputs (one 16-byte store) per thread step
   for (int t = blockIdx.x; t < T; t += gridDim.x) {
     __syncthreads();
     if (threadIdx.x < K) {
@@ -434,19 +452,17 @@ __global__ void __launch_bounds__(128) combine_kernel(
       for (int k = 0; k < K; ++k) {
         const int r = rows[k];
         if (r < 0) continue;
-        const float4* src = reinterpret_cast<const float4*>(y_perm + static_cast<long long>(r) * H) + 2 * v;
-        const float4 a = __ldg(src), b = __ldg(src + 1);
+        float f[8];
+        load8(y_perm + static_cast<long long>(r) * H, v, f);
         const float wv = wk[k];
-        acc[0] = fmaf(wv, a.x, acc[0]); acc[1] = fmaf(wv, a.y, acc[1]);
-        acc[2] = fmaf(wv, a.z, acc[2]); acc[3] = fmaf(wv, a.w, acc[3]);
-        acc[4] = fmaf(wv, b.x, acc[4]); acc[5] = fmaf(wv, b.y, acc[5]);
-        acc[6] = fmaf(wv, b.z, acc[6]); acc[7] = fmaf(wv, b.w, acc[7]);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = fmaf(wv, f[i], acc[i]);
       }
       if (y_sh) {
-        const float4* src = reinterpret_cast<const float4*>(y_sh + static_cast<long long>(t) * H) + 2 * v;
-        const float4 a = __ldg(src), b = __ldg(src + 1);
-        acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
-        acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+        float f[8];
+        load8(y_sh + static_cast<long long>(t) * H, v, f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] += f[i];
       }
       reinterpret_cast<uint4*>(out + static_cast<long long>(t) * H)[v] =
           make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
@@ -455,13 +471,18 @@ __global__ void __launch_bounds__(128) combine_kernel(
   }
 }
 
-cudaError_t launch_combine(const moe_params_t& p, const float* y_perm, const int32_t* row_of_pair,
+cudaError_t launch_combine(const moe_params_t& p, const void* y_perm, const int32_t* row_of_pair,
                            const float* w, const float* y_shared, void* out, cudaStream_t st) {
   if (p.T == 0) return cudaSuccess;
   const int grid = p.T < num_sms() * 16 ? p.T : num_sms() * 16;
   trace_before(MOE_K_COMBINE, st);
-  combine_kernel<<<grid, 128, 0, st>>>(y_perm, row_of_pair, w, y_shared,
-                                       static_cast<__nv_bfloat16*>(out), p.T, p.H, p.K);
+  if (p.dtype == MOE_DTYPE_FP8_E4M3)
+    combine_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(y_perm), row_of_pair,
+                                                        w, y_shared, static_cast<__nv_bfloat16*>(out), p.T,
+                                                        p.H, p.K);
+  else
+    combine_kernel<float><<<grid, 128, 0, st>>>(static_cast<const float*>(y_perm), row_of_pair, w, y_shared,
+                                                static_cast<__nv_bfloat16*>(out), p.T, p.H, p.K);
   trace_after(MOE_K_COMBINE, st);
   return cudaGetLastError();
 }

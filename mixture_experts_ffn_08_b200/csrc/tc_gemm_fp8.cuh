@@ -23,7 +23,9 @@
 //                  two scale that keeps |h| / scale <= 448; writes the codes and the scale
 //                  atoms the down projection consumes.  One accumulator; the epilogue
 //                  releases TMEM as soon as it has read it, before quantising.
-//   EPI8_F32       fp32 store (down projection), two accumulators.
+//   EPI8_BF16      bf16 store (down projection), two accumulators.  The FP8 layer's
+//                  2e-2 -> 6e-2 RMS bound leaves room for this rounding, and it halves
+//                  the bytes of the y_perm round trip through HBM.
 #pragma once
 
 #include <cuda_fp8.h>
@@ -89,7 +91,7 @@ __host__ __device__ constexpr uint32_t idesc_mxf8_e4m3(int M, int N, uint32_t a_
 // 32 K-elements): rows m0 + 32*m1 keep their 4 scales at 16*m0 + 4*m1.
 MOE_DEVINL int sf_atom_offset(int m) { return 16 * (m & 31) + 4 * ((m >> 5) & 3); }
 
-enum Fp8Epi { EPI8_SWIGLU_Q = 0, EPI8_F32 = 1 };
+enum Fp8Epi { EPI8_SWIGLU_Q = 0, EPI8_BF16 = 1 };
 
 struct Fp8Params {
   const int32_t* offsets;  // [G+1] first row of each group (multiples of 128)
@@ -100,7 +102,7 @@ struct Fp8Params {
   const uint8_t* sfa;      // A scale atoms [m_tiles][K/128][512]
   const uint8_t* sfb0;     // B scale atoms [G][N/128][K/128][512] (gate, or the down weight)
   const uint8_t* sfb1;     // up-projection scale atoms (SwiGLU only)
-  void* out;               // SwiGLU: e4m3 codes [rows, ldo]; F32: fp32 [rows, ldo]
+  void* out;               // SwiGLU: e4m3 codes [rows, ldo]; BF16: bf16 [rows, ldo]
   int64_t ldo;             // elements
   uint8_t* out_sf;         // SwiGLU: h scale atoms [m_tiles][N/128][512]
   int32_t* status;
@@ -340,16 +342,21 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         uint8_t* sf = p.out_sf + (static_cast<size_t>(t.m_tile) * (p.N / 128) + t.n_tile) * 512;
         *reinterpret_cast<uint32_t*>(sf + sf_atom_offset(row_in_tile)) = byte * 0x01010101u;
       } else {
-        float* out = static_cast<float*>(p.out) + row * p.ldo + col0;
+        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + row * p.ldo + col0;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
           uint32_t r[32];
           tmem_ld_32x32b_x32(tbase + c, r);
           tmem_ld_wait();
           if (row_ok && col0 + c < p.N) {
+            uint32_t packed[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              packed[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
             uint4* dst = reinterpret_cast<uint4*>(out + c);
 #pragma unroll
-            for (int v = 0; v < 8; ++v) dst[v] = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+            for (int v = 0; v < 4; ++v)
+              dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
           }
         }
         tc_fence_before();

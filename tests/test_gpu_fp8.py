@@ -36,7 +36,7 @@ def _expert_ffn_fp8(wl, d, ids_np):
     r = _permute_fp8(wl, ids_np, d)
     p = B.params(wl)
     rows = B.moe_max_padded_rows(p)
-    y = torch.full((rows, wl.H), float("nan"), dtype=torch.float32, device="cuda")
+    y = torch.full((rows, wl.H), float("nan"), dtype=torch.bfloat16, device="cuda")
     B.check(B.moe_expert_ffn(p, r["xp"], r["xps"], r["offs"], r["counts"], d["w_gate_q"], d["w_up_q"],
                              d["w_down_q"], d["w_gate_s"], d["w_up_s"], d["w_down_s"], y, r["ws"],
                              r["ws"].numel()))
