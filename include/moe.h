@@ -77,8 +77,9 @@ typedef struct moe_params {
   float routed_scale;   /* factor applied to the (renormalised) weights                  */
   int32_t I_shared;     /* intermediate size of the shared expert, 0 = none              */
   int32_t dtype;        /* MOE_DTYPE_BF16 or MOE_DTYPE_FP8_E4M3                          */
-  int32_t block_m;      /* row alignment of each expert's bucket; 0 = default (128).     */
-                        /* Only 128 is accepted by this build.                           */
+  int32_t block_m;      /* row alignment of each expert's bucket: 128 (one-SM GEMM tiles), */
+                        /* 256 (two-SM cta_group::2 tiles), 0 = choose: 256 when buckets */
+                        /* average >= 512 rows (T*K >= 512*E), else 128                  */
 } moe_params_t;
 
 /* ---------------------------------------------------------------------------------- */
@@ -92,6 +93,9 @@ size_t moe_workspace_size(const moe_params_t* p);
 /* Bytes of workspace moe_layer_forward_host() needs: moe_workspace_size() plus device
  * staging for the copied activations and output.  0 if the parameters are invalid. */
 size_t moe_workspace_size_host(const moe_params_t* p);
+
+/* Bucket alignment the calls use for these parameters (128 or 256); -1 if invalid. */
+int32_t moe_effective_block_m(const moe_params_t* p);
 
 /* Upper bound on the padded row count P + E*(block_m-1): the row capacity that
  * pair_of_row, x_perm and y_perm must have.  -1 if the parameters are invalid. */

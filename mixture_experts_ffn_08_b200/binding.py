@@ -49,7 +49,7 @@ class MoeParams(ctypes.Structure):
 def params(wl: W.Workload) -> MoeParams:
     return MoeParams(wl.T, wl.H, wl.I, wl.E, wl.K, wl.n_group, wl.topk_group, wl.group_topn,
                      wl.score_fn, int(wl.renormalize), float(wl.routed_scale), wl.I_shared,
-                     wl.dtype, 0)
+                     wl.dtype, wl.block_m)
 
 
 _P = ctypes.c_void_p
@@ -58,6 +58,7 @@ _SIGS = {
     "moe_workspace_size": (ctypes.c_size_t, [_PP]),
     "moe_workspace_size_host": (ctypes.c_size_t, [_PP]),
     "moe_max_padded_rows": (ctypes.c_int64, [_PP]),
+    "moe_effective_block_m": (ctypes.c_int32, [_PP]),
     "moe_route": (ctypes.c_int, [_PP, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_permute": (ctypes.c_int, [_PP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "moe_grouped_topk": (ctypes.c_int, [_PP, _P, _P, _P, _P, _P]),
@@ -135,6 +136,10 @@ def moe_workspace_size_host(p: MoeParams) -> int:
 
 def moe_max_padded_rows(p: MoeParams) -> int:
     return lib(require_gpu=False).moe_max_padded_rows(ctypes.byref(p))
+
+
+def moe_effective_block_m(p: MoeParams) -> int:
+    return lib(require_gpu=False).moe_effective_block_m(ctypes.byref(p))
 
 
 def moe_layer_launch_count(p: MoeParams) -> int:

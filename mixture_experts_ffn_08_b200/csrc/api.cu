@@ -71,12 +71,20 @@ struct Layout {
 
 bool is_fp8(const moe_params_t* p) { return p->dtype == MOE_DTYPE_FP8_E4M3; }
 
+// Bucket alignment: 256 rows (two-SM GEMMs) when buckets average at least 512 rows, where
+// the extra padding is small against the traffic the pair tiles save; else 128.
+int block_m_of(const moe_params_t* p) {
+  if (p->block_m != 0) return p->block_m;
+  return static_cast<long long>(p->T) * p->K >= 512LL * p->E ? kBlockM2 : kBlockM;
+}
+
 Layout layout(const moe_params_t* p) {
   Layout L{};
   const long long T = p->T, H = p->H, I = p->I, E = p->E, K = p->K;
   const long long P = T * K;
-  const long long rows = P + E * (kBlockM - 1);
-  const long long rows_t = (rows + kBlockM - 1) / kBlockM * kBlockM;  // whole M-tiles
+  const long long bm = block_m_of(p);
+  const long long rows = P + E * (bm - 1);
+  const long long rows_t = (rows + kBlockM2 - 1) / kBlockM2 * kBlockM2;  // whole M-tile pairs
   const long long nchunks = (P + kPermChunk - 1) / kPermChunk;
   const size_t xelem = is_fp8(p) ? 1 : 2;
   size_t o = 0;
@@ -132,9 +140,9 @@ moe_status_t validate(const moe_params_t* p) {
   }
   if (p->I_shared < 0) return MOE_ERR_INVALID_ARG;
   if (p->H % 128 != 0 || p->I % 128 != 0 || p->I_shared % 128 != 0) return MOE_ERR_UNSUPPORTED;
-  if (p->block_m != 0 && p->block_m != kBlockM) return MOE_ERR_UNSUPPORTED;
+  if (p->block_m != 0 && p->block_m != kBlockM && p->block_m != kBlockM2) return MOE_ERR_UNSUPPORTED;
   if (p->dtype == MOE_DTYPE_FP8_E4M3 && p->I_shared > 0) return MOE_ERR_UNSUPPORTED;
-  const long long rows = static_cast<long long>(p->T) * p->K + static_cast<long long>(p->E) * (kBlockM - 1);
+  const long long rows = static_cast<long long>(p->T) * p->K + static_cast<long long>(p->E) * (kBlockM2 - 1);
   if (rows >= (1LL << 31) / 2) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
@@ -178,7 +186,7 @@ moe_status_t do_permute(const moe_params_t* p, const int32_t* ids, const void* x
                         int32_t* counts, int32_t* offsets, int32_t* rop, int32_t* por, void* x_perm,
                         float* x_perm_scale, void* ws, cudaStream_t st) {
   const Layout L = layout(p);
-  return cuda_status(launch_permute(*p, ids, x, x_scale, counts, offsets, rop, por, x_perm, x_perm_scale,
+  return cuda_status(launch_permute(*p, block_m_of(p), ids, x, x_scale, counts, offsets, rop, por, x_perm, x_perm_scale,
                                     at<int32_t>(ws, L.chunk_counts), at<int32_t>(ws, L.status), st));
 }
 
@@ -196,6 +204,14 @@ moe_status_t do_expert_ffn_fp8(const moe_params_t* p, const void* x_perm, const 
   MOE_CUDA(launch_sf_rows_to_atoms(x_perm_scale, p->H / 128, offsets, p->E, L.max_rows,
                                    at<uint8_t>(ws, L.x_atoms), st));
   void* h = at<void>(ws, L.h);
+  if (block_m_of(p) == kBlockM2) {
+    MOE_CUDA(gemm_pair_gateup_swiglu_fp8(x_perm, at<uint8_t>(ws, L.x_atoms), L.max_rows, offsets, counts, p->E,
+                                         w_gate, w_up, at<uint8_t>(ws, L.wg_atoms), at<uint8_t>(ws, L.wu_atoms),
+                                         p->I, p->H, h, at<uint8_t>(ws, L.h_atoms), status, st));
+    MOE_CUDA(gemm_pair_down_fp8(h, at<uint8_t>(ws, L.h_atoms), L.max_rows, offsets, counts, p->E, w_down,
+                                at<uint8_t>(ws, L.wd_atoms), p->H, p->I, y_perm, status, st));
+    return MOE_OK;
+  }
   MOE_CUDA(gemm_gateup_swiglu_fp8(x_perm, at<uint8_t>(ws, L.x_atoms), L.max_rows, offsets, counts, p->E,
                                   w_gate, w_up, at<uint8_t>(ws, L.wg_atoms), at<uint8_t>(ws, L.wu_atoms),
                                   p->I, p->H, h, at<uint8_t>(ws, L.h_atoms), status, st));
@@ -210,6 +226,12 @@ moe_status_t do_expert_ffn(const moe_params_t* p, const void* x_perm, const int3
   const Layout L = layout(p);
   int32_t* status = at<int32_t>(ws, L.status);
   void* h = at<void>(ws, L.h);
+  if (block_m_of(p) == kBlockM2) {
+    MOE_CUDA(gemm_pair_gateup_swiglu(x_perm, L.max_rows, offsets, counts, p->E, w_gate, w_up, p->I, p->H, h,
+                                     status, st));
+    MOE_CUDA(gemm_pair_down(h, L.max_rows, offsets, counts, p->E, w_down, p->H, p->I, y_perm, status, st));
+    return MOE_OK;
+  }
   MOE_CUDA(gemm_gateup_swiglu(x_perm, L.max_rows, offsets, counts, p->E, 0, w_gate, w_up, p->I, p->H,
                               h, status, MOE_K_GATEUP, st));
   MOE_CUDA(gemm_down(h, L.max_rows, offsets, counts, p->E, 0, w_down, p->H, p->I, y_perm, status,
@@ -288,6 +310,11 @@ size_t moe_workspace_size(const moe_params_t* p) {
 size_t moe_workspace_size_host(const moe_params_t* p) {
   if (validate(p) != MOE_OK) return 0;
   return layout(p).total_host;
+}
+
+int32_t moe_effective_block_m(const moe_params_t* p) {
+  if (validate(p) != MOE_OK) return -1;
+  return block_m_of(p);
 }
 
 int64_t moe_max_padded_rows(const moe_params_t* p) {

@@ -9,7 +9,8 @@
 
 namespace moe {
 
-constexpr int kBlockM = 128;    // M-tile of the grouped GEMM = row alignment of buckets
+constexpr int kBlockM = 128;    // M-tile of the one-SM grouped GEMM (bucket alignment)
+constexpr int kBlockM2 = 256;   // bucket alignment for the two-SM (cta_group::2) GEMMs
 constexpr int kMaxExperts = 1024;
 constexpr int kMaxTopK = 32;
 constexpr int kPermChunk = 256;  // pairs per chunk of the stable bucket ranking
@@ -29,7 +30,7 @@ cudaError_t launch_topk(const float* logits, const moe_params_t& p, const float*
 cudaError_t launch_bias_update(const int32_t* counts, int E, float gamma, float* bias, cudaStream_t st);
 
 // ---------------------------------------------------------------- dispatch (kernels.cu)
-cudaError_t launch_permute(const moe_params_t& p, const int32_t* ids, const void* x,
+cudaError_t launch_permute(const moe_params_t& p, int block_m, const int32_t* ids, const void* x,
                            const float* x_scale, int32_t* counts, int32_t* offsets,
                            int32_t* row_of_pair, int32_t* pair_of_row, void* x_perm,
                            float* x_perm_scale, int32_t* chunk_counts, int32_t* status,
@@ -73,5 +74,20 @@ cudaError_t gemm_down_fp8(const void* A, const uint8_t* a_atoms, int64_t a_rows,
                           const int32_t* offsets, const int32_t* counts, int G, const void* w,
                           const uint8_t* w_atoms, int N, int K, void* y, int32_t* status,
                           cudaStream_t st);
+
+// ---------------------------------------------------------------- two-SM GEMMs (gemm_2cta.cu)
+cudaError_t gemm_pair_gateup_swiglu(const void* A, int64_t a_rows, const int32_t* offsets, const int32_t* counts,
+                                    int G, const void* w_gate, const void* w_up, int N, int K, void* h,
+                                    int32_t* status, cudaStream_t st);
+cudaError_t gemm_pair_down(const void* A, int64_t a_rows, const int32_t* offsets, const int32_t* counts, int G,
+                           const void* w, int N, int K, float* y, int32_t* status, cudaStream_t st);
+cudaError_t gemm_pair_gateup_swiglu_fp8(const void* A, const uint8_t* a_atoms, int64_t a_rows,
+                                        const int32_t* offsets, const int32_t* counts, int G, const void* w_gate,
+                                        const void* w_up, const uint8_t* gate_atoms, const uint8_t* up_atoms,
+                                        int N, int K, void* h, uint8_t* h_atoms, int32_t* status,
+                                        cudaStream_t st);
+cudaError_t gemm_pair_down_fp8(const void* A, const uint8_t* a_atoms, int64_t a_rows, const int32_t* offsets,
+                               const int32_t* counts, int G, const void* w, const uint8_t* w_atoms, int N, int K,
+                               void* y, int32_t* status, cudaStream_t st);
 
 }  // namespace moe

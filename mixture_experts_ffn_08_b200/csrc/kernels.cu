@@ -374,14 +374,14 @@ __global__ void __launch_bounds__(256) perm_gather_kernel(
   }
 }
 
-cudaError_t launch_permute(const moe_params_t& p, const int32_t* ids, const void* x,
+cudaError_t launch_permute(const moe_params_t& p, int block_m, const int32_t* ids, const void* x,
                            const float* x_scale, int32_t* counts, int32_t* offsets,
                            int32_t* row_of_pair, int32_t* pair_of_row, void* x_perm,
                            float* x_perm_scale, int32_t* chunk_counts, int32_t* status,
                            cudaStream_t st) {
   const int P = p.T * p.K;
   const int nchunks = (P + kPermChunk - 1) / kPermChunk;
-  const int bm = kBlockM;
+  const int bm = block_m;
   cudaError_t err;
   if (nchunks > 0) {
     trace_before(MOE_K_PERM_COUNT, st);

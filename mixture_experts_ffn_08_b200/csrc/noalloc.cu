@@ -75,7 +75,7 @@ extern "C" moe_status_t moe_permute_noalloc(const moe_params_t* p, const int32_t
   int32_t* scratch = nullptr;
   const moe_status_t s = scratch_for_current_device(&scratch);
   if (s != MOE_OK) return s;
-  const cudaError_t e = launch_permute(*p, topk_ids, x, x_scale, counts, offsets_padded, row_of_pair,
+  const cudaError_t e = launch_permute(*p, moe_effective_block_m(p), topk_ids, x, x_scale, counts, offsets_padded, row_of_pair,
                                        pair_of_row, x_perm, x_perm_scale, scratch, device_status,
                                        static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;

@@ -37,6 +37,7 @@ class Workload:
     I_shared: int = 0       # intermediate size of the always-active shared expert (0 = none)
     dtype: int = DTYPE_BF16
     skewed: bool = False    # Zipf-shaped router for the skew stress case
+    block_m: int = 0        # bucket row alignment: 128, 256 (two-SM GEMM tiles), 0 = library choice
 
     @property
     def P(self) -> int:

@@ -157,8 +157,8 @@ def check_routing(gpu_ids, gpu_w, s, bias, wl, w_rtol=1e-4):
     return len(mism), wt
 
 
-def check_permutation(gpu_ids, E, counts, offsets, rop, por, n_rows=None):
-    o_counts, o_off, o_rop, o_por = o.permute(gpu_ids, E, B.BLOCK_M)
+def check_permutation(gpu_ids, E, counts, offsets, rop, por, block_m=B.BLOCK_M):
+    o_counts, o_off, o_rop, o_por = o.permute(gpu_ids, E, block_m)
     np.testing.assert_array_equal(counts, o_counts)
     np.testing.assert_array_equal(offsets, o_off)
     np.testing.assert_array_equal(rop, o_rop)

@@ -53,14 +53,16 @@ def test_sizes(lib):
     for wl in W.ALL.values():
         p = B.params(wl)
         rows = B.moe_max_padded_rows(p)
-        assert rows == wl.T * wl.K + wl.E * (B.BLOCK_M - 1)
+        bm = B.moe_effective_block_m(p)
+        assert bm == (256 if wl.T * wl.K >= 512 * wl.E else 128)
+        assert rows == wl.T * wl.K + wl.E * (bm - 1)
         ws = B.moe_workspace_size(p)
         assert ws >= rows * wl.H * (1 if wl.dtype else 2) * 2
         assert B.moe_workspace_size_host(p) > ws
         assert B.moe_layer_launch_count(p) == 9 + (2 if wl.I_shared else 0) + (5 if wl.dtype else 0)
 
 
-@pytest.mark.parametrize("change", [dict(H=100), dict(I=200), dict(K=0), dict(E=2000),
+@pytest.mark.parametrize("change", [dict(H=100), dict(I=200), dict(K=0), dict(E=2000), dict(block_m=64),
                                     dict(K=40), dict(n_group=3), dict(topk_group=9),
                                     dict(group_topn=40), dict(score_fn=5), dict(dtype=7),
                                     dict(I_shared=100), dict(T=-1)])

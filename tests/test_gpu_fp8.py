@@ -47,7 +47,8 @@ def _expert_ffn_fp8(wl, d, ids_np):
 
 def _check_vs_oracle(wl, d, ids_np, r, y):
     x = P.x_f64(d, wl)
-    ref, _ = o.expert_outputs(x, ids_np, P.expert_weights_fn(d, wl), wl.E, BM, h_format="e4m3")
+    ref, _ = o.expert_outputs(x, ids_np, P.expert_weights_fn(d, wl), wl.E,
+                              B.moe_effective_block_m(B.params(wl)), h_format="e4m3")
     offs = r["offs"].cpu().numpy()
     total = offs[wl.E]
     real = r["por"].cpu().numpy()[:total] >= 0
@@ -80,9 +81,11 @@ def test_fp8_expert_ffn_unit_scales(E, K, T, H, I):
     _check_vs_oracle(wl, d, ids, r, y)
 
 
-@pytest.mark.parametrize("E,K,T,H,I", [(1, 1, 200, 256, 256), (6, 2, 500, 512, 384), (16, 4, 300, 1024, 768)])
-def test_fp8_expert_ffn_block_scales(E, K, T, H, I):
-    wl = W.Workload("f8", T=T, H=H, I=I, E=E, K=K, dtype=W.DTYPE_FP8)
+@pytest.mark.parametrize("E,K,T,H,I,bm", [(1, 1, 200, 256, 256, 0), (6, 2, 500, 512, 384, 0),
+                                          (16, 4, 300, 1024, 768, 0), (1, 1, 300, 256, 256, 256),
+                                          (6, 2, 700, 512, 384, 256), (3, 3, 600, 1024, 768, 256)])
+def test_fp8_expert_ffn_block_scales(E, K, T, H, I, bm):
+    wl = W.Workload("f8", T=T, H=H, I=I, E=E, K=K, dtype=W.DTYPE_FP8, block_m=bm)
     d = inputs.make_inputs(wl, seed=4, device="cuda")
     rng = np.random.default_rng(4)
     ids = np.stack([rng.choice(E, K, replace=False) for _ in range(T)]).astype(np.int32)
@@ -93,8 +96,9 @@ def test_fp8_expert_ffn_block_scales(E, K, T, H, I):
 SMALL_FP8 = W.SKEWED_FP8.with_(name="skewed_fp8_small", T=600, H=512, I=384, E=16, K=4)
 
 
-def test_fp8_layer_small_all_elements():
-    wl = SMALL_FP8
+@pytest.mark.parametrize("bm", [0, 256])
+def test_fp8_layer_small_all_elements(bm):
+    wl = SMALL_FP8.with_(block_m=bm)
     d = inputs.make_inputs(wl, seed=0, device="cuda")
     res = P.run_layer(wl, d)
     assert B.moe_get_device_status(res["ws"]) == 0

@@ -24,6 +24,10 @@ SMALL = {
                                              I_shared=256),
     "one_token": W.MIXTRAL_PREFILL.with_(name="one_token", T=1, H=256, I=128, E=4, K=2),
     "dense_like": W.TINY.with_(name="dense_like", T=300, E=1, K=1),
+    # buckets aligned to 256 rows: the two-SM (cta_group::2) GEMMs
+    "mixtral_small_pair": W.MIXTRAL_PREFILL.with_(name="mixtral_small_pair", T=1000, H=512, I=384, block_m=256),
+    "dsv3_small_pair": W.DSV3_PREFILL.with_(name="dsv3_small_pair", T=300, H=512, I=256, E=32, I_shared=256,
+                                            block_m=256),
 }
 
 

@@ -89,7 +89,8 @@ def _permute(wl, ids_np, x=None):
 
 
 def _check_perm(wl, ids_np, r):
-    P.check_permutation(ids_np, wl.E, r["counts"], r["offs"], r["rop"], r["por"])
+    P.check_permutation(ids_np, wl.E, r["counts"], r["offs"], r["rop"], r["por"],
+                        B.moe_effective_block_m(B.params(wl)))
     total = r["offs"][wl.E]
     por = r["por"][:total]
     real = por >= 0
@@ -99,9 +100,9 @@ def _check_perm(wl, ids_np, r):
     assert (xp[torch.as_tensor(np.where(~real)[0], device="cuda")] == 0).all()
 
 
-@pytest.mark.parametrize("seed", [0, 1])
-def test_permute_random(seed):
-    wl = W.Workload("perm", T=3000, H=256, I=128, E=64, K=6)
+@pytest.mark.parametrize("seed,block_m", [(0, 0), (1, 0), (2, 256)])
+def test_permute_random(seed, block_m):
+    wl = W.Workload("perm", T=3000, H=256, I=128, E=64, K=6, block_m=block_m)
     rng = np.random.default_rng(seed)
     ids = np.stack([rng.choice(wl.E, wl.K, replace=False) for _ in range(wl.T)]).astype(np.int32)
     r = _permute(wl, ids)
@@ -153,10 +154,12 @@ def test_permute_bad_ids_are_reported_and_skipped():
 
 
 # ------------------------------------------------------------------ expert FFN
-@pytest.mark.parametrize("E,K,T,H,I", [(1, 1, 300, 256, 128), (6, 2, 700, 384, 256),
-                                       (16, 4, 64, 512, 384), (3, 3, 129, 1024, 640)])
-def test_expert_ffn_grouped_gemm(E, K, T, H, I):
-    wl = W.Workload("ffn", T=T, H=H, I=I, E=E, K=K)
+@pytest.mark.parametrize("E,K,T,H,I,bm", [(1, 1, 300, 256, 128, 0), (6, 2, 700, 384, 256, 0),
+                                          (16, 4, 64, 512, 384, 0), (3, 3, 129, 1024, 640, 0),
+                                          (1, 1, 300, 256, 128, 256), (6, 2, 700, 512, 256, 256),
+                                          (3, 3, 700, 384, 640, 256)])
+def test_expert_ffn_grouped_gemm(E, K, T, H, I, bm):
+    wl = W.Workload("ffn", T=T, H=H, I=I, E=E, K=K, block_m=bm)
     d = inputs.make_inputs(wl, seed=5, device="cuda")
     rng = np.random.default_rng(5)
     ids = np.stack([rng.choice(E, K, replace=False) for _ in range(T)]).astype(np.int32)
@@ -165,7 +168,8 @@ def test_expert_ffn_grouped_gemm(E, K, T, H, I):
     rows = B.moe_max_padded_rows(p)
     offs = torch.as_tensor(r["offs"], device="cuda")
     counts = torch.as_tensor(r["counts"], device="cuda")
-    ref, _ = o.expert_outputs(P.f64(d["x"]), ids, P.expert_weights_fn(d, wl), E, BM, h_format="bf16")
+    ref, _ = o.expert_outputs(P.f64(d["x"]), ids, P.expert_weights_fn(d, wl), E,
+                              B.moe_effective_block_m(p), h_format="bf16")
     total = r["offs"][E]
     real = r["por"][:total] >= 0
     # with counts: pad rows are left untouched; without: they are computed (zero input -> 0)
