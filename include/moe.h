@@ -78,8 +78,8 @@ typedef struct moe_params {
   int32_t I_shared;     /* intermediate size of the shared expert, 0 = none              */
   int32_t dtype;        /* MOE_DTYPE_BF16 or MOE_DTYPE_FP8_E4M3                          */
   int32_t block_m;      /* row alignment of each expert's bucket: 128 (one-SM GEMM tiles), */
-                        /* 256 (two-SM cta_group::2 tiles), 0 = choose: 256 when buckets */
-                        /* average >= 512 rows (T*K >= 512*E), else 128                  */
+                        /* 256 (two-SM cta_group::2 tiles: a third less SM-side operand  */
+                        /* traffic, more pad rows), 0 = default (128)                    */
 } moe_params_t;
 
 /* ---------------------------------------------------------------------------------- */

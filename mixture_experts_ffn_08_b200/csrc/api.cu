@@ -71,12 +71,11 @@ struct Layout {
 
 bool is_fp8(const moe_params_t* p) { return p->dtype == MOE_DTYPE_FP8_E4M3; }
 
-// Bucket alignment: 256 rows (two-SM GEMMs) when buckets average at least 512 rows, where
-// the extra padding is small against the traffic the pair tiles save; else 128.
-int block_m_of(const moe_params_t* p) {
-  if (p->block_m != 0) return p->block_m;
-  return static_cast<long long>(p->T) * p->K >= 512LL * p->E ? kBlockM2 : kBlockM;
-}
+// Bucket alignment: 128 rows (one-SM GEMM tiles) unless the caller asks for 256 (two-SM
+// cta_group::2 tiles).  Measured on B200, the pair tiles' third less SM-side traffic did
+// not pay for the extra pad rows that 256-row buckets add (about 6% more MMA work on the
+// Mixtral and FP8 skew shapes), so they are opt-in.
+int block_m_of(const moe_params_t* p) { return p->block_m != 0 ? p->block_m : kBlockM; }
 
 Layout layout(const moe_params_t* p) {
   Layout L{};

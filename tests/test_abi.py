@@ -54,7 +54,7 @@ def test_sizes(lib):
         p = B.params(wl)
         rows = B.moe_max_padded_rows(p)
         bm = B.moe_effective_block_m(p)
-        assert bm == (256 if wl.T * wl.K >= 512 * wl.E else 128)
+        assert bm == 128 and B.moe_effective_block_m(B.params(wl.with_(block_m=256))) == 256
         assert rows == wl.T * wl.K + wl.E * (bm - 1)
         ws = B.moe_workspace_size(p)
         assert ws >= rows * wl.H * (1 if wl.dtype else 2) * 2
