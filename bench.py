@@ -85,6 +85,10 @@ def _describe(wl):
     s += f" renorm x{wl.routed_scale:g}" if wl.renormalize else f" x{wl.routed_scale:g}"
     if wl.I_shared:
         s += f" +shared I={wl.I_shared}"
+    if wl.fused_combine:
+        s += " fused-combine"
+    if wl.block_m:
+        s += f" block_m={wl.block_m}"
     return s + (" fp8" if wl.dtype else " bf16")
 
 
@@ -205,6 +209,10 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     wl = {**W.ALL, **W.PROFILE}[args.workload]
+    if args.fused_combine:
+        wl = wl.with_(fused_combine=True)
+    if args.block_m:
+        wl = wl.with_(block_m=args.block_m)
     p = B.params(wl)
     d = inputs.make_inputs(wl, seed=rank, device="cuda")
     fp8 = wl.dtype == W.DTYPE_FP8
@@ -471,6 +479,10 @@ def main():
     ap.add_argument("--workload", default="mixtral_prefill", choices=sorted(W.ALL) + sorted(W.PROFILE))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fused-combine", action="store_true",
+                    help="down projection adds into the output with fp32 atomics (non-deterministic)")
+    ap.add_argument("--block-m", type=int, default=0, choices=[0, 128, 256],
+                    help="bucket alignment: 256 selects the two-SM (cta_group::2) GEMM tiles")
     ap.add_argument("--micro", choices=["grouped_topk"], default=None,
                     help="time one stage alone instead of the layer")
     args = ap.parse_args()

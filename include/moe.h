@@ -45,7 +45,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 1
+#define MOE_ABI_VERSION 2
 
 typedef enum moe_status {
   MOE_OK = 0,
@@ -80,6 +80,10 @@ typedef struct moe_params {
   int32_t block_m;      /* row alignment of each expert's bucket: 128 (one-SM GEMM tiles), */
                         /* 256 (two-SM cta_group::2 tiles: a third less SM-side operand  */
                         /* traffic, more pad rows), 0 = default (128)                    */
+  int32_t fused_combine; /* moe_layer_forward only, bf16, block_m 128: 0 = separate,     */
+                        /* deterministic combine (default); 1 = the down projection adds */
+                        /* w * y straight into an fp32 token accumulator with atomic     */
+                        /* vector reductions (no y_perm round trip; run-to-run bits vary)*/
 } moe_params_t;
 
 /* ---------------------------------------------------------------------------------- */

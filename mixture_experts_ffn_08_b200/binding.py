@@ -43,13 +43,14 @@ class MoeParams(ctypes.Structure):
                 ("topk_group", ctypes.c_int32), ("group_topn", ctypes.c_int32),
                 ("score_fn", ctypes.c_int32), ("renormalize", ctypes.c_int32),
                 ("routed_scale", ctypes.c_float), ("I_shared", ctypes.c_int32),
-                ("dtype", ctypes.c_int32), ("block_m", ctypes.c_int32)]
+                ("dtype", ctypes.c_int32), ("block_m", ctypes.c_int32),
+                ("fused_combine", ctypes.c_int32)]
 
 
 def params(wl: W.Workload) -> MoeParams:
     return MoeParams(wl.T, wl.H, wl.I, wl.E, wl.K, wl.n_group, wl.topk_group, wl.group_topn,
                      wl.score_fn, int(wl.renormalize), float(wl.routed_scale), wl.I_shared,
-                     wl.dtype, wl.block_m)
+                     wl.dtype, wl.block_m, int(wl.fused_combine))
 
 
 _P = ctypes.c_void_p

@@ -104,7 +104,7 @@ Layout layout(const moe_params_t* p) {
   L.h = take(rows_t * I * 2);
   L.y_perm = take(rows * H * 4);
   L.h_sh = take(T * static_cast<long long>(p->I_shared) * 2);
-  L.y_sh = take(p->I_shared > 0 ? T * H * 4 : 0);
+  L.y_sh = take(p->I_shared > 0 || p->fused_combine ? T * H * 4 : 0);  // also the fused-combine accumulator
   const bool f8 = is_fp8(p);
   L.x_atoms = take(f8 ? rows_t * (H / 128) * 4 : 0);
   L.h_atoms = take(f8 ? rows_t * (I / 128) * 4 : 0);
@@ -141,6 +141,8 @@ moe_status_t validate(const moe_params_t* p) {
   if (p->H % 128 != 0 || p->I % 128 != 0 || p->I_shared % 128 != 0) return MOE_ERR_UNSUPPORTED;
   if (p->block_m != 0 && p->block_m != kBlockM && p->block_m != kBlockM2) return MOE_ERR_UNSUPPORTED;
   if (p->dtype == MOE_DTYPE_FP8_E4M3 && p->I_shared > 0) return MOE_ERR_UNSUPPORTED;
+  if (p->fused_combine != 0 && p->fused_combine != 1) return MOE_ERR_INVALID_ARG;
+  if (p->fused_combine && (p->dtype != MOE_DTYPE_BF16 || p->block_m == kBlockM2)) return MOE_ERR_UNSUPPORTED;
   const long long rows = static_cast<long long>(p->T) * p->K + static_cast<long long>(p->E) * (kBlockM2 - 1);
   if (rows >= (1LL << 31) / 2) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
@@ -266,6 +268,20 @@ moe_status_t do_layer(const moe_params_t* p, const void* x, const float* x_scale
   MOE_TRY(do_route(p, x, x_scale, w_r, bias, ids, w, ws, st));
   MOE_TRY(do_permute(p, ids, x, x_scale, counts, offsets, rop, at<int32_t>(ws, L.pair_of_row),
                      at<void>(ws, L.x_perm), at<float>(ws, L.x_perm_scale), ws, st));
+  if (p->fused_combine) {
+    // acc starts as the shared expert's output (or zero); the routed down projection adds
+    // w * y of every pair into it; one pass rounds it to bf16
+    float* acc = at<float>(ws, L.y_sh);
+    if (p->I_shared > 0) MOE_TRY(do_shared(p, x, wsg, wsu, wsd, acc, ws, st));
+    else MOE_CUDA(cudaMemsetAsync(acc, 0, static_cast<size_t>(p->T) * p->H * sizeof(float), st));
+    int32_t* status = at<int32_t>(ws, L.status);
+    void* h = at<void>(ws, L.h);
+    MOE_CUDA(gemm_gateup_swiglu(at<void>(ws, L.x_perm), L.max_rows, offsets, counts, p->E, 0, w_gate, w_up,
+                                p->I, p->H, h, status, MOE_K_GATEUP, st));
+    MOE_CUDA(gemm_down_combine(h, L.max_rows, offsets, counts, p->E, w_down, p->H, p->I,
+                               at<int32_t>(ws, L.pair_of_row), w, p->K, acc, status, st));
+    return cuda_status(launch_f32_to_bf16(acc, static_cast<long long>(p->T) * p->H, out, st));
+  }
   if (is_fp8(p))
     MOE_TRY(do_expert_ffn_fp8(p, at<void>(ws, L.x_perm), at<float>(ws, L.x_perm_scale), offsets, counts,
                               w_gate, w_up, w_down, wgs, wus, wds, y_perm, ws, st));

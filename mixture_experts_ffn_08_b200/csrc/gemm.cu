@@ -152,4 +152,34 @@ cudaError_t gemm_down(const void* A, int64_t a_rows, const int32_t* offsets,
   return launch<Cfg>(ta, tb, tb, gp, ceil_div(a_rows, 128) * ceil_div(N, 128), kid, st);
 }
 
+cudaError_t gemm_down_combine(const void* A, int64_t a_rows, const int32_t* offsets, const int32_t* counts,
+                              int G, const void* w, int N, int K, const int32_t* pair_of_row,
+                              const float* pair_weight, int topk, float* acc, int32_t* status, cudaStream_t st) {
+  CUtensorMap ta, tb;
+  const bool wide = N % 256 == 0;
+  if (!make_tmap_bf16(&ta, A, a_rows, K, 128) ||
+      !make_tmap_bf16(&tb, w, static_cast<uint64_t>(G) * N, K, wide ? 256 : 128))
+    return cudaErrorInvalidValue;
+  GemmParams gp{};
+  gp.offsets = offsets;
+  gp.counts = counts;
+  gp.G = G;
+  gp.dense_rows = 0;
+  gp.K = K;
+  gp.N = N;
+  gp.b_rows_per_group = N;
+  gp.out = acc;
+  gp.ldo = N;
+  gp.status = status;
+  gp.pair_of_row = pair_of_row;
+  gp.pair_weight = pair_weight;
+  gp.topk = topk;
+  if (wide) {
+    using Cfg = GemmCfg<256, EPI_COMBINE, 4>;
+    return launch<Cfg>(ta, tb, tb, gp, ceil_div(a_rows, 128) * ceil_div(N, 256), MOE_K_DOWN, st);
+  }
+  using Cfg = GemmCfg<128, EPI_COMBINE, 6>;
+  return launch<Cfg>(ta, tb, tb, gp, ceil_div(a_rows, 128) * ceil_div(N, 128), MOE_K_DOWN, st);
+}
+
 }  // namespace moe

@@ -57,6 +57,14 @@ cudaError_t gemm_down(const void* A, int64_t a_rows, const int32_t* offsets,
                       const int32_t* counts, int G, int dense_rows, const void* w, int N, int K,
                       float* y, int32_t* status, int kid, cudaStream_t st);
 
+// acc[t] += w[p] * (A W^T)[r] for every bucket row r of pair p = pair_of_row[r], t = p / topk
+// (down projection fused with the combine; fp32 vector reductions, order not fixed).
+cudaError_t gemm_down_combine(const void* A, int64_t a_rows, const int32_t* offsets, const int32_t* counts,
+                              int G, const void* w, int N, int K, const int32_t* pair_of_row,
+                              const float* pair_weight, int topk, float* acc, int32_t* status, cudaStream_t st);
+// out[i] = bf16(acc[i]) for n values (n multiple of 8).
+cudaError_t launch_f32_to_bf16(const float* acc, long long n, void* out, cudaStream_t st);
+
 // ---------------------------------------------------------------- FP8 GEMMs (gemm_fp8.cu)
 // fp32 power-of-two scales -> 512-byte UE8M0 scale atoms (see tc_gemm_fp8.cuh).
 cudaError_t launch_sf_rows_to_atoms(const float* scales, int nk, const int32_t* offsets, int G,

@@ -471,6 +471,26 @@ __global__ void __launch_bounds__(128) combine_kernel(
   }
 }
 
+__global__ void f32_to_bf16_kernel(const float* __restrict__ acc, long long n8, __nv_bfloat16* __restrict__ out) {
+  for (long long v = blockIdx.x * (long long)blockDim.x + threadIdx.x; v < n8; v += (long long)gridDim.x * blockDim.x) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(acc) + 2 * v);
+    const float4 b = __ldg(reinterpret_cast<const float4*>(acc) + 2 * v + 1);
+    reinterpret_cast<uint4*>(out)[v] = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w),
+                                                  pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
+  }
+}
+
+cudaError_t launch_f32_to_bf16(const float* acc, long long n, void* out, cudaStream_t st) {
+  const long long n8 = n / 8;
+  if (n8 == 0) return cudaSuccess;
+  const long long want = (n8 + 255) / 256;
+  const int grid = static_cast<int>(want < num_sms() * 8LL ? want : num_sms() * 8LL);
+  trace_before(MOE_K_COMBINE, st);
+  f32_to_bf16_kernel<<<grid, 256, 0, st>>>(acc, n8, static_cast<__nv_bfloat16*>(out));
+  trace_after(MOE_K_COMBINE, st);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_combine(const moe_params_t& p, const void* y_perm, const int32_t* row_of_pair,
                            const float* w, const float* y_shared, void* out, cudaStream_t st) {
   if (p.T == 0) return cudaSuccess;

@@ -28,6 +28,11 @@
 //                           h = SiLU(gate) * up, rounded to bf16
 //                EPI_F32    store fp32 (router logits, down-projection outputs),
 //                           columns >= N dropped
+//                EPI_COMBINE down projection fused with the combine: each row r of a
+//                           bucket is pair p = pair_of_row[r] of token t = p / K, and
+//                           w[p] * y[r] is added to the fp32 token accumulator
+//                           acc[t] with vector reductions (order of the K additions,
+//                           and so the last bits, vary from run to run)
 //
 // Every wait on an mbarrier is bounded; on timeout the CTA sets MOE_DEV_TIMEOUT in the
 // status word, drains the copies and MMAs it issued, frees TMEM and exits.
@@ -37,7 +42,7 @@
 
 namespace moe {
 
-enum EpiKind { EPI_BF16 = 0, EPI_SWIGLU = 1, EPI_F32 = 2 };
+enum EpiKind { EPI_BF16 = 0, EPI_SWIGLU = 1, EPI_F32 = 2, EPI_COMBINE = 3 };
 
 struct GemmParams {
   const int32_t* offsets;  // [G+1] first row of each group (multiples of 128); nullptr: dense
@@ -51,7 +56,16 @@ struct GemmParams {
   void* out;               // [rows, ldo] bf16 or fp32
   int64_t ldo;             // leading dimension of out, in elements
   int32_t* status;         // device status word (may be null)
+  const int32_t* pair_of_row;  // EPI_COMBINE: pair of each bucket row
+  const float* pair_weight;    // EPI_COMBINE: combine weight of each pair [T*K]
+  int topk;                    // EPI_COMBINE: K (pair p belongs to token p / K)
 };
+
+MOE_DEVINL void red_add_v4(float* addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d, float w) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(w * __uint_as_float(a)),
+               "f"(w * __uint_as_float(b)), "f"(w * __uint_as_float(c)), "f"(w * __uint_as_float(d))
+               : "memory");
+}
 
 template <int BN_, int EPI_, int STAGES_>
 struct GemmCfg {
@@ -267,6 +281,21 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 #pragma unroll
             for (int v = 0; v < 4; ++v)
               dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+          }
+        }
+      } else if constexpr (Cfg::EPI == EPI_COMBINE) {
+        int pair = -1;
+        if (row_ok) pair = __ldg(p.pair_of_row + row);
+        const float wgt = pair >= 0 ? __ldg(p.pair_weight + pair) : 0.f;
+        float* out = static_cast<float*>(p.out) + static_cast<long long>(pair >= 0 ? pair / p.topk : 0) * p.ldo + col0;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tbase + c, r);
+          tmem_ld_wait();
+          if (pair >= 0 && col0 + c < p.N) {
+#pragma unroll
+            for (int v = 0; v < 8; ++v) red_add_v4(out + c + 4 * v, r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3], wgt);
           }
         }
       } else if constexpr (Cfg::EPI == EPI_BF16) {

@@ -38,6 +38,7 @@ class Workload:
     dtype: int = DTYPE_BF16
     skewed: bool = False    # Zipf-shaped router for the skew stress case
     block_m: int = 0        # bucket row alignment: 128, 256 (two-SM GEMM tiles), 0 = library choice
+    fused_combine: bool = False  # down projection adds into the output (atomic, non-deterministic)
 
     @property
     def P(self) -> int:

@@ -28,6 +28,11 @@ SMALL = {
     "mixtral_small_pair": W.MIXTRAL_PREFILL.with_(name="mixtral_small_pair", T=1000, H=512, I=384, block_m=256),
     "dsv3_small_pair": W.DSV3_PREFILL.with_(name="dsv3_small_pair", T=300, H=512, I=256, E=32, I_shared=256,
                                             block_m=256),
+    # down projection fused with the combine (fp32 atomic accumulation)
+    "mixtral_small_fused": W.MIXTRAL_PREFILL.with_(name="mixtral_small_fused", T=1000, H=512, I=384,
+                                                   fused_combine=True),
+    "dsv3_small_fused": W.DSV3_PREFILL.with_(name="dsv3_small_fused", T=200, H=384, I=256, E=32, I_shared=256,
+                                             fused_combine=True),
 }
 
 
@@ -63,12 +68,12 @@ def test_layer_is_deterministic():
         assert torch.equal(again["ids"], first["ids"])
 
 
-FULL = ["mixtral_prefill", "dsv3_prefill", "dsv3_decode"]
+FULL = ["mixtral_prefill", "dsv3_prefill", "dsv3_decode", "dsv3_prefill_fused"]
 
 
 @pytest.mark.parametrize("name", FULL)
 def test_layer_full_size_sampled(name):
-    wl = W.ALL[name]
+    wl = W.ALL[name] if name in W.ALL else W.ALL[name[:-len("_fused")]].with_(fused_combine=True)
     d = inputs.make_inputs(wl, seed=0, device="cuda")
     r = P.run_layer(wl, d)
     assert B.moe_get_device_status(r["ws"]) == 0
