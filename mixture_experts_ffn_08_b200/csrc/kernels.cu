@@ -82,7 +82,16 @@ MOE_DEVINL float warp_max(float v) {
   return v;
 }
 
-// Lane l holds experts l, l+32, l+64, ... (EPL of them): E <= 32 * EPL.
+// Lane l holds experts l, l+32, l+64, ... (EPL of them): E <= 32 * EPL, so register j
+// of all lanes covers experts [32j, 32j+32).
+//
+// Group stage: when every group is a whole number of registers (group size a multiple
+// of 32) and the group score uses at most the two best experts, all group scores come
+// out of one butterfly that carries each register's top-2 across the warp, the groups'
+// registers merged in parallel; every lane then ranks the groups itself.  Any other
+// grouping takes the general path (one warp argmax per group and rank).
+// Top-K: each lane sorts its EPL candidates (descending score, ascending expert id), so
+// every one of the K rounds is a single warp argmax over the lanes' heads.
 template <int EPL>
 __global__ void __launch_bounds__(128) topk_kernel(
     const float* __restrict__ logits, int T, int E, int K, int n_group, int topk_group,
@@ -125,53 +134,111 @@ __global__ void __launch_bounds__(128) topk_kernel(
 
   if (n_group > 1) {
     const int gs = E / n_group;
-    float my_gscore = -CUDART_INF_F;  // lane g keeps the score of group g
-    for (int g = 0; g < n_group; ++g) {
-      uint32_t taken = 0;
-      float acc = 0.f;
-      for (int r = 0; r < group_topn; ++r) {
-        float bv = -CUDART_INF_F;
-        int bi = 0x7fffffff;
+    uint32_t keep = 0;
+    if (gs % 32 == 0 && group_topn <= 2) {
+      // top-2 of every register across the warp, all registers at once
+      float t1[EPL], t2[EPL];
+#pragma unroll
+      for (int j = 0; j < EPL; ++j) { t1[j] = c[j]; t2[j] = -CUDART_INF_F; }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
 #pragma unroll
         for (int j = 0; j < EPL; ++j) {
-          const int e = j * 32 + lane;
-          if (e < E && e / gs == g && !((taken >> j) & 1u) && better(c[j], e, bv, bi)) {
-            bv = c[j];
-            bi = e;
+          const float b1 = __shfl_xor_sync(kFull, t1[j], o);
+          const float b2 = __shfl_xor_sync(kFull, t2[j], o);
+          const float hi = fmaxf(t1[j], b1);
+          t2[j] = fmaxf(fminf(t1[j], b1), fmaxf(t2[j], b2));
+          t1[j] = hi;
+        }
+      }
+      // group g spans registers [g*R, (g+1)*R); merge their top-2 lists
+      // here every group is at least one register, so n_group <= EPL
+      const int R = gs / 32;
+      float gscore[EPL];
+#pragma unroll
+      for (int g = 0; g < EPL; ++g) {
+        float a1 = -CUDART_INF_F, a2 = -CUDART_INF_F;
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) {
+          if (j / R == g) {
+            const float hi = fmaxf(a1, t1[j]);
+            a2 = fmaxf(fminf(a1, t1[j]), fmaxf(a2, t2[j]));
+            a1 = hi;
           }
         }
-        warp_argmax(bv, bi);
-        acc += bv;
-        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+        gscore[g] = g < n_group ? (group_topn == 1 ? a1 : a1 + a2) : -CUDART_INF_F;
       }
-      if (lane == g) my_gscore = acc;
-    }
-    uint32_t keep = 0;
-    float cand = lane < n_group ? my_gscore : -CUDART_INF_F;
-    for (int r = 0; r < topk_group; ++r) {
-      float bv = cand;
-      int bi = lane;
-      warp_argmax(bv, bi);
-      keep |= 1u << bi;
-      if (lane == bi) cand = -CUDART_INF_F;
-    }
+      // rank the groups in registers (all lanes agree): best score, lower index on ties
+      for (int r = 0; r < topk_group; ++r) {
+        int best = -1;
+        float bv = -CUDART_INF_F;
 #pragma unroll
-    for (int j = 0; j < EPL; ++j) {
-      const int e = j * 32 + lane;
-      if (e < E && !((keep >> (e / gs)) & 1u)) c[j] = -CUDART_INF_F;
+        for (int g = 0; g < EPL; ++g)
+          if (g < n_group && !((keep >> g) & 1u) && (best < 0 || gscore[g] > bv)) { bv = gscore[g]; best = g; }
+        keep |= 1u << best;
+      }
+#pragma unroll
+      for (int j = 0; j < EPL; ++j)
+        if (j * 32 < E && !((keep >> (j / R)) & 1u)) c[j] = -CUDART_INF_F;
+    } else {
+      int grp[EPL];
+#pragma unroll
+      for (int j = 0; j < EPL; ++j) grp[j] = (j * 32 + lane) / gs;
+      float my_gscore = -CUDART_INF_F;  // lane g keeps the score of group g
+      for (int g = 0; g < n_group; ++g) {
+        uint32_t taken = 0;
+        float acc = 0.f;
+        for (int r = 0; r < group_topn; ++r) {
+          float bv = -CUDART_INF_F;
+          int bi = 0x7fffffff;
+#pragma unroll
+          for (int j = 0; j < EPL; ++j) {
+            const int e = j * 32 + lane;
+            if (e < E && grp[j] == g && !((taken >> j) & 1u) && better(c[j], e, bv, bi)) {
+              bv = c[j];
+              bi = e;
+            }
+          }
+          warp_argmax(bv, bi);
+          acc += bv;
+          if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+        }
+        if (lane == g) my_gscore = acc;
+      }
+      float cand = lane < n_group ? my_gscore : -CUDART_INF_F;
+      for (int r = 0; r < topk_group; ++r) {
+        float bv = cand;
+        int bi = lane;
+        warp_argmax(bv, bi);
+        keep |= 1u << bi;
+        if (lane == bi) cand = -CUDART_INF_F;
+      }
+#pragma unroll
+      for (int j = 0; j < EPL; ++j)
+        if (j * 32 + lane < E && !((keep >> grp[j]) & 1u)) c[j] = -CUDART_INF_F;
     }
   }
 
+  // sort this lane's candidates: descending c, ascending expert id (insertion network)
+  float sc[EPL];
+  int se[EPL];
+#pragma unroll
+  for (int j = 0; j < EPL; ++j) { sc[j] = c[j]; se[j] = j * 32 + lane; }
+#pragma unroll
+  for (int a = 1; a < EPL; ++a) {
+#pragma unroll
+    for (int b = a; b > 0; --b) {
+      if (better(sc[b], se[b], sc[b - 1], se[b - 1])) {
+        const float tv = sc[b]; sc[b] = sc[b - 1]; sc[b - 1] = tv;
+        const int te = se[b]; se[b] = se[b - 1]; se[b - 1] = te;
+      }
+    }
+  }
   int my_id = -1;
   float my_w = 0.f;
   for (int k = 0; k < K; ++k) {
-    float bv = -CUDART_INF_F;
-    int bi = 0x7fffffff;
-#pragma unroll
-    for (int j = 0; j < EPL; ++j) {
-      const int e = j * 32 + lane;
-      if (e < E && better(c[j], e, bv, bi)) { bv = c[j]; bi = e; }
-    }
+    float bv = sc[0];
+    int bi = se[0];
     warp_argmax(bv, bi);
     const int owner = bi & 31, jj = bi >> 5;
     float sv = 0.f;
@@ -179,10 +246,11 @@ __global__ void __launch_bounds__(128) topk_kernel(
     for (int j = 0; j < EPL; ++j)
       if (j == jj) sv = s[j];
     sv = __shfl_sync(kFull, sv, owner);
-    if (lane == owner) {
+    if (lane == owner) {   // pop the head
 #pragma unroll
-      for (int j = 0; j < EPL; ++j)
-        if (j == jj) c[j] = -CUDART_INF_F;
+      for (int j = 0; j < EPL - 1; ++j) { sc[j] = sc[j + 1]; se[j] = se[j + 1]; }
+      sc[EPL - 1] = -CUDART_INF_F;
+      se[EPL - 1] = 0x7fffffff;
     }
     if (lane == k) { my_id = bi; my_w = sv; }
   }
