@@ -106,11 +106,13 @@ Layout layout(const moe_params_t* p) {
   L.h_sh = take(T * static_cast<long long>(p->I_shared) * 2);
   L.y_sh = take(p->I_shared > 0 || p->fused_combine ? T * H * 4 : 0);  // also the fused-combine accumulator
   const bool f8 = is_fp8(p);
-  L.x_atoms = take(f8 ? rows_t * (H / 128) * 4 : 0);
-  L.h_atoms = take(f8 ? rows_t * (I / 128) * 4 : 0);
-  L.wg_atoms = take(f8 ? E * (I / 128) * (H / 128) * 512 : 0);
-  L.wu_atoms = take(f8 ? E * (I / 128) * (H / 128) * 512 : 0);
-  L.wd_atoms = take(f8 ? E * (H / 128) * (I / 128) * 512 : 0);
+  // e4m3 scale atoms: 512 bytes per 128 rows and 4 K blocks of 128
+  const long long hk4 = (H / 128 + 3) / 4, ik4 = (I / 128 + 3) / 4;
+  L.x_atoms = take(f8 ? rows_t / 128 * hk4 * 512 : 0);
+  L.h_atoms = take(f8 ? rows_t / 128 * ik4 * 512 : 0);
+  L.wg_atoms = take(f8 ? E * (I / 128) * hk4 * 512 : 0);
+  L.wu_atoms = take(f8 ? E * (I / 128) * hk4 * 512 : 0);
+  L.wd_atoms = take(f8 ? E * (H / 128) * ik4 * 512 : 0);
   L.total = o;
   L.x_stage = take(T * H * xelem);
   L.x_scale_stage = take(is_fp8(p) ? T * (H / 128) * 4 : 0);
@@ -198,10 +200,11 @@ moe_status_t do_expert_ffn_fp8(const moe_params_t* p, const void* x_perm, const 
                                cudaStream_t st) {
   const Layout L = layout(p);
   int32_t* status = at<int32_t>(ws, L.status);
-  const long long nb_gu = static_cast<long long>(p->E) * (p->I / 128) * (p->H / 128);
-  MOE_CUDA(launch_sf_blocks_to_atoms(wgs, nb_gu, at<uint8_t>(ws, L.wg_atoms), st));
-  MOE_CUDA(launch_sf_blocks_to_atoms(wus, nb_gu, at<uint8_t>(ws, L.wu_atoms), st));
-  MOE_CUDA(launch_sf_blocks_to_atoms(wds, nb_gu, at<uint8_t>(ws, L.wd_atoms), st));
+  const long long rows_gu = static_cast<long long>(p->E) * (p->I / 128);   // 128-row weight blocks
+  const long long rows_d = static_cast<long long>(p->E) * (p->H / 128);
+  MOE_CUDA(launch_sf_blocks_to_atoms(wgs, rows_gu, p->H / 128, at<uint8_t>(ws, L.wg_atoms), st));
+  MOE_CUDA(launch_sf_blocks_to_atoms(wus, rows_gu, p->H / 128, at<uint8_t>(ws, L.wu_atoms), st));
+  MOE_CUDA(launch_sf_blocks_to_atoms(wds, rows_d, p->I / 128, at<uint8_t>(ws, L.wd_atoms), st));
   MOE_CUDA(launch_sf_rows_to_atoms(x_perm_scale, p->H / 128, offsets, p->E, L.max_rows,
                                    at<uint8_t>(ws, L.x_atoms), st));
   void* h = at<void>(ws, L.h);

@@ -127,12 +127,13 @@ cudaError_t gemm_pair_gateup_swiglu_fp8(const void* A, const uint8_t* a_atoms, i
                                         cudaStream_t st) {
   using Cfg = Pair2Cfg<256, EPI2_SWIGLU_E4M3, 6, true>;
   const uint64_t m_tiles = static_cast<uint64_t>(cdiv2(a_rows, 256) * 2);
-  const uint64_t w_atoms = static_cast<uint64_t>(G) * (N / 128) * (K / 128);
+  const uint64_t kb4 = (K / 128 + 3) / 4;
+  const uint64_t w_atoms = static_cast<uint64_t>(G) * (N / 128) * kb4;
   CUtensorMap ta, tg, tu, tsa, tsg, tsu;
   if (!tmap_rows128(&ta, A, true, a_rows, K, 128) ||
       !tmap_rows128(&tg, w_gate, true, static_cast<uint64_t>(G) * N, K, 128) ||
       !tmap_rows128(&tu, w_up, true, static_cast<uint64_t>(G) * N, K, 128) ||
-      !tmap_atoms(&tsa, a_atoms, m_tiles * (K / 128)) || !tmap_atoms(&tsg, gate_atoms, w_atoms) ||
+      !tmap_atoms(&tsa, a_atoms, m_tiles * kb4) || !tmap_atoms(&tsg, gate_atoms, w_atoms) ||
       !tmap_atoms(&tsu, up_atoms, w_atoms))
     return cudaErrorInvalidValue;
   const Pair2Params pp = pair_params(offsets, counts, G, K, N, h, h_atoms, status);
@@ -144,11 +145,12 @@ cudaError_t gemm_pair_down_fp8(const void* A, const uint8_t* a_atoms, int64_t a_
                                void* y, int32_t* status, cudaStream_t st) {
   using Cfg = Pair2Cfg<128, EPI2_BF16, 8, true>;
   const uint64_t m_tiles = static_cast<uint64_t>(cdiv2(a_rows, 256) * 2);
-  const uint64_t n_w_atoms = static_cast<uint64_t>(G) * (N / 128) * (K / 128);
+  const uint64_t kb4 = (K / 128 + 3) / 4;
+  const uint64_t n_w_atoms = static_cast<uint64_t>(G) * (N / 128) * kb4;
   CUtensorMap ta, tb, tsa, tsb;
   if (!tmap_rows128(&ta, A, true, a_rows, K, 128) ||
       !tmap_rows128(&tb, w, true, static_cast<uint64_t>(G) * N, K, 64) ||
-      !tmap_atoms(&tsa, a_atoms, m_tiles * (K / 128)) || !tmap_atoms(&tsb, w_atoms, n_w_atoms))
+      !tmap_atoms(&tsa, a_atoms, m_tiles * kb4) || !tmap_atoms(&tsb, w_atoms, n_w_atoms))
     return cudaErrorInvalidValue;
   const Pair2Params pp = pair_params(offsets, counts, G, K, N, y, nullptr, status);
   return launch_pair<Cfg>(ta, tb, tb, tsa, tsb, tsb, pp, cdiv2(a_rows, 256) * cdiv2(N, 128), MOE_K_DOWN, st);

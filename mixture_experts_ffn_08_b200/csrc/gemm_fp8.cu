@@ -53,29 +53,40 @@ cudaError_t launch8(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorM
 // UE8M0 byte of a power-of-two fp32 scale: its biased exponent field.
 __device__ __forceinline__ uint32_t ue8m0_of(float s) { return (__float_as_uint(s) >> 23) & 0xFFu; }
 
-// Per-row scales [rows, nk] (one per 128 columns) -> atoms [rows/128][nk][512], for the
-// rows of the buckets (offsets[G] of them).
+// Per-row scales [rows, nk] (one per 128 columns) -> atoms [rows/128][ceil(nk/4)][512]:
+// scale kb of row r is byte kb % 4 of the row's word in atom kb / 4.  For the rows of the
+// buckets (offsets[G] of them).
 __global__ void sf_rows_to_atoms_kernel(const float* __restrict__ scales, int nk,
                                         const int32_t* __restrict__ offsets, int G,
                                         uint8_t* __restrict__ atoms) {
   const long long n = static_cast<long long>(__ldg(offsets + G)) * nk;
+  const int nk4 = (nk + 3) / 4;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
        i += (long long)gridDim.x * blockDim.x) {
     const long long r = i / nk;
     const int kb = static_cast<int>(i % nk);
-    const uint32_t word = ue8m0_of(__ldg(scales + i)) * 0x01010101u;
-    uint8_t* atom = atoms + ((r >> 7) * nk + kb) * 512;
-    *reinterpret_cast<uint32_t*>(atom + sf_atom_offset(static_cast<int>(r & 127))) = word;
+    uint8_t* atom = atoms + ((r >> 7) * nk4 + (kb >> 2)) * 512;
+    atom[sf_atom_offset(static_cast<int>(r & 127)) + (kb & 3)] = static_cast<uint8_t>(ue8m0_of(__ldg(scales + i)));
   }
 }
 
-// One scale per 128x128 weight block -> one atom (512 equal bytes) per block.
-__global__ void sf_blocks_to_atoms_kernel(const float* __restrict__ scales, long long nblocks,
+// One scale per 128x128 weight block, blocks [nblk][nk] -> atoms [nblk][ceil(nk/4)][512]
+// whose 128 words all hold the scales of four consecutive K blocks.
+__global__ void sf_blocks_to_atoms_kernel(const float* __restrict__ scales, long long nblk, int nk,
                                           uint8_t* __restrict__ atoms) {
-  const long long n = nblocks * 32;  // 32 x 16 bytes per atom
+  const int nk4 = (nk + 3) / 4;
+  const long long n = nblk * nk4 * 32;  // 32 x 16 bytes per atom
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
        i += (long long)gridDim.x * blockDim.x) {
-    const uint32_t w = ue8m0_of(__ldg(scales + (i >> 5))) * 0x01010101u;
+    const long long a = i >> 5;
+    const long long blk = a / nk4;
+    const int kb0 = static_cast<int>(a % nk4) * 4;
+    uint32_t w = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t b = kb0 + j < nk ? ue8m0_of(__ldg(scales + blk * nk + kb0 + j)) : 127u;
+      w |= b << (8 * j);
+    }
     reinterpret_cast<uint4*>(atoms)[i] = make_uint4(w, w, w, w);
   }
 }
@@ -94,12 +105,12 @@ cudaError_t launch_sf_rows_to_atoms(const float* scales, int nk, const int32_t* 
   return cudaGetLastError();
 }
 
-cudaError_t launch_sf_blocks_to_atoms(const float* scales, long long nblocks, uint8_t* atoms,
+cudaError_t launch_sf_blocks_to_atoms(const float* scales, long long nblk, int nk, uint8_t* atoms,
                                       cudaStream_t st) {
-  const long long n = nblocks * 32;
+  const long long n = nblk * ((nk + 3) / 4) * 32;
   const int grid = static_cast<int>(cdiv(n, 256) < num_sms() * 8LL ? cdiv(n, 256) : num_sms() * 8LL);
   trace_before(MOE_K_SCALE_ATOMS, st);
-  sf_blocks_to_atoms_kernel<<<grid > 0 ? grid : 1, 256, 0, st>>>(scales, nblocks, atoms);
+  sf_blocks_to_atoms_kernel<<<grid > 0 ? grid : 1, 256, 0, st>>>(scales, nblk, nk, atoms);
   trace_after(MOE_K_SCALE_ATOMS, st);
   return cudaGetLastError();
 }

@@ -69,7 +69,7 @@ cudaError_t launch_f32_to_bf16(const float* acc, long long n, void* out, cudaStr
 // fp32 power-of-two scales -> 512-byte UE8M0 scale atoms (see tc_gemm_fp8.cuh).
 cudaError_t launch_sf_rows_to_atoms(const float* scales, int nk, const int32_t* offsets, int G,
                                     long long max_rows, uint8_t* atoms, cudaStream_t st);
-cudaError_t launch_sf_blocks_to_atoms(const float* scales, long long nblocks, uint8_t* atoms,
+cudaError_t launch_sf_blocks_to_atoms(const float* scales, long long nblk, int nk, uint8_t* atoms,
                                       cudaStream_t st);
 // h (e4m3 [rows, N] + scale atoms) = quant(SiLU(A Wg^T) * (A Wu^T)), block-scaled e4m3 GEMM.
 cudaError_t gemm_gateup_swiglu_fp8(const void* A, const uint8_t* a_atoms, int64_t a_rows,

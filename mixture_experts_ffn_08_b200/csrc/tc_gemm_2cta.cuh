@@ -217,6 +217,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   const int NT = (p.N + Cfg::OUT_COLS - 1) / Cfg::OUT_COLS;
   const int total = num_pairs * NT;
   const int KB = p.K / BK;
+  const int KB4 = (KB + 3) / 4;  // FP8 scale atoms along K (four K steps each)
   const int cluster_id = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
   if (cluster_id >= total) return;  // same decision in both CTAs of the cluster
 
@@ -269,18 +270,22 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           uint8_t* sb = sa + Cfg::A_BYTES;
           uint8_t* ssf = sb + Cfg::B_BYTES;
           const uint32_t bar = mapa_shared(smem_u32(&full_bar[s]), 0);
-          if (leader) mbar_arrive_expect_tx(&full_bar[s], 2 * Cfg::CTA_TX);
+          const bool new_sf = Cfg::FP8 && (kb & 3) == 0;
+          if (leader) mbar_arrive_expect_tx(&full_bar[s], 2 * (Cfg::CTA_TX - (new_sf ? 0 : Cfg::SF_BYTES)));
           tma_load_2d_pair(sa, &tmA, kb * BK, a_row, bar);
           tma_load_2d_pair(sb, (Cfg::SWIGLU && rank == 1) ? &tmB1 : &tmB0, kb * BK, b_row, bar);
           if constexpr (Cfg::FP8) {
-            tma_load_2d_pair(ssf, &tmSfa, 0, t.m_tile * KB + kb, bar);
-            if constexpr (Cfg::SWIGLU) {
-              tma_load_2d_pair(ssf + 512, &tmSfb0, 0, wblk * KB + kb, bar);
-              tma_load_2d_pair(ssf + 1024, &tmSfb1, 0, wblk * KB + kb, bar);
-            } else {
+            if (new_sf) {
+              const int kb4 = kb >> 2;
+              tma_load_2d_pair(ssf, &tmSfa, 0, t.m_tile * KB4 + kb4, bar);
+              if constexpr (Cfg::SWIGLU) {
+                tma_load_2d_pair(ssf + 512, &tmSfb0, 0, wblk * KB4 + kb4, bar);
+                tma_load_2d_pair(ssf + 1024, &tmSfb1, 0, wblk * KB4 + kb4, bar);
+              } else {
 #pragma unroll
-              for (int a = 0; a < Cfg::SFB_ATOMS; ++a)
-                tma_load_2d_pair(ssf + 512 * (1 + a), &tmSfb0, 0, (wblk + a) * KB + kb, bar);
+                for (int a = 0; a < Cfg::SFB_ATOMS; ++a)
+                  tma_load_2d_pair(ssf + 512 * (1 + a), &tmSfb0, 0, (wblk + a) * KB4 + kb4, bar);
+              }
             }
           }
           ++issued;
@@ -319,14 +324,17 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           const uint32_t b0 = a0 + Cfg::A_BYTES;
           if constexpr (Cfg::FP8) {
             const uint32_t sf0 = b0 + Cfg::B_BYTES;
-            tmem_cp_pair_32x128b_warpx4(sfa_t, smem_desc_rows16(sf0));
+            if ((kb & 3) == 0) {
+              tmem_cp_pair_32x128b_warpx4(sfa_t, smem_desc_rows16(sf0));
 #pragma unroll
-            for (int a = 0; a < Cfg::SFB_ATOMS; ++a)
-              tmem_cp_pair_32x128b_warpx4(sfb_t + 4 * a, smem_desc_rows16(sf0 + 512 * (1 + a)));
+              for (int a = 0; a < Cfg::SFB_ATOMS; ++a)
+                tmem_cp_pair_32x128b_warpx4(sfb_t + 4 * a, smem_desc_rows16(sf0 + 512 * (1 + a)));
+            }
+            const uint32_t idesc = idesc_mxf8_e4m3(256, BN, kb & 3, kb & 3);
 #pragma unroll
             for (int kk = 0; kk < BK / 32; ++kk)
-              umma_mxf8_pair(d_tmem, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32),
-                             idesc_mxf8_e4m3(256, BN, kk, kk), sfa_t, sfb_t, (kb | kk) != 0);
+              umma_mxf8_pair(d_tmem, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32), idesc, sfa_t,
+                             sfb_t, (kb | kk) != 0);
           } else {
 #pragma unroll
             for (int k = 0; k < BK / 16; ++k)
@@ -419,8 +427,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                 e4m3x4(hv[12] * inv, hv[13] * inv, hv[14] * inv, hv[15] * inv));
           }
         }
-        uint8_t* sf = p.out_sf + (static_cast<size_t>(t.m_tile) * (p.N / 128) + t.n_tile) * 512;
-        *reinterpret_cast<uint32_t*>(sf + sf_atom_offset(row_in_tile)) = static_cast<uint32_t>(e + 127) * 0x01010101u;
+        const int kb4n = (p.N / 128 + 3) / 4;
+        uint8_t* sf = p.out_sf + (static_cast<size_t>(t.m_tile) * kb4n + (t.n_tile >> 2)) * 512;
+        sf[sf_atom_offset(row_in_tile) + (t.n_tile & 3)] = static_cast<uint8_t>(e + 127);
       } else if constexpr (Cfg::EPI == EPI2_F32) {
         float* out = static_cast<float*>(p.out) + row * p.ldo + col0;
 #pragma unroll 1

@@ -9,13 +9,15 @@
 // the four 32-element sub-blocks it covers and the products come out exactly as
 //   sum_k (s_x[r,k/128] q_x[r,k]) (s_w[n/128,k/128] q_w[n,k]).
 //
-// Scales travel as 512-byte "atoms" (128 rows x 4 sub-blocks of one 128-wide K step):
-// row m0 + 32*m1 (m0 < 32, m1 < 4) keeps its four scale bytes in the 32-bit word at byte
-// 16*m0 + 4*m1.  Per pipeline stage the producer brings the A atom and one B atom per
+// Scales travel as 512-byte "atoms" (128 rows x one 32-bit word): row m0 + 32*m1
+// (m0 < 32, m1 < 4) keeps its word at byte 16*m0 + 4*m1, and the MMA reads one byte of
+// each word, chosen by the sf-id fields of the instruction descriptor.  Because the
+// layer's scales cover 128 K-elements (four MX sub-blocks of 32), byte b of a word holds
+// the scale of the b-th of four consecutive 128-wide K steps: one atom serves four
+// pipeline stages.  Every fourth stage the producer brings the A atom and one B atom per
 // 128 rows of B next to the A/B tiles (1D bulk copies on the same mbarrier); the MMA
 // thread copies them to TMEM with tcgen05.cp.32x128b.warpx4 (32 lanes x 4 columns,
-// replicated into the four lane quadrants) and issues four K=32 MMAs that select scale
-// byte kk of each word through the instruction descriptor.
+// replicated into the four lane quadrants) and all MMAs of K step kb select byte kb % 4.
 //
 // Epilogues:
 //   EPI8_SWIGLU_Q  B = [128 gate rows; 128 up rows]; h = SiLU(gate) * up in fp32, then
@@ -99,12 +101,12 @@ struct Fp8Params {
   int G;
   int K;                   // reduction length, multiple of 128
   int N;                   // output columns of one group
-  const uint8_t* sfa;      // A scale atoms [m_tiles][K/128][512]
-  const uint8_t* sfb0;     // B scale atoms [G][N/128][K/128][512] (gate, or the down weight)
+  const uint8_t* sfa;      // A scale atoms [m_tiles][ceil(K/512)][512]
+  const uint8_t* sfb0;     // B scale atoms [G][N/128][ceil(K/512)][512] (gate, or down weight)
   const uint8_t* sfb1;     // up-projection scale atoms (SwiGLU only)
   void* out;               // SwiGLU: e4m3 codes [rows, ldo]; BF16: bf16 [rows, ldo]
   int64_t ldo;             // elements
-  uint8_t* out_sf;         // SwiGLU: h scale atoms [m_tiles][N/128][512]
+  uint8_t* out_sf;         // SwiGLU: h scale atoms [m_tiles][ceil(N/512)][512]
   int32_t* status;
 };
 
@@ -170,6 +172,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   const int NT = (p.N + Cfg::OUT_COLS - 1) / Cfg::OUT_COLS;
   const int total = num_m_tiles * NT;
   const int KB = p.K / BK;
+  const int KB4 = (KB + 3) / 4;  // scale atoms along K (four K steps each)
   if ((int)blockIdx.x >= total) return;
 
   // the item decoder of the bf16 kernel works on these fields only
@@ -223,21 +226,28 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           uint8_t* sa = smem + s * Cfg::STAGE_BYTES;
           uint8_t* sb = sa + Cfg::A_BYTES;
           uint8_t* ssf = sb + Cfg::B_BYTES;
-          mbar_arrive_expect_tx(&full_bar[s], Cfg::A_BYTES + Cfg::B_BYTES + Cfg::SF_BYTES);
+          const bool new_sf = (kb & 3) == 0;
+          mbar_arrive_expect_tx(&full_bar[s], Cfg::A_BYTES + Cfg::B_BYTES + (new_sf ? Cfg::SF_BYTES : 0));
           tma_load_2d(sa, &tmA, kb * BK, a_row, &full_bar[s]);
-          bulk_load(ssf, p.sfa + (static_cast<size_t>(t.m_tile) * KB + kb) * 512, 512, &full_bar[s]);
-          const size_t wsf = (static_cast<size_t>(wblk) * KB + kb) * 512;
           if (Cfg::EPI == EPI8_SWIGLU_Q) {
             tma_load_2d(sb, &tmB0, kb * BK, b_row, &full_bar[s]);
             tma_load_2d(sb + 128 * BK, &tmB1, kb * BK, b_row, &full_bar[s]);
-            bulk_load(ssf + 512, p.sfb0 + wsf, 512, &full_bar[s]);
-            bulk_load(ssf + 1024, p.sfb1 + wsf, 512, &full_bar[s]);
           } else {
             tma_load_2d(sb, &tmB0, kb * BK, b_row, &full_bar[s]);
+          }
+          if (new_sf) {
+            const int kb4 = kb >> 2;
+            bulk_load(ssf, p.sfa + (static_cast<size_t>(t.m_tile) * KB4 + kb4) * 512, 512, &full_bar[s]);
+            const size_t wsf = (static_cast<size_t>(wblk) * KB4 + kb4) * 512;
+            if (Cfg::EPI == EPI8_SWIGLU_Q) {
+              bulk_load(ssf + 512, p.sfb0 + wsf, 512, &full_bar[s]);
+              bulk_load(ssf + 1024, p.sfb1 + wsf, 512, &full_bar[s]);
+            } else {
 #pragma unroll
-            for (int a = 0; a < Cfg::SFB_ATOMS; ++a)
-              bulk_load(ssf + 512 * (1 + a), p.sfb0 + wsf + static_cast<size_t>(a) * KB * 512, 512,
-                        &full_bar[s]);
+              for (int a = 0; a < Cfg::SFB_ATOMS; ++a)
+                bulk_load(ssf + 512 * (1 + a), p.sfb0 + wsf + static_cast<size_t>(a) * KB4 * 512, 512,
+                          &full_bar[s]);
+            }
           }
           ++issued;
           if (++s == STAGES) { s = 0; ph ^= 1u; }
@@ -269,14 +279,17 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           const uint32_t a0 = smem_u32(smem + s * Cfg::STAGE_BYTES);
           const uint32_t b0 = a0 + Cfg::A_BYTES;
           const uint32_t sf0 = b0 + Cfg::B_BYTES;
-          tmem_cp_32x128b_warpx4(sfa_t, smem_desc_rows16(sf0));
+          if ((kb & 3) == 0) {  // new scale atoms (four K steps each) into TMEM
+            tmem_cp_32x128b_warpx4(sfa_t, smem_desc_rows16(sf0));
 #pragma unroll
-          for (int a = 0; a < Cfg::SFB_ATOMS; ++a)
-            tmem_cp_32x128b_warpx4(sfb_t + 4 * a, smem_desc_rows16(sf0 + 512 * (1 + a)));
+            for (int a = 0; a < Cfg::SFB_ATOMS; ++a)
+              tmem_cp_32x128b_warpx4(sfb_t + 4 * a, smem_desc_rows16(sf0 + 512 * (1 + a)));
+          }
+          const uint32_t idesc = idesc_mxf8_e4m3(BM, BN, kb & 3, kb & 3);
 #pragma unroll
           for (int kk = 0; kk < BK / 32; ++kk) {
-            umma_mxf8(d_tmem, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32),
-                      idesc_mxf8_e4m3(BM, BN, kk, kk), sfa_t, sfb_t, (kb | kk) != 0);
+            umma_mxf8(d_tmem, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32), idesc, sfa_t, sfb_t,
+                      (kb | kk) != 0);
           }
           umma_commit(&empty_bar[s]);
           if (++s == STAGES) { s = 0; ph ^= 1u; }
@@ -338,9 +351,10 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                 e4m3x4(hv[12] * inv, hv[13] * inv, hv[14] * inv, hv[15] * inv));
           }
         }
-        const uint32_t byte = static_cast<uint32_t>(e + 127);
-        uint8_t* sf = p.out_sf + (static_cast<size_t>(t.m_tile) * (p.N / 128) + t.n_tile) * 512;
-        *reinterpret_cast<uint32_t*>(sf + sf_atom_offset(row_in_tile)) = byte * 0x01010101u;
+        // byte (n_tile % 4) of this row's word in atom (m_tile, n_tile / 4) of the down GEMM
+        const int kb4n = (p.N / 128 + 3) / 4;
+        uint8_t* sf = p.out_sf + (static_cast<size_t>(t.m_tile) * kb4n + (t.n_tile >> 2)) * 512;
+        sf[sf_atom_offset(row_in_tile) + (t.n_tile & 3)] = static_cast<uint8_t>(e + 127);
       } else {
         __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + row * p.ldo + col0;
 #pragma unroll 1
