@@ -31,6 +31,8 @@ Readings where the pages are silent (each also listed in the design notes):
     goes to the lower index.
   - Pairs p = t*K + k are bucketed stably: inside an expert, rows follow p.
   - Each expert's rows start at a multiple of `block_m`; pad rows carry no pair.
+  - Masked layout: expert e owns rows [e*cap, (e+1)*cap); a pair ranked cap or later
+    inside its expert gets no row and contributes nothing.
   - Renormalise first, then multiply by routed_scale; the shared expert is added with
     weight 1.
   - The SwiGLU output h is an activation and is stored in the workload's activation
@@ -242,6 +244,39 @@ def permute(ids, E: int, block_m: int):
             row_of_pair.astype(np.int32), pair_of_row.astype(np.int32))
 
 
+def permute_masked(ids, E: int, cap: int):
+    """The masked grouped layout ("MoE" chapter index §1, the grouped-GEMM entry: the
+    second of its two layouts): expert e owns the fixed row range [e*cap, (e+1)*cap)
+    and its pairs fill the first rows of that range, stably in p.
+
+    The page names the layout only.  Reading used here: a pair whose rank inside its
+    expert is cap or more has no row (row_of_pair = -1) and is left out of the layer
+    output; counts [E] is the number of rows in use, min(n_e, cap).  With cap >= T no
+    pair is ever left out, since a token chooses K distinct experts.
+
+    Returns counts [E], offsets [E+1] = e*cap, row_of_pair [P], pair_of_row [E*cap]
+    (-1 on unused rows) and the number of pairs left out."""
+    flat = np.asarray(ids, np.int64).reshape(-1)
+    P = flat.shape[0]
+    rank = np.zeros(E, dtype=np.int64)
+    row_of_pair = np.full(P, -1, dtype=np.int64)
+    pair_of_row = np.full(E * cap, -1, dtype=np.int64)
+    dropped = 0
+    for p in range(P):
+        e = flat[p]
+        if rank[e] < cap:
+            row = e * cap + rank[e]
+            row_of_pair[p] = row
+            pair_of_row[row] = p
+        else:
+            dropped += 1
+        rank[e] += 1
+    counts = np.minimum(rank, cap)
+    offsets = np.arange(E + 1, dtype=np.int64) * cap
+    return (counts.astype(np.int32), offsets.astype(np.int32), row_of_pair.astype(np.int32),
+            pair_of_row.astype(np.int32), dropped)
+
+
 # ----------------------------------------------------------------------------------
 # Expert FFN and combine
 # ----------------------------------------------------------------------------------
@@ -279,14 +314,17 @@ def expert_outputs(x, ids, expert_weights, E: int, block_m: int, h_format=None):
 
 
 def combine(y_perm, row_of_pair, w, y_shared=None) -> np.ndarray:
-    """out[t] = sum_k w[t, k] * y_perm[row_of_pair[t*K + k]]  (+ y_shared[t])."""
+    """out[t] = sum_k w[t, k] * y_perm[row_of_pair[t*K + k]]  (+ y_shared[t]).
+    A pair without a row (row_of_pair = -1, left out by the masked layout) adds 0."""
     w = np.asarray(w, np.float64)
     T, K = w.shape
     y_perm = np.asarray(y_perm, np.float64)
     out = np.zeros((T, y_perm.shape[1]), dtype=np.float64)
     for t in range(T):
         for k in range(K):
-            out[t] += w[t, k] * y_perm[row_of_pair[t * K + k]]
+            r = row_of_pair[t * K + k]
+            if r >= 0:
+                out[t] += w[t, k] * y_perm[r]
     if y_shared is not None:
         out += np.asarray(y_shared, np.float64)
     return out

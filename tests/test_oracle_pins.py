@@ -55,6 +55,53 @@ def test_bucket_example():
         assert [int(pair_of_row[r]) // g["K"] for r in rows] == g["buckets"][e]
 
 
+@pytest.mark.parametrize("cap", [3, 4, 8])
+def test_bucket_example_masked_layout(cap):
+    """The page's dispatch example in the masked layout: expert e's tokens fill rows
+    e*cap onwards in the printed order."""
+    g = load_golden("bucket_example.txt")
+    ids = np.array([[e for (t, e) in g["pairs"][i * g["K"]:(i + 1) * g["K"]]] for i in range(g["T"])])
+    counts, offs, rop, por, dropped = o.permute_masked(ids, g["E"], cap)
+    assert counts.tolist() == g["counts"] and dropped == 0
+    assert offs.tolist() == [e * cap for e in range(g["E"] + 1)]
+    for e in range(g["E"]):
+        rows = range(e * cap, e * cap + counts[e])
+        assert [int(por[r]) // g["K"] for r in rows] == g["buckets"][e]
+        assert (por[e * cap + counts[e]:(e + 1) * cap] == -1).all()
+    for p in range(ids.size):
+        assert por[rop[p]] == p
+
+
+def test_masked_layout_overflow_keeps_the_first_pairs():
+    """Expert 2 of the page's dispatch example has 3 tokens; with cap 2 the third
+    (token 2, the last pair of expert 2 in pair order) has no row."""
+    g = load_golden("bucket_example.txt")
+    ids = np.array([[e for (t, e) in g["pairs"][i * g["K"]:(i + 1) * g["K"]]] for i in range(g["T"])])
+    counts, offs, rop, por, dropped = o.permute_masked(ids, g["E"], 2)
+    assert counts.tolist() == [1, 1, 2, 1] and dropped == 1
+    assert rop.tolist() == [2, 4, 0, 5, 6, -1]
+    # the dropped pair adds nothing to its token: out[2] = w * y of expert 3 alone
+    y = np.arange(8, dtype=np.float64)[:, None] * np.ones((1, 2))
+    w = np.ones((3, 2))
+    out = o.combine(y, rop, w)
+    assert out[2].tolist() == [6.0, 6.0] and out[0].tolist() == [6.0, 6.0]
+
+
+@pytest.mark.parametrize("cap", [37, 64])
+def test_masked_ranks_match_contiguous_ranks(cap):
+    """With room for every pair, the masked row of a pair is e*cap plus its rank, the
+    same rank the contiguous layout gives (brute-force count of earlier pairs)."""
+    rng = np.random.default_rng(cap)
+    T, K, E = 37, 3, 9
+    ids = np.stack([rng.choice(E, size=K, replace=False) for _ in range(T)])
+    counts, offs, rop, por, dropped = o.permute_masked(ids, E, cap)
+    assert dropped == 0 and counts.sum() == T * K
+    flat = ids.ravel()
+    for p in range(T * K):
+        e = flat[p]
+        assert rop[p] == e * cap + sum(1 for q in range(p) if flat[q] == e)
+
+
 @pytest.mark.parametrize("group_topn", [1, 2])
 def test_grouped_topk_example(group_topn):
     g = load_golden("grouped_topk_example.txt")
