@@ -89,6 +89,8 @@ def _describe(wl):
         s += " fused-combine"
     if wl.block_m:
         s += f" block_m={wl.block_m}"
+    if wl.masked_cap:
+        s += f" masked-layout cap={wl.masked_cap}"
     return s + (" fp8" if wl.dtype else " bf16")
 
 
@@ -213,6 +215,8 @@ def run_ours(args):
         wl = wl.with_(fused_combine=True)
     if args.block_m:
         wl = wl.with_(block_m=args.block_m)
+    if args.masked_cap:
+        wl = wl.with_(masked_cap=args.masked_cap)
     p = B.params(wl)
     d = inputs.make_inputs(wl, seed=rank, device="cuda")
     fp8 = wl.dtype == W.DTYPE_FP8
@@ -483,6 +487,8 @@ def main():
                     help="down projection adds into the output with fp32 atomics (non-deterministic)")
     ap.add_argument("--block-m", type=int, default=0, choices=[0, 128, 256],
                     help="bucket alignment: 256 selects the two-SM (cta_group::2) GEMM tiles")
+    ap.add_argument("--masked-cap", type=int, default=0,
+                    help="masked bucket layout: expert e owns rows [e*cap, (e+1)*cap) (multiple of 128)")
     ap.add_argument("--micro", choices=["grouped_topk"], default=None,
                     help="time one stage alone instead of the layer")
     args = ap.parse_args()

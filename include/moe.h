@@ -45,7 +45,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 2
+#define MOE_ABI_VERSION 3
 
 typedef enum moe_status {
   MOE_OK = 0,
@@ -59,6 +59,8 @@ typedef enum moe_status {
 /* Bits of the device status word (moe_get_device_status). */
 #define MOE_DEV_BAD_EXPERT_ID 0x1   /* a topk id outside [0,E): the pair was skipped      */
 #define MOE_DEV_TIMEOUT 0x2         /* a GEMM pipeline wait exceeded its limit and exited */
+#define MOE_DEV_CAPACITY 0x4        /* masked layout: an expert had more than masked_cap    */
+                                    /* pairs; the pairs past it got no row (left out)       */
 
 enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 };
 enum { MOE_DTYPE_BF16 = 0, MOE_DTYPE_FP8_E4M3 = 1 };
@@ -84,6 +86,14 @@ typedef struct moe_params {
                         /* deterministic combine (default); 1 = the down projection adds */
                         /* w * y straight into an fp32 token accumulator with atomic     */
                         /* vector reductions (no y_perm round trip; run-to-run bits vary)*/
+  int32_t masked_cap;   /* bucket layout ("MoE" chapter index §1, grouped-GEMM entry):   */
+                        /* 0 = contiguous (expert e's bucket starts at offsets_padded[e],*/
+                        /* a multiple of block_m, and holds exactly its pairs); > 0 =    */
+                        /* masked: expert e owns the fixed rows [e*cap, (e+1)*cap), its  */
+                        /* counts[e] pairs fill the first of them, the rest are unused.  */
+                        /* cap is a multiple of 128, block_m must be 128.  An expert     */
+                        /* with more than cap pairs keeps the first cap (in pair order)  */
+                        /* and sets MOE_DEV_CAPACITY; cap >= T never drops a pair.       */
 } moe_params_t;
 
 /* ---------------------------------------------------------------------------------- */
@@ -101,8 +111,9 @@ size_t moe_workspace_size_host(const moe_params_t* p);
 /* Bucket alignment the calls use for these parameters (128 or 256); -1 if invalid. */
 int32_t moe_effective_block_m(const moe_params_t* p);
 
-/* Upper bound on the padded row count P + E*(block_m-1): the row capacity that
- * pair_of_row, x_perm and y_perm must have.  -1 if the parameters are invalid. */
+/* Row capacity that pair_of_row, x_perm and y_perm must have: the bound P + E*(block_m-1)
+ * on the padded row count (contiguous layout), or E*masked_cap (masked layout).  -1 if
+ * the parameters are invalid. */
 int64_t moe_max_padded_rows(const moe_params_t* p);
 
 /* ---------------------------------------------------------------------------------- */
@@ -142,6 +153,9 @@ moe_status_t moe_aux_free_bias_update(const int32_t* counts, int32_t E, float ga
 /*   x_perm         [moe_max_padded_rows, H] out: x[t] copied to each pair's row, pad   */
 /*                  rows zero (bf16, or e4m3 codes + x_perm_scale [rows, H/128] fp32)   */
 /* An id outside [0,E) sets MOE_DEV_BAD_EXPERT_ID and that pair is left out.            */
+/* Masked layout (masked_cap > 0): offsets_padded[e] = e*cap; counts[e] = rows in use,  */
+/* min(pairs of e, cap); a pair past cap gets row_of_pair = -1 (MOE_DEV_CAPACITY); the  */
+/* unused rows get pair_of_row = -1 but their x_perm rows are not written.              */
 /* ---------------------------------------------------------------------------------- */
 moe_status_t moe_permute(const moe_params_t* p, const int32_t* topk_ids, const void* x,
                          const float* x_scale, int32_t* counts, int32_t* offsets_padded,
@@ -175,6 +189,9 @@ moe_status_t moe_permute_noalloc(const moe_params_t* p, const int32_t* topk_ids,
 /* for every row r of expert e's bucket (pad rows included; their result is unused).    */
 /*   offsets_padded [E+1], counts [E] as written by moe_permute (read on the device     */
 /*                  only); counts may be NULL, then pad rows are computed and stored too */
+/*                  Masked layout: counts (the rows in use of each expert) is required   */
+/*                  and offsets_padded may be NULL (then e*cap); 128-row tiles wholly    */
+/*                  past counts[e] are skipped by every kernel                           */
 /*   y_perm [moe_max_padded_rows, H] out, fp32 for MOE_DTYPE_BF16 and bf16 for FP8; rows */
 /*                  past counts[e] in a bucket are not written when counts is given     */
 /* The SwiGLU intermediate h (bf16, or e4m3 + scales) lives in ws.  For bf16 workloads  */

@@ -22,6 +22,7 @@ _lib = None
 MOE_OK = 0
 MOE_DEV_BAD_EXPERT_ID = 0x1
 MOE_DEV_TIMEOUT = 0x2
+MOE_DEV_CAPACITY = 0x4
 BLOCK_M = 128
 
 # Kernel ids for tracing (include/moe.h).
@@ -44,13 +45,13 @@ class MoeParams(ctypes.Structure):
                 ("score_fn", ctypes.c_int32), ("renormalize", ctypes.c_int32),
                 ("routed_scale", ctypes.c_float), ("I_shared", ctypes.c_int32),
                 ("dtype", ctypes.c_int32), ("block_m", ctypes.c_int32),
-                ("fused_combine", ctypes.c_int32)]
+                ("fused_combine", ctypes.c_int32), ("masked_cap", ctypes.c_int32)]
 
 
 def params(wl: W.Workload) -> MoeParams:
     return MoeParams(wl.T, wl.H, wl.I, wl.E, wl.K, wl.n_group, wl.topk_group, wl.group_topn,
                      wl.score_fn, int(wl.renormalize), float(wl.routed_scale), wl.I_shared,
-                     wl.dtype, wl.block_m, int(wl.fused_combine))
+                     wl.dtype, wl.block_m, int(wl.fused_combine), wl.masked_cap)
 
 
 _P = ctypes.c_void_p

@@ -62,7 +62,7 @@ constexpr size_t kAlign = 256;
 size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 struct Layout {
-  size_t status, logits, xb, ids, w, counts, offsets, row_of_pair, pair_of_row, chunk_counts;
+  size_t status, logits, xb, ids, w, counts, offsets, sched, row_of_pair, pair_of_row, chunk_counts;
   size_t x_perm, x_perm_scale, h, y_perm, h_sh, y_sh, total;
   size_t x_atoms, h_atoms, wg_atoms, wu_atoms, wd_atoms;
   size_t x_stage, x_scale_stage, out_stage, total_host;
@@ -82,7 +82,7 @@ Layout layout(const moe_params_t* p) {
   const long long T = p->T, H = p->H, I = p->I, E = p->E, K = p->K;
   const long long P = T * K;
   const long long bm = block_m_of(p);
-  const long long rows = P + E * (bm - 1);
+  const long long rows = p->masked_cap > 0 ? E * p->masked_cap : P + E * (bm - 1);
   const long long rows_t = (rows + kBlockM2 - 1) / kBlockM2 * kBlockM2;  // whole M-tile pairs
   const long long nchunks = (P + kPermChunk - 1) / kPermChunk;
   const size_t xelem = is_fp8(p) ? 1 : 2;
@@ -96,6 +96,7 @@ Layout layout(const moe_params_t* p) {
   L.w = take(P * 4);
   L.counts = take(E * 4);
   L.offsets = take((E + 1) * 4);
+  L.sched = take(p->masked_cap > 0 ? (E + 1) * 4 : 0);
   L.row_of_pair = take(P * 4);
   L.pair_of_row = take(rows * 4);
   L.chunk_counts = take((nchunks > 0 ? nchunks : 1) * E * 4);
@@ -147,6 +148,11 @@ moe_status_t validate(const moe_params_t* p) {
   if (p->fused_combine && (p->dtype != MOE_DTYPE_BF16 || p->block_m == kBlockM2)) return MOE_ERR_UNSUPPORTED;
   const long long rows = static_cast<long long>(p->T) * p->K + static_cast<long long>(p->E) * (kBlockM2 - 1);
   if (rows >= (1LL << 31) / 2) return MOE_ERR_INVALID_ARG;
+  if (p->masked_cap < 0) return MOE_ERR_INVALID_ARG;
+  if (p->masked_cap > 0) {
+    if (p->masked_cap % kBlockM != 0 || p->block_m == kBlockM2) return MOE_ERR_UNSUPPORTED;
+    if (static_cast<long long>(p->E) * p->masked_cap >= (1LL << 31) / 2) return MOE_ERR_INVALID_ARG;
+  }
   return MOE_OK;
 }
 
@@ -200,6 +206,13 @@ moe_status_t do_expert_ffn_fp8(const moe_params_t* p, const void* x_perm, const 
                                cudaStream_t st) {
   const Layout L = layout(p);
   int32_t* status = at<int32_t>(ws, L.status);
+  // masked layout: the GEMMs walk a compact schedule and address expert e's rows at e*cap
+  const int cap = p->masked_cap;
+  const int32_t* sched = offsets;
+  if (cap > 0) {
+    MOE_CUDA(launch_masked_schedule(counts, p->E, at<int32_t>(ws, L.sched), st));
+    sched = at<int32_t>(ws, L.sched);
+  }
   const long long rows_gu = static_cast<long long>(p->E) * (p->I / 128);   // 128-row weight blocks
   const long long rows_d = static_cast<long long>(p->E) * (p->H / 128);
   MOE_CUDA(launch_sf_blocks_to_atoms(wgs, rows_gu, p->H / 128, at<uint8_t>(ws, L.wg_atoms), st));
@@ -216,11 +229,11 @@ moe_status_t do_expert_ffn_fp8(const moe_params_t* p, const void* x_perm, const 
                                 at<uint8_t>(ws, L.wd_atoms), p->H, p->I, y_perm, status, st));
     return MOE_OK;
   }
-  MOE_CUDA(gemm_gateup_swiglu_fp8(x_perm, at<uint8_t>(ws, L.x_atoms), L.max_rows, offsets, counts, p->E,
+  MOE_CUDA(gemm_gateup_swiglu_fp8(x_perm, at<uint8_t>(ws, L.x_atoms), L.max_rows, sched, counts, p->E,
                                   w_gate, w_up, at<uint8_t>(ws, L.wg_atoms), at<uint8_t>(ws, L.wu_atoms),
-                                  p->I, p->H, h, at<uint8_t>(ws, L.h_atoms), status, st));
-  MOE_CUDA(gemm_down_fp8(h, at<uint8_t>(ws, L.h_atoms), L.max_rows, offsets, counts, p->E, w_down,
-                         at<uint8_t>(ws, L.wd_atoms), p->H, p->I, y_perm, status, st));
+                                  p->I, p->H, h, at<uint8_t>(ws, L.h_atoms), status, st, cap));
+  MOE_CUDA(gemm_down_fp8(h, at<uint8_t>(ws, L.h_atoms), L.max_rows, sched, counts, p->E, w_down,
+                         at<uint8_t>(ws, L.wd_atoms), p->H, p->I, y_perm, status, st, cap));
   return MOE_OK;
 }
 
@@ -236,10 +249,16 @@ moe_status_t do_expert_ffn(const moe_params_t* p, const void* x_perm, const int3
     MOE_CUDA(gemm_pair_down(h, L.max_rows, offsets, counts, p->E, w_down, p->H, p->I, y_perm, status, st));
     return MOE_OK;
   }
-  MOE_CUDA(gemm_gateup_swiglu(x_perm, L.max_rows, offsets, counts, p->E, 0, w_gate, w_up, p->I, p->H,
-                              h, status, MOE_K_GATEUP, st));
-  MOE_CUDA(gemm_down(h, L.max_rows, offsets, counts, p->E, 0, w_down, p->H, p->I, y_perm, status,
-                     MOE_K_DOWN, st));
+  const int cap = p->masked_cap;
+  const int32_t* sched = offsets;
+  if (cap > 0) {  // masked layout: compact schedule, expert e's rows at e*cap
+    MOE_CUDA(launch_masked_schedule(counts, p->E, at<int32_t>(ws, L.sched), st));
+    sched = at<int32_t>(ws, L.sched);
+  }
+  MOE_CUDA(gemm_gateup_swiglu(x_perm, L.max_rows, sched, counts, p->E, 0, w_gate, w_up, p->I, p->H,
+                              h, status, MOE_K_GATEUP, st, cap));
+  MOE_CUDA(gemm_down(h, L.max_rows, sched, counts, p->E, 0, w_down, p->H, p->I, y_perm, status,
+                     MOE_K_DOWN, st, cap));
   return MOE_OK;
 }
 
@@ -279,10 +298,16 @@ moe_status_t do_layer(const moe_params_t* p, const void* x, const float* x_scale
     else MOE_CUDA(cudaMemsetAsync(acc, 0, static_cast<size_t>(p->T) * p->H * sizeof(float), st));
     int32_t* status = at<int32_t>(ws, L.status);
     void* h = at<void>(ws, L.h);
-    MOE_CUDA(gemm_gateup_swiglu(at<void>(ws, L.x_perm), L.max_rows, offsets, counts, p->E, 0, w_gate, w_up,
-                                p->I, p->H, h, status, MOE_K_GATEUP, st));
-    MOE_CUDA(gemm_down_combine(h, L.max_rows, offsets, counts, p->E, w_down, p->H, p->I,
-                               at<int32_t>(ws, L.pair_of_row), w, p->K, acc, status, st));
+    const int cap = p->masked_cap;
+    const int32_t* sched = offsets;
+    if (cap > 0) {
+      MOE_CUDA(launch_masked_schedule(counts, p->E, at<int32_t>(ws, L.sched), st));
+      sched = at<int32_t>(ws, L.sched);
+    }
+    MOE_CUDA(gemm_gateup_swiglu(at<void>(ws, L.x_perm), L.max_rows, sched, counts, p->E, 0, w_gate, w_up,
+                                p->I, p->H, h, status, MOE_K_GATEUP, st, cap));
+    MOE_CUDA(gemm_down_combine(h, L.max_rows, sched, counts, p->E, w_down, p->H, p->I,
+                               at<int32_t>(ws, L.pair_of_row), w, p->K, acc, status, st, cap));
     return cuda_status(launch_f32_to_bf16(acc, static_cast<long long>(p->T) * p->H, out, st));
   }
   if (is_fp8(p))
@@ -385,12 +410,19 @@ moe_status_t moe_expert_ffn(const moe_params_t* p, const void* x_perm, const flo
                             void* ws, size_t ws_bytes, void* stream) {
   MOE_TRY(validate(p));
   MOE_TRY(check_ws(p, ws, ws_bytes, false));
-  if (!x_perm || !offsets_padded || !w_gate || !w_up || !w_down || !y_perm) return MOE_ERR_INVALID_ARG;
+  if (!x_perm || !w_gate || !w_up || !w_down || !y_perm) return MOE_ERR_INVALID_ARG;
+  if (p->masked_cap > 0 ? !counts : !offsets_padded) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x_perm) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down) || !aligned16(y_perm))
     return MOE_ERR_INVALID_ARG;
   if (is_fp8(p) && (!x_perm_scale || !w_gate_scale || !w_up_scale || !w_down_scale))
     return MOE_ERR_INVALID_ARG;
   if (p->T == 0) return MOE_OK;
+  if (offsets_padded == nullptr) {  // masked layout: expert e's rows start at e*cap
+    const Layout L = layout(p);
+    int32_t* offs = at<int32_t>(ws, L.offsets);
+    MOE_CUDA(launch_masked_offsets(p->E, p->masked_cap, offs, static_cast<cudaStream_t>(stream)));
+    offsets_padded = offs;
+  }
   if (is_fp8(p))
     return do_expert_ffn_fp8(p, x_perm, x_perm_scale, offsets_padded, counts, w_gate, w_up, w_down,
                              w_gate_scale, w_up_scale, w_down_scale, y_perm, ws,
@@ -536,6 +568,7 @@ int32_t moe_layer_launch_count(const moe_params_t* p) {
   n += 2;                                    // gate/up, down
   if (p->I_shared > 0) n += 2;               // shared gate/up, down
   n += 1;                                    // combine
+  if (p->masked_cap > 0) n += 1;             // compact GEMM schedule of the masked layout
   return n;
 }
 

@@ -103,7 +103,7 @@ cudaError_t gemm_router(const void* x, const void* w_r, int T, int H, int E, flo
 cudaError_t gemm_gateup_swiglu(const void* A, int64_t a_rows, const int32_t* offsets,
                                const int32_t* counts, int G, int dense_rows, const void* w_gate,
                                const void* w_up, int N, int K, void* h, int32_t* status, int kid,
-                               cudaStream_t st) {
+                               cudaStream_t st, int masked_cap) {
   using Cfg = GemmCfg<256, EPI_SWIGLU, 4>;
   CUtensorMap ta, tg, tu;
   if (!make_tmap_bf16(&ta, A, a_rows, K, 128) ||
@@ -121,13 +121,14 @@ cudaError_t gemm_gateup_swiglu(const void* A, int64_t a_rows, const int32_t* off
   gp.out = h;
   gp.ldo = N;
   gp.status = status;
+  gp.masked_cap = masked_cap;
   const long long items = ceil_div(a_rows, 128) * ceil_div(N, Cfg::OUT_COLS);
   return launch<Cfg>(ta, tg, tu, gp, items, kid, st);
 }
 
 cudaError_t gemm_down(const void* A, int64_t a_rows, const int32_t* offsets,
                       const int32_t* counts, int G, int dense_rows, const void* w, int N, int K,
-                      float* y, int32_t* status, int kid, cudaStream_t st) {
+                      float* y, int32_t* status, int kid, cudaStream_t st, int masked_cap) {
   CUtensorMap ta, tb;
   const bool wide = N % 256 == 0;
   if (!make_tmap_bf16(&ta, A, a_rows, K, 128) ||
@@ -144,6 +145,7 @@ cudaError_t gemm_down(const void* A, int64_t a_rows, const int32_t* offsets,
   gp.out = y;
   gp.ldo = N;
   gp.status = status;
+  gp.masked_cap = masked_cap;
   if (wide) {
     using Cfg = GemmCfg<256, EPI_F32, 4>;
     return launch<Cfg>(ta, tb, tb, gp, ceil_div(a_rows, 128) * ceil_div(N, 256), kid, st);
@@ -154,7 +156,8 @@ cudaError_t gemm_down(const void* A, int64_t a_rows, const int32_t* offsets,
 
 cudaError_t gemm_down_combine(const void* A, int64_t a_rows, const int32_t* offsets, const int32_t* counts,
                               int G, const void* w, int N, int K, const int32_t* pair_of_row,
-                              const float* pair_weight, int topk, float* acc, int32_t* status, cudaStream_t st) {
+                              const float* pair_weight, int topk, float* acc, int32_t* status, cudaStream_t st,
+                              int masked_cap) {
   CUtensorMap ta, tb;
   const bool wide = N % 256 == 0;
   if (!make_tmap_bf16(&ta, A, a_rows, K, 128) ||
@@ -174,6 +177,7 @@ cudaError_t gemm_down_combine(const void* A, int64_t a_rows, const int32_t* offs
   gp.pair_of_row = pair_of_row;
   gp.pair_weight = pair_weight;
   gp.topk = topk;
+  gp.masked_cap = masked_cap;
   if (wide) {
     using Cfg = GemmCfg<256, EPI_COMBINE, 4>;
     return launch<Cfg>(ta, tb, tb, gp, ceil_div(a_rows, 128) * ceil_div(N, 256), MOE_K_DOWN, st);

@@ -119,7 +119,7 @@ cudaError_t gemm_gateup_swiglu_fp8(const void* A, const uint8_t* a_atoms, int64_
                                    const int32_t* offsets, const int32_t* counts, int G,
                                    const void* w_gate, const void* w_up, const uint8_t* gate_atoms,
                                    const uint8_t* up_atoms, int N, int K, void* h, uint8_t* h_atoms,
-                                   int32_t* status, cudaStream_t st) {
+                                   int32_t* status, cudaStream_t st, int masked_cap) {
   using Cfg = Fp8Cfg<256, EPI8_SWIGLU_Q, 4>;
   CUtensorMap ta, tg, tu;
   if (!make_tmap_u8(&ta, A, a_rows, K, 128) ||
@@ -139,13 +139,14 @@ cudaError_t gemm_gateup_swiglu_fp8(const void* A, const uint8_t* a_atoms, int64_
   fp.ldo = N;
   fp.out_sf = h_atoms;
   fp.status = status;
+  fp.masked_cap = masked_cap;
   return launch8<Cfg>(ta, tg, tu, fp, cdiv(a_rows, 128) * cdiv(N, 128), MOE_K_GATEUP, st);
 }
 
 cudaError_t gemm_down_fp8(const void* A, const uint8_t* a_atoms, int64_t a_rows,
                           const int32_t* offsets, const int32_t* counts, int G, const void* w,
                           const uint8_t* w_atoms, int N, int K, void* y, int32_t* status,
-                          cudaStream_t st) {
+                          cudaStream_t st, int masked_cap) {
   using Cfg = Fp8Cfg<128, EPI8_BF16, 5>;
   CUtensorMap ta, tb;
   if (!make_tmap_u8(&ta, A, a_rows, K, 128) || !make_tmap_u8(&tb, w, static_cast<uint64_t>(G) * N, K, 128))
@@ -163,6 +164,7 @@ cudaError_t gemm_down_fp8(const void* A, const uint8_t* a_atoms, int64_t a_rows,
   fp.ldo = N;
   fp.out_sf = nullptr;
   fp.status = status;
+  fp.masked_cap = masked_cap;
   return launch8<Cfg>(ta, tb, tb, fp, cdiv(a_rows, 128) * cdiv(N, 128), MOE_K_DOWN, st);
 }
 

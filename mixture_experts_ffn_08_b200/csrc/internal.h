@@ -30,6 +30,12 @@ cudaError_t launch_topk(const float* logits, const moe_params_t& p, const float*
 cudaError_t launch_bias_update(const int32_t* counts, int E, float gamma, float* bias, cudaStream_t st);
 
 // ---------------------------------------------------------------- dispatch (kernels.cu)
+// Masked layout with a compact GEMM schedule: with masked_cap > 0 the grouped GEMMs take
+// `offsets` as the schedule, the 128-padded prefix sums of counts (masked_schedule), and
+// address group g's rows at g * masked_cap.
+cudaError_t launch_masked_schedule(const int32_t* counts, int E, int32_t* sched, cudaStream_t st);
+// offsets[e] = e * cap for e in [0, E] (masked layout row ranges).
+cudaError_t launch_masked_offsets(int E, int cap, int32_t* offsets, cudaStream_t st);
 cudaError_t launch_permute(const moe_params_t& p, int block_m, const int32_t* ids, const void* x,
                            const float* x_scale, int32_t* counts, int32_t* offsets,
                            int32_t* row_of_pair, int32_t* pair_of_row, void* x_perm,
@@ -50,18 +56,19 @@ cudaError_t gemm_router(const void* x, const void* w_r, int T, int H, int E, flo
 cudaError_t gemm_gateup_swiglu(const void* A, int64_t a_rows, const int32_t* offsets,
                                const int32_t* counts, int G, int dense_rows, const void* w_gate,
                                const void* w_up, int N, int K, void* h, int32_t* status, int kid,
-                               cudaStream_t st);
+                               cudaStream_t st, int masked_cap = 0);
 // y [rows, N] fp32 = A W^T, grouped by offsets (or dense when null); with counts, pad
 // rows of each group are not stored.
 cudaError_t gemm_down(const void* A, int64_t a_rows, const int32_t* offsets,
                       const int32_t* counts, int G, int dense_rows, const void* w, int N, int K,
-                      float* y, int32_t* status, int kid, cudaStream_t st);
+                      float* y, int32_t* status, int kid, cudaStream_t st, int masked_cap = 0);
 
 // acc[t] += w[p] * (A W^T)[r] for every bucket row r of pair p = pair_of_row[r], t = p / topk
 // (down projection fused with the combine; fp32 vector reductions, order not fixed).
 cudaError_t gemm_down_combine(const void* A, int64_t a_rows, const int32_t* offsets, const int32_t* counts,
                               int G, const void* w, int N, int K, const int32_t* pair_of_row,
-                              const float* pair_weight, int topk, float* acc, int32_t* status, cudaStream_t st);
+                              const float* pair_weight, int topk, float* acc, int32_t* status, cudaStream_t st,
+                              int masked_cap = 0);
 // out[i] = bf16(acc[i]) for n values (n multiple of 8).
 cudaError_t launch_f32_to_bf16(const float* acc, long long n, void* out, cudaStream_t st);
 
@@ -76,12 +83,12 @@ cudaError_t gemm_gateup_swiglu_fp8(const void* A, const uint8_t* a_atoms, int64_
                                    const int32_t* offsets, const int32_t* counts, int G,
                                    const void* w_gate, const void* w_up, const uint8_t* gate_atoms,
                                    const uint8_t* up_atoms, int N, int K, void* h, uint8_t* h_atoms,
-                                   int32_t* status, cudaStream_t st);
+                                   int32_t* status, cudaStream_t st, int masked_cap = 0);
 // y [rows, N] bf16 = A W^T, block-scaled e4m3 GEMM.
 cudaError_t gemm_down_fp8(const void* A, const uint8_t* a_atoms, int64_t a_rows,
                           const int32_t* offsets, const int32_t* counts, int G, const void* w,
                           const uint8_t* w_atoms, int N, int K, void* y, int32_t* status,
-                          cudaStream_t st);
+                          cudaStream_t st, int masked_cap = 0);
 
 // ---------------------------------------------------------------- two-SM GEMMs (gemm_2cta.cu)
 cudaError_t gemm_pair_gateup_swiglu(const void* A, int64_t a_rows, const int32_t* offsets, const int32_t* counts,

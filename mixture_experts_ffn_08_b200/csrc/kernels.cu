@@ -331,16 +331,18 @@ __global__ void __launch_bounds__(kPermChunk) perm_count_kernel(
 
 // 2) one block: expert totals, padded exclusive scan -> offsets, and per-chunk bases
 //    (chunk_counts is overwritten with the first row of each (chunk, expert) run).
+//    cap > 0 (masked layout): every expert spans cap rows, counts are capped at cap.
 __global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t* __restrict__ chunk_counts,
-                                                         int nchunks, int E, int block_m,
+                                                         int nchunks, int E, int block_m, int cap,
                                                          int32_t* __restrict__ counts,
-                                                         int32_t* __restrict__ offsets) {
+                                                         int32_t* __restrict__ offsets,
+                                                         int32_t* status) {
   __shared__ int warp_tot[32];
   const int e = threadIdx.x, lane = e & 31, w = e >> 5;
   int total = 0;
   if (e < E)
     for (int c = 0; c < nchunks; ++c) total += chunk_counts[static_cast<long long>(c) * E + e];
-  const int padded = e < E ? (total + block_m - 1) / block_m * block_m : 0;
+  const int padded = e >= E ? 0 : cap > 0 ? cap : (total + block_m - 1) / block_m * block_m;
   // inclusive scan of `padded` across the block
   int v = padded;
 #pragma unroll
@@ -363,7 +365,8 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t* __restrict__ c
   const int incl = v + (w > 0 ? warp_tot[w - 1] : 0);
   const int excl = incl - padded;
   if (e < E) {
-    counts[e] = total;
+    if (cap > 0 && total > cap) set_status(status, MOE_DEV_CAPACITY);
+    counts[e] = cap > 0 && total > cap ? cap : total;
     offsets[e] = excl;
     int run = excl;
     for (int c = 0; c < nchunks; ++c) {
@@ -379,8 +382,9 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t* __restrict__ c
 // 3) stable rank inside each chunk: one warp per chunk walks its pairs in order,
 //    32 at a time; lanes with the same expert are ranked by lane (warp match).
 constexpr int kRankWarps = 4;
+//    cap > 0 (masked layout): a pair whose row falls past its expert's cap rows gets none.
 __global__ void __launch_bounds__(32 * kRankWarps) perm_rank_kernel(
-    const int32_t* __restrict__ ids, int P, int E, const int32_t* __restrict__ chunk_base,
+    const int32_t* __restrict__ ids, int P, int E, int cap, const int32_t* __restrict__ chunk_base,
     int32_t* __restrict__ row_of_pair, int32_t* __restrict__ pair_of_row) {
   extern __shared__ int run_cnt[];  // [kRankWarps][E]
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -401,8 +405,9 @@ __global__ void __launch_bounds__(32 * kRankWarps) perm_rank_kernel(
     __syncwarp();
     if (ok) {
       const int row = __ldg(base + e) + run + rank;
-      row_of_pair[p] = row;
-      pair_of_row[row] = p;
+      const bool kept = cap <= 0 || row < (e + 1) * cap;
+      row_of_pair[p] = kept ? row : -1;
+      if (kept) pair_of_row[row] = p;
       if (rank == 0) my[e] = run + __popc(peers);
     } else if (p < P) {
       row_of_pair[p] = -1;
@@ -411,13 +416,14 @@ __global__ void __launch_bounds__(32 * kRankWarps) perm_rank_kernel(
   }
 }
 
-// 4) row gather: x_perm[r] = x[pair_of_row[r] / K]; pad rows -> zero, pair -1.
+// 4) row gather: x_perm[r] = x[pair_of_row[r] / K]; pad rows -> pair -1 and, unless
+//    zero_pad is false (masked layout: unused rows are left as they are), zero.
 template <bool FP8>
 __global__ void __launch_bounds__(256) perm_gather_kernel(
     const void* __restrict__ x, const float* __restrict__ x_scale, int H, int K, int E,
     const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets,
     int32_t* __restrict__ pair_of_row, void* __restrict__ x_perm,
-    float* __restrict__ x_perm_scale) {
+    float* __restrict__ x_perm_scale, bool zero_pad) {
   const int total = __ldg(offsets + E);
   const int row_bytes = FP8 ? H : 2 * H;
   const int nvec = row_bytes / 16;
@@ -431,6 +437,7 @@ __global__ void __launch_bounds__(256) perm_gather_kernel(
     const bool pad = r - __ldg(offsets + lo) >= __ldg(counts + lo);
     const long long t = pad ? 0 : pair_of_row[r] / K;
     if (pad && threadIdx.x == 0) pair_of_row[r] = -1;
+    if (pad && !zero_pad) continue;
     uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(x_perm) + static_cast<long long>(r) * row_bytes);
     const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(x) + t * row_bytes);
     for (int v = threadIdx.x; v < nvec; v += blockDim.x)
@@ -458,27 +465,72 @@ cudaError_t launch_permute(const moe_params_t& p, int block_m, const int32_t* id
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
   trace_before(MOE_K_PERM_SCAN, st);
-  perm_scan_kernel<<<1, 1024, 0, st>>>(chunk_counts, nchunks, p.E, bm, counts, offsets);
+  perm_scan_kernel<<<1, 1024, 0, st>>>(chunk_counts, nchunks, p.E, bm, p.masked_cap, counts, offsets, status);
   trace_after(MOE_K_PERM_SCAN, st);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   if (nchunks > 0) {
     trace_before(MOE_K_PERM_RANK, st);
     const int blocks = (nchunks + kRankWarps - 1) / kRankWarps;
     perm_rank_kernel<<<blocks, 32 * kRankWarps, kRankWarps * p.E * sizeof(int), st>>>(
-        ids, P, p.E, chunk_counts, row_of_pair, pair_of_row);
+        ids, P, p.E, p.masked_cap, chunk_counts, row_of_pair, pair_of_row);
     trace_after(MOE_K_PERM_RANK, st);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
-  const long long max_rows = static_cast<long long>(P) + static_cast<long long>(p.E) * (bm - 1);
+  const bool masked = p.masked_cap > 0;
+  const long long max_rows = masked ? static_cast<long long>(p.E) * p.masked_cap
+                                    : static_cast<long long>(P) + static_cast<long long>(p.E) * (bm - 1);
   const int grid = static_cast<int>(max_rows < num_sms() * 16LL ? (max_rows > 0 ? max_rows : 1) : num_sms() * 16LL);
   trace_before(MOE_K_PERM_GATHER, st);
   if (p.dtype == MOE_DTYPE_FP8_E4M3)
     perm_gather_kernel<true><<<grid, 256, 0, st>>>(x, x_scale, p.H, p.K, p.E, counts, offsets,
-                                                   pair_of_row, x_perm, x_perm_scale);
+                                                   pair_of_row, x_perm, x_perm_scale, !masked);
   else
     perm_gather_kernel<false><<<grid, 256, 0, st>>>(x, x_scale, p.H, p.K, p.E, counts, offsets,
-                                                    pair_of_row, x_perm, x_perm_scale);
+                                                    pair_of_row, x_perm, x_perm_scale, !masked);
   trace_after(MOE_K_PERM_GATHER, st);
+  return cudaGetLastError();
+}
+
+// sched[e] = sum over j < e of counts[j] rounded up to 128 (one block, E <= 1024).
+__global__ void __launch_bounds__(1024) masked_schedule_kernel(const int32_t* __restrict__ counts, int E,
+                                                               int32_t* __restrict__ sched) {
+  __shared__ int warp_tot[32];
+  const int e = threadIdx.x, lane = e & 31, w = e >> 5;
+  const int padded = e < E ? (__ldg(counts + e) + 127) / 128 * 128 : 0;
+  int v = padded;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(kFull, v, o);
+    if (lane >= o) v += n;
+  }
+  if (lane == 31) warp_tot[w] = v;
+  __syncthreads();
+  if (w == 0) {
+    int t = warp_tot[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(kFull, t, o);
+      if (lane >= o) t += n;
+    }
+    warp_tot[lane] = t;
+  }
+  __syncthreads();
+  const int incl = v + (w > 0 ? warp_tot[w - 1] : 0);
+  if (e < E) sched[e] = incl - padded;
+  if (e == E - 1) sched[E] = incl;
+}
+
+cudaError_t launch_masked_schedule(const int32_t* counts, int E, int32_t* sched, cudaStream_t st) {
+  masked_schedule_kernel<<<1, 1024, 0, st>>>(counts, E, sched);
+  return cudaGetLastError();
+}
+
+__global__ void masked_offsets_kernel(int E, int cap, int32_t* __restrict__ offsets) {
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e <= E; e += gridDim.x * blockDim.x) offsets[e] = e * cap;
+}
+
+cudaError_t launch_masked_offsets(int E, int cap, int32_t* offsets, cudaStream_t st) {
+  masked_offsets_kernel<<<(E + 256) / 256, 256, 0, st>>>(E, cap, offsets);
   return cudaGetLastError();
 }
 

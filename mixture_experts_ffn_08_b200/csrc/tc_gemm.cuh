@@ -59,6 +59,9 @@ struct GemmParams {
   const int32_t* pair_of_row;  // EPI_COMBINE: pair of each bucket row
   const float* pair_weight;    // EPI_COMBINE: combine weight of each pair [T*K]
   int topk;                    // EPI_COMBINE: K (pair p belongs to token p / K)
+  int masked_cap;              // > 0: masked layout.  offsets is then only the schedule (the
+                               // compact 128-padded prefix of counts); group g's rows sit at
+                               // g * masked_cap in A and out
 };
 
 MOE_DEVINL void red_add_v4(float* addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d, float w) {
@@ -89,9 +92,11 @@ struct GemmCfg {
 };
 
 struct TileCoord {
-  int m_tile;
+  int m_tile;  // position in the schedule
   int n_tile;
   int group;
+  int local0;  // first row of the tile inside its group
+  int row0;    // first row of the tile in A and out
 };
 
 // Work item -> (M-tile, N-tile, group).  Items of group g occupy [mt0*NT, mt1*NT) where
@@ -115,6 +120,8 @@ MOE_DEVINL TileCoord decode_item(int item, int NT, const GemmParams& p, int num_
   t.m_tile = mt0 + local % cnt;
   t.n_tile = local / cnt;
   t.group = g;
+  t.local0 = (t.m_tile - mt0) * 128;
+  t.row0 = p.masked_cap > 0 ? g * p.masked_cap + t.local0 : t.m_tile * 128;
   return t;
 }
 
@@ -181,7 +188,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       bool ok = true;
       for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
         const TileCoord t = decode_item(item, NT, p, num_m_tiles);
-        const int a_row = t.m_tile * BM;
+        const int a_row = t.row0;
         const int b_row = t.group * p.b_rows_per_group + t.n_tile * Cfg::OUT_COLS;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, &abort_flag)) { ok = false; break; }
@@ -254,11 +261,11 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       if (!ready) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * Cfg::ACC_COLS;
-      const long long row = static_cast<long long>(t.m_tile) * BM + q * 32 + lane;
+      const long long row = static_cast<long long>(t.row0) + q * 32 + lane;
       bool row_ok;
       if (p.offsets == nullptr) row_ok = row < p.dense_rows;
       else if (p.counts == nullptr) row_ok = true;
-      else row_ok = row - __ldg(p.offsets + t.group) < __ldg(p.counts + t.group);
+      else row_ok = t.local0 + q * 32 + lane < __ldg(p.counts + t.group);
       const int col0 = t.n_tile * Cfg::OUT_COLS;
 
       if constexpr (Cfg::EPI == EPI_SWIGLU) {

@@ -108,6 +108,8 @@ struct Fp8Params {
   int64_t ldo;             // elements
   uint8_t* out_sf;         // SwiGLU: h scale atoms [m_tiles][ceil(N/512)][512]
   int32_t* status;
+  int masked_cap;          // > 0: masked layout (offsets = compact schedule; rows of group g
+                           // at g * masked_cap), as in GemmParams
 };
 
 template <int BN_, int EPI_, int STAGES_>
@@ -179,6 +181,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   GemmParams gp{};
   gp.offsets = p.offsets;
   gp.G = p.G;
+  gp.masked_cap = p.masked_cap;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -218,7 +221,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       const int nblk = p.N / 128;  // 128-row weight blocks per group
       for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
         const TileCoord t = decode_item(item, NT, gp, num_m_tiles);
-        const int a_row = t.m_tile * BM;
+        const int a_row = t.row0;
         const int b_row = t.group * p.N + t.n_tile * Cfg::OUT_COLS;
         const int wblk = t.group * nblk + (t.n_tile * Cfg::OUT_COLS) / 128;
         for (int kb = 0; kb < KB; ++kb) {
@@ -237,7 +240,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           }
           if (new_sf) {
             const int kb4 = kb >> 2;
-            bulk_load(ssf, p.sfa + (static_cast<size_t>(t.m_tile) * KB4 + kb4) * 512, 512, &full_bar[s]);
+            bulk_load(ssf, p.sfa + (static_cast<size_t>(t.row0 / BM) * KB4 + kb4) * 512, 512, &full_bar[s]);
             const size_t wsf = (static_cast<size_t>(wblk) * KB4 + kb4) * 512;
             if (Cfg::EPI == EPI8_SWIGLU_Q) {
               bulk_load(ssf + 512, p.sfb0 + wsf, 512, &full_bar[s]);
@@ -315,9 +318,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * Cfg::ACC_COLS;
       const int row_in_tile = q * 32 + lane;
-      const long long row = static_cast<long long>(t.m_tile) * BM + row_in_tile;
-      const bool row_ok = p.counts == nullptr ||
-                          row - __ldg(p.offsets + t.group) < __ldg(p.counts + t.group);
+      const long long row = static_cast<long long>(t.row0) + row_in_tile;
+      const bool row_ok = p.counts == nullptr || t.local0 + row_in_tile < __ldg(p.counts + t.group);
       const int col0 = t.n_tile * Cfg::OUT_COLS;
 
       if constexpr (Cfg::EPI == EPI8_SWIGLU_Q) {
@@ -351,9 +353,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                 e4m3x4(hv[12] * inv, hv[13] * inv, hv[14] * inv, hv[15] * inv));
           }
         }
-        // byte (n_tile % 4) of this row's word in atom (m_tile, n_tile / 4) of the down GEMM
+        // byte (n_tile % 4) of this row's word in atom (row0 / 128, n_tile / 4) of the down GEMM
         const int kb4n = (p.N / 128 + 3) / 4;
-        uint8_t* sf = p.out_sf + (static_cast<size_t>(t.m_tile) * kb4n + (t.n_tile >> 2)) * 512;
+        uint8_t* sf = p.out_sf + (static_cast<size_t>(t.row0 / BM) * kb4n + (t.n_tile >> 2)) * 512;
         sf[sf_atom_offset(row_in_tile) + (t.n_tile & 3)] = static_cast<uint8_t>(e + 127);
       } else {
         __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + row * p.ldo + col0;

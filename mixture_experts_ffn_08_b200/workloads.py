@@ -39,6 +39,7 @@ class Workload:
     skewed: bool = False    # Zipf-shaped router for the skew stress case
     block_m: int = 0        # bucket row alignment: 128, 256 (two-SM GEMM tiles), 0 = library choice
     fused_combine: bool = False  # down projection adds into the output (atomic, non-deterministic)
+    masked_cap: int = 0     # 0 = contiguous buckets; > 0 = masked layout, expert e owns rows [e*cap, (e+1)*cap)
 
     @property
     def P(self) -> int:

@@ -38,7 +38,7 @@ def test_exports_every_declared_symbol(lib):
     for name in declared:
         assert hasattr(raw, name), name
     assert declared == set(B.EXPORTED), declared ^ set(B.EXPORTED)
-    assert lib.moe_abi_version() == 2
+    assert lib.moe_abi_version() == 3
 
 
 def test_params_struct_matches_header():
@@ -60,6 +60,17 @@ def test_sizes(lib):
         assert ws >= rows * wl.H * (1 if wl.dtype else 2) * 2
         assert B.moe_workspace_size_host(p) > ws
         assert B.moe_layer_launch_count(p) == 9 + (2 if wl.I_shared else 0) + (5 if wl.dtype else 0)
+
+
+def test_masked_layout_sizes(lib):
+    wl = W.DSV3_DECODE.with_(masked_cap=128)
+    p = B.params(wl)
+    assert B.moe_max_padded_rows(p) == wl.E * 128
+    assert B.moe_effective_block_m(p) == 128
+    assert B.moe_workspace_size(p) >= wl.E * 128 * wl.H * 4
+    for bad in (dict(masked_cap=100), dict(masked_cap=128, block_m=256), dict(masked_cap=-128)):
+        q = B.params(wl.with_(**bad))
+        assert B.moe_workspace_size(q) == 0 and B.moe_max_padded_rows(q) == -1
 
 
 @pytest.mark.parametrize("change", [dict(H=100), dict(I=200), dict(K=0), dict(E=2000), dict(block_m=64),
