@@ -147,9 +147,12 @@ cudaError_t gemm_down_fp8(const void* A, const uint8_t* a_atoms, int64_t a_rows,
                           const int32_t* offsets, const int32_t* counts, int G, const void* w,
                           const uint8_t* w_atoms, int N, int K, void* y, int32_t* status,
                           cudaStream_t st, int masked_cap) {
-  using Cfg = Fp8Cfg<128, EPI8_BF16, 5>;
+  // 256-column tiles (one accumulator) read A half as often per output as 128-column
+  // ones; they need whole 256-row weight slices, so N % 256 == 0.
+  const bool wide = N % 256 == 0;
   CUtensorMap ta, tb;
-  if (!make_tmap_u8(&ta, A, a_rows, K, 128) || !make_tmap_u8(&tb, w, static_cast<uint64_t>(G) * N, K, 128))
+  if (!make_tmap_u8(&ta, A, a_rows, K, 128) ||
+      !make_tmap_u8(&tb, w, static_cast<uint64_t>(G) * N, K, wide ? 256 : 128))
     return cudaErrorInvalidValue;
   Fp8Params fp{};
   fp.offsets = offsets;
@@ -165,6 +168,11 @@ cudaError_t gemm_down_fp8(const void* A, const uint8_t* a_atoms, int64_t a_rows,
   fp.out_sf = nullptr;
   fp.status = status;
   fp.masked_cap = masked_cap;
+  if (wide) {
+    using Cfg = Fp8Cfg<256, EPI8_BF16, 4>;
+    return launch8<Cfg>(ta, tb, tb, fp, cdiv(a_rows, 128) * cdiv(N, 256), MOE_K_DOWN, st);
+  }
+  using Cfg = Fp8Cfg<128, EPI8_BF16, 5>;
   return launch8<Cfg>(ta, tb, tb, fp, cdiv(a_rows, 128) * cdiv(N, 128), MOE_K_DOWN, st);
 }
 

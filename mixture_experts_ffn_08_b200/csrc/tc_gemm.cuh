@@ -275,7 +275,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           uint32_t rg[32], ru[32];
           tmem_ld_32x32b_x32(tbase + c, rg);
           tmem_ld_32x32b_x32(tbase + BN / 2 + c, ru);
-          tmem_ld_wait();
+          tmem_ld_wait(rg);
+          reg_fence(ru);
           uint32_t packed[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
@@ -299,7 +300,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         for (int c = 0; c < BN; c += 32) {
           uint32_t r[32];
           tmem_ld_32x32b_x32(tbase + c, r);
-          tmem_ld_wait();
+          tmem_ld_wait(r);
           if (pair >= 0 && col0 + c < p.N) {
 #pragma unroll
             for (int v = 0; v < 8; ++v) red_add_v4(out + c + 4 * v, r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3], wgt);
@@ -311,7 +312,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         for (int c = 0; c < BN; c += 32) {
           uint32_t r[32];
           tmem_ld_32x32b_x32(tbase + c, r);
-          tmem_ld_wait();
+          tmem_ld_wait(r);
           if (row_ok && col0 + c < p.N) {
             uint32_t packed[16];
 #pragma unroll
@@ -329,7 +330,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         for (int c = 0; c < BN; c += 16) {
           uint32_t r[16];
           tmem_ld_32x32b_x16(tbase + c, r);
-          tmem_ld_wait();
+          tmem_ld_wait(r);
           if (row_ok) {
             if (col0 + c + 16 <= p.N && (p.ldo & 3) == 0) {
               uint4* dst = reinterpret_cast<uint4*>(out + c);

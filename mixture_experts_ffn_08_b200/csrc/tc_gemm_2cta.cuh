@@ -384,7 +384,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           uint32_t rg[32], ru[32];
           tmem_ld_32x32b_x32(tbase + c, rg);
           tmem_ld_32x32b_x32(tbase + BN / 2 + c, ru);
-          tmem_ld_wait();
+          tmem_ld_wait(rg);
+          reg_fence(ru);
           uint32_t packed[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i)
@@ -405,7 +406,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           uint32_t rg[32], ru[32];
           tmem_ld_32x32b_x32(tbase + c, rg);
           tmem_ld_32x32b_x32(tbase + 128 + c, ru);
-          tmem_ld_wait();
+          tmem_ld_wait(rg);
+          reg_fence(ru);
 #pragma unroll
           for (int i = 0; i < 32; ++i) h[c + i] = silu_mul(__uint_as_float(rg[i]), __uint_as_float(ru[i]));
         }
@@ -436,7 +438,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         for (int c = 0; c < BN; c += 32) {
           uint32_t r[32];
           tmem_ld_32x32b_x32(tbase + c, r);
-          tmem_ld_wait();
+          tmem_ld_wait(r);
           if (row_ok && col0 + c < p.N) {
             uint4* dst = reinterpret_cast<uint4*>(out + c);
 #pragma unroll
@@ -450,7 +452,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         for (int c = 0; c < BN; c += 32) {
           uint32_t r[32];
           tmem_ld_32x32b_x32(tbase + c, r);
-          tmem_ld_wait();
+          tmem_ld_wait(r);
           if (row_ok && col0 + c < p.N) {
             uint32_t packed[16];
 #pragma unroll

@@ -126,7 +126,9 @@ struct Fp8Cfg {
   static constexpr int STAGE_BYTES = (A_BYTES + B_BYTES + SF_BYTES + 1023) / 1024 * 1024;
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
   static constexpr int OUT_COLS = EPI == EPI8_SWIGLU_Q ? BN / 2 : BN;
-  static constexpr int ACC_STAGES = EPI == EPI8_SWIGLU_Q ? 1 : 2;
+  // TMEM holds 512 columns: two 256-column accumulators would leave none for the scales,
+  // so 256-column tiles keep one and their epilogue hands it back as soon as it is read.
+  static constexpr int ACC_STAGES = BN == 256 ? 1 : 2;
   static constexpr int ACC_COLS = BN;
   static constexpr int SF_COL = ACC_STAGES * ACC_COLS;      // A scales; B scales at +4
   static constexpr int TMEM_COLS = 512;
@@ -323,19 +325,40 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       const int col0 = t.n_tile * Cfg::OUT_COLS;
 
       if constexpr (Cfg::EPI == EPI8_SWIGLU_Q) {
+        // h = SiLU(g) * u in fp32 (h is rounded to e4m3 next, and an intermediate rounding
+        // of g, u or h would move some values across e4m3 rounding boundaries).  The
+        // first 64 columns are computed while the accumulator is held; the last 64 are
+        // read raw into registers, the accumulator goes back to the MMA warp, and their
+        // SwiGLU runs after the release.
         float h[128];
 #pragma unroll
-        for (int c = 0; c < 128; c += 32) {
+        for (int c = 0; c < 64; c += 32) {
           uint32_t rg[32], ru[32];
           tmem_ld_32x32b_x32(tbase + c, rg);
           tmem_ld_32x32b_x32(tbase + 128 + c, ru);
-          tmem_ld_wait();
+          tmem_ld_wait(rg);
+          reg_fence(ru);
 #pragma unroll
           for (int i = 0; i < 32; ++i) h[c + i] = silu_mul(__uint_as_float(rg[i]), __uint_as_float(ru[i]));
         }
-        // accumulator read: hand TMEM back to the MMA warp before quantising
-        tc_fence_before();
-        mbar_arrive(&tempty_bar[acc]);
+        {
+          uint32_t rg0[32], ru0[32], rg1[32], ru1[32];
+          tmem_ld_32x32b_x32(tbase + 64, rg0);
+          tmem_ld_32x32b_x32(tbase + 128 + 64, ru0);
+          tmem_ld_32x32b_x32(tbase + 96, rg1);
+          tmem_ld_32x32b_x32(tbase + 128 + 96, ru1);
+          tmem_ld_wait(rg0);
+          reg_fence(ru0);
+          reg_fence(rg1);
+          reg_fence(ru1);
+          tc_fence_before();
+          mbar_arrive(&tempty_bar[acc]);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            h[64 + i] = silu_mul(__uint_as_float(rg0[i]), __uint_as_float(ru0[i]));
+            h[96 + i] = silu_mul(__uint_as_float(rg1[i]), __uint_as_float(ru1[i]));
+          }
+        }
         float amax = 0.f;
 #pragma unroll
         for (int i = 0; i < 128; ++i) amax = fmaxf(amax, fabsf(h[i]));
@@ -345,25 +368,52 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           uint8_t* out = static_cast<uint8_t*>(p.out) + row * p.ldo + col0;
 #pragma unroll
           for (int v = 0; v < 8; ++v) {
-            const float* hv = h + 16 * v;
-            reinterpret_cast<uint4*>(out)[v] = make_uint4(
-                e4m3x4(hv[0] * inv, hv[1] * inv, hv[2] * inv, hv[3] * inv),
-                e4m3x4(hv[4] * inv, hv[5] * inv, hv[6] * inv, hv[7] * inv),
-                e4m3x4(hv[8] * inv, hv[9] * inv, hv[10] * inv, hv[11] * inv),
-                e4m3x4(hv[12] * inv, hv[13] * inv, hv[14] * inv, hv[15] * inv));
+            uint32_t w[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float* hv = h + 16 * v + 4 * j;
+              w[j] = e4m3x4(hv[0] * inv, hv[1] * inv, hv[2] * inv, hv[3] * inv);
+            }
+            reinterpret_cast<uint4*>(out)[v] = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
         // byte (n_tile % 4) of this row's word in atom (row0 / 128, n_tile / 4) of the down GEMM
         const int kb4n = (p.N / 128 + 3) / 4;
         uint8_t* sf = p.out_sf + (static_cast<size_t>(t.row0 / BM) * kb4n + (t.n_tile >> 2)) * 512;
         sf[sf_atom_offset(row_in_tile) + (t.n_tile & 3)] = static_cast<uint8_t>(e + 127);
+      } else if constexpr (ACC_STAGES == 1) {
+        // one accumulator: read it all as bf16 pairs, release it, then store
+        uint32_t pk[BN / 2];
+#pragma unroll
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tbase + c, r);
+          tmem_ld_wait(r);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pk[c / 2 + i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+        }
+        tc_fence_before();
+        mbar_arrive(&tempty_bar[acc]);
+        if (row_ok) {
+          __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + row * p.ldo + col0;
+#pragma unroll
+          for (int c = 0; c < BN; c += 32) {
+            if (col0 + c < p.N) {
+              uint4* dst = reinterpret_cast<uint4*>(out + c);
+#pragma unroll
+              for (int v = 0; v < 4; ++v)
+                dst[v] = make_uint4(pk[c / 2 + 4 * v], pk[c / 2 + 4 * v + 1], pk[c / 2 + 4 * v + 2],
+                                    pk[c / 2 + 4 * v + 3]);
+            }
+          }
+        }
       } else {
         __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + row * p.ldo + col0;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
           uint32_t r[32];
           tmem_ld_32x32b_x32(tbase + c, r);
-          tmem_ld_wait();
+          tmem_ld_wait(r);
           if (row_ok && col0 + c < p.N) {
             uint32_t packed[16];
 #pragma unroll
