@@ -418,32 +418,48 @@ __global__ void __launch_bounds__(32 * kRankWarps) perm_rank_kernel(
 
 // 4) row gather: x_perm[r] = x[pair_of_row[r] / K]; pad rows -> pair -1 and, unless
 //    zero_pad is false (masked layout: unused rows are left as they are), zero.
+//    One warp per row; each lane keeps up to 8 16-byte loads in flight, so the copy runs
+//    at HBM write speed rather than at the latency of one load per thread.
+constexpr int kGatherWarps = 8;
 template <bool FP8>
-__global__ void __launch_bounds__(256) perm_gather_kernel(
+__global__ void __launch_bounds__(32 * kGatherWarps) perm_gather_kernel(
     const void* __restrict__ x, const float* __restrict__ x_scale, int H, int K, int E,
     const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets,
     int32_t* __restrict__ pair_of_row, void* __restrict__ x_perm,
     float* __restrict__ x_perm_scale, bool zero_pad) {
+  const int lane = threadIdx.x & 31;
   const int total = __ldg(offsets + E);
   const int row_bytes = FP8 ? H : 2 * H;
   const int nvec = row_bytes / 16;
   const int nsc = H / 128;
-  for (int r = blockIdx.x; r < total; r += gridDim.x) {
+  const int warps = gridDim.x * kGatherWarps;
+  for (int r = blockIdx.x * kGatherWarps + (threadIdx.x >> 5); r < total; r += warps) {
     int lo = 0, hi = E - 1;  // expert owning row r: smallest e with offsets[e+1] > r
     while (lo < hi) {
       const int mid = (lo + hi) >> 1;
       if (__ldg(offsets + mid + 1) > r) hi = mid; else lo = mid + 1;
     }
     const bool pad = r - __ldg(offsets + lo) >= __ldg(counts + lo);
-    const long long t = pad ? 0 : pair_of_row[r] / K;
-    if (pad && threadIdx.x == 0) pair_of_row[r] = -1;
+    if (pad && lane == 0) pair_of_row[r] = -1;
     if (pad && !zero_pad) continue;
+    const long long t = pad ? 0 : pair_of_row[r] / K;
     uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(x_perm) + static_cast<long long>(r) * row_bytes);
     const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(x) + t * row_bytes);
-    for (int v = threadIdx.x; v < nvec; v += blockDim.x)
-      dst[v] = pad ? make_uint4(0, 0, 0, 0) : __ldg(src + v);
+    for (int v0 = 0; v0 < nvec; v0 += 32 * 8) {
+      uint4 buf[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int v = v0 + 32 * u + lane;
+        buf[u] = (v < nvec && !pad) ? __ldg(src + v) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int v = v0 + 32 * u + lane;
+        if (v < nvec) dst[v] = buf[u];
+      }
+    }
     if (FP8) {
-      for (int j = threadIdx.x; j < nsc; j += blockDim.x)
+      for (int j = lane; j < nsc; j += 32)
         x_perm_scale[static_cast<long long>(r) * nsc + j] = pad ? 1.0f : __ldg(x_scale + t * nsc + j);
     }
   }
@@ -479,13 +495,14 @@ cudaError_t launch_permute(const moe_params_t& p, int block_m, const int32_t* id
   const bool masked = p.masked_cap > 0;
   const long long max_rows = masked ? static_cast<long long>(p.E) * p.masked_cap
                                     : static_cast<long long>(P) + static_cast<long long>(p.E) * (bm - 1);
-  const int grid = static_cast<int>(max_rows < num_sms() * 16LL ? (max_rows > 0 ? max_rows : 1) : num_sms() * 16LL);
+  const long long blocks = (max_rows + kGatherWarps - 1) / kGatherWarps;
+  const int grid = static_cast<int>(blocks < num_sms() * 8LL ? (blocks > 0 ? blocks : 1) : num_sms() * 8LL);
   trace_before(MOE_K_PERM_GATHER, st);
   if (p.dtype == MOE_DTYPE_FP8_E4M3)
-    perm_gather_kernel<true><<<grid, 256, 0, st>>>(x, x_scale, p.H, p.K, p.E, counts, offsets,
+    perm_gather_kernel<true><<<grid, 32 * kGatherWarps, 0, st>>>(x, x_scale, p.H, p.K, p.E, counts, offsets,
                                                    pair_of_row, x_perm, x_perm_scale, !masked);
   else
-    perm_gather_kernel<false><<<grid, 256, 0, st>>>(x, x_scale, p.H, p.K, p.E, counts, offsets,
+    perm_gather_kernel<false><<<grid, 32 * kGatherWarps, 0, st>>>(x, x_scale, p.H, p.K, p.E, counts, offsets,
                                                     pair_of_row, x_perm, x_perm_scale, !masked);
   trace_after(MOE_K_PERM_GATHER, st);
   return cudaGetLastError();
