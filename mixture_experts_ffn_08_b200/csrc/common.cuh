@@ -220,6 +220,14 @@ MOE_DEVINL void reg_fence(uint32_t (&r)[32]) {
                : "memory");
 }
 
+// One 32-byte global store (addr 32-byte aligned): a warp storing one such segment per
+// row fills whole 32-byte sectors, where 16-byte stores to 32 rows fill half of each.
+MOE_DEVINL void st_global_v8(void* addr, const uint32_t* v) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(addr), "r"(v[0]), "r"(v[1]),
+               "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
+
 MOE_DEVINL uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

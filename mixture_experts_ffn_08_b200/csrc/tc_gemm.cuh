@@ -270,6 +270,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 
       if constexpr (Cfg::EPI == EPI_SWIGLU) {
         __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + row * p.ldo + col0;
+        const bool v8 = ((reinterpret_cast<uintptr_t>(p.out) | (static_cast<uintptr_t>(p.ldo) * 2)) & 31) == 0;
 #pragma unroll 1
         for (int c = 0; c < BN / 2; c += 32) {
           uint32_t rg[32], ru[32];
@@ -285,10 +286,15 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             packed[i] = pack_bf16x2(h0, h1);
           }
           if (row_ok && col0 + c < p.N) {
-            uint4* dst = reinterpret_cast<uint4*>(out + c);
+            if (v8) {
+              st_global_v8(out + c, packed);
+              st_global_v8(out + c + 16, packed + 8);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(out + c);
 #pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+              for (int v = 0; v < 4; ++v)
+                dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+            }
           }
         }
       } else if constexpr (Cfg::EPI == EPI_COMBINE) {
@@ -322,6 +328,25 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 #pragma unroll
             for (int v = 0; v < 4; ++v)
               dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+          }
+        }
+      } else if constexpr (BN % 32 == 0) {
+        float* out = static_cast<float*>(p.out) + row * p.ldo + col0;
+        const bool v8 = ((reinterpret_cast<uintptr_t>(p.out) | (static_cast<uintptr_t>(p.ldo) * 4)) & 31) == 0;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tbase + c, r);
+          tmem_ld_wait(r);
+          if (row_ok) {
+            if (v8 && col0 + c + 32 <= p.N) {
+#pragma unroll
+              for (int v = 0; v < 4; ++v) st_global_v8(out + c + 8 * v, r + 8 * v);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (col0 + c + i < p.N) out[c + i] = __uint_as_float(r[i]);
+            }
           }
         }
       } else {

@@ -366,15 +366,21 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         const float inv = ldexpf(1.f, -e);
         if (row_ok) {
           uint8_t* out = static_cast<uint8_t*>(p.out) + row * p.ldo + col0;
+          const bool v8 = ((reinterpret_cast<uintptr_t>(p.out) | static_cast<uintptr_t>(p.ldo)) & 31) == 0;
 #pragma unroll
-          for (int v = 0; v < 8; ++v) {
-            uint32_t w[4];
+          for (int v = 0; v < 4; ++v) {  // 32 codes per 32-byte segment
+            uint32_t w[8];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const float* hv = h + 16 * v + 4 * j;
+            for (int j = 0; j < 8; ++j) {
+              const float* hv = h + 32 * v + 4 * j;
               w[j] = e4m3x4(hv[0] * inv, hv[1] * inv, hv[2] * inv, hv[3] * inv);
             }
-            reinterpret_cast<uint4*>(out)[v] = make_uint4(w[0], w[1], w[2], w[3]);
+            if (v8) {
+              st_global_v8(out + 32 * v, w);
+            } else {
+              reinterpret_cast<uint4*>(out + 32 * v)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+              reinterpret_cast<uint4*>(out + 32 * v)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            }
           }
         }
         // byte (n_tile % 4) of this row's word in atom (row0 / 128, n_tile / 4) of the down GEMM
@@ -396,14 +402,20 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         mbar_arrive(&tempty_bar[acc]);
         if (row_ok) {
           __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + row * p.ldo + col0;
+          const bool v8 = ((reinterpret_cast<uintptr_t>(p.out) | (static_cast<uintptr_t>(p.ldo) * 2)) & 31) == 0;
 #pragma unroll
           for (int c = 0; c < BN; c += 32) {
             if (col0 + c < p.N) {
-              uint4* dst = reinterpret_cast<uint4*>(out + c);
+              if (v8) {
+                st_global_v8(out + c, pk + c / 2);
+                st_global_v8(out + c + 16, pk + c / 2 + 8);
+              } else {
+                uint4* dst = reinterpret_cast<uint4*>(out + c);
 #pragma unroll
-              for (int v = 0; v < 4; ++v)
-                dst[v] = make_uint4(pk[c / 2 + 4 * v], pk[c / 2 + 4 * v + 1], pk[c / 2 + 4 * v + 2],
-                                    pk[c / 2 + 4 * v + 3]);
+                for (int v = 0; v < 4; ++v)
+                  dst[v] = make_uint4(pk[c / 2 + 4 * v], pk[c / 2 + 4 * v + 1], pk[c / 2 + 4 * v + 2],
+                                      pk[c / 2 + 4 * v + 3]);
+              }
             }
           }
         }
