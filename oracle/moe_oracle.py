@@ -42,6 +42,8 @@ Readings where the pages are silent (each also listed in the design notes):
     one power-of-two scale per row and 128 columns for the FP8 workload.
   - FP8 workload: e4m3 (max 448, round to nearest even, saturating); one
     power-of-two scale per 1x128 activation block and per 128x128 weight block.
+  - FP8 x FP4 workload: activations as in the FP8 workload; weights e2m1 (OCP MX
+    FP4) with one UE8M0 (power-of-two) scale per row and 32 consecutive K elements.
   - No residual is added; the layer returns routed + shared only.
 
 Parity status: routed_scale and group_topn = 2 are not fixed by any worked example on
@@ -117,6 +119,36 @@ def quantize_rows_1x128(h) -> np.ndarray:
     b = h.reshape(R, C // QBLOCK, QBLOCK)
     s = pow2_scale(np.abs(b).max(axis=2))
     return (quantize_e4m3(b / s[:, :, None]) * s[:, :, None]).reshape(R, C)
+
+
+# ----------------------------------------------------------------------------------
+# e2m1 (OCP MX FP4) weights with one UE8M0 scale per 32 consecutive K elements: the
+# FP4 operand of the FP8 x FP4 GEMM ("DeepGEMM质变", §5.3; §一 1.3 for the UE8M0
+# scale buffers of the FP4 path)
+# ----------------------------------------------------------------------------------
+FP4_BLOCK = 32
+
+
+def decode_e2m1(codes) -> np.ndarray:
+    """Value of each 4-bit code: sign bit 3, 2 exponent bits (bias 1), 1 mantissa bit;
+    exponent field 0 is subnormal (m/2).  No infinities or NaN."""
+    c = np.asarray(codes, dtype=np.int64) & 0xF
+    sign = np.where(c & 0x8, -1.0, 1.0)
+    e = (c >> 1) & 0x3
+    m = c & 0x1
+    return sign * np.where(e == 0, m / 2.0, (1.0 + m / 2.0) * np.power(2.0, e - 1.0))
+
+
+def dequant_fp4(packed, scale_bytes) -> np.ndarray:
+    """packed [R, C/2] uint8 (element 2j in the low nibble, 2j+1 in the high one) with
+    UE8M0 scale bytes [R, C/32] (value 2^(byte-127)) -> float64 [R, C]."""
+    p = np.asarray(packed, dtype=np.uint8)
+    R = p.shape[0]
+    codes = np.empty((R, p.shape[1] * 2), dtype=np.uint8)
+    codes[:, 0::2] = p & 0xF
+    codes[:, 1::2] = p >> 4
+    s = np.ldexp(1.0, np.asarray(scale_bytes, np.int64) - 127)
+    return decode_e2m1(codes) * np.repeat(s, FP4_BLOCK, axis=1)
 
 
 def round_bf16(v) -> np.ndarray:

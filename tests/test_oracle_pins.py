@@ -437,3 +437,35 @@ def test_aux_free_bias_update_balanced_is_fixed_point():
     # only the sign of the imbalance matters, not its size
     a = o.aux_free_bias_update(np.zeros(3), [1, 2, 100], 0.5)
     np.testing.assert_array_equal(a, [0.5, 0.5, -0.5])
+
+
+# ------------------------------------------------------------------ e2m1 (FP4) weights
+def test_e2m1_decode_matches_ml_dtypes():
+    """All 16 codes against an independent implementation of OCP FP4 (ml_dtypes)."""
+    ml = pytest.importorskip("ml_dtypes")
+    codes = np.arange(16, dtype=np.uint8)
+    ref = codes.view(ml.float4_e2m1fn).astype(np.float64)
+    got = o.decode_e2m1(codes)
+    assert np.array_equal(got, ref) and np.array_equal(np.signbit(got), np.signbit(ref))
+
+
+def test_e2m1_spec_constants():
+    """OCP MX v1.0 FP4 E2M1: largest normal 6.0, smallest normal 1.0, only subnormal
+    0.5; positive codes increase with the code; the sign bit negates."""
+    v = o.decode_e2m1(np.arange(16))
+    assert v[7] == 6.0 and v[2] == 1.0 and v[1] == 0.5 and v[0] == 0.0
+    assert (np.diff(v[:8]) > 0).all()
+    assert np.array_equal(v[8:], -v[:8])
+
+
+def test_dequant_fp4_nibble_order_and_block_scales():
+    """Element 2j sits in the low nibble; each 32-element block has its own 2^(s-127)."""
+    packed = np.zeros((1, 32), dtype=np.uint8)      # 64 elements, two scale blocks
+    packed[0, 0] = 0x71                             # element 0 = code 1 (0.5), element 1 = code 7 (6)
+    packed[0, 16] = 0x2A                            # element 32 = code 0xA (-1), element 33 = code 2 (1)
+    scales = np.array([[127 + 3, 127 - 1]], dtype=np.uint8)
+    w = o.dequant_fp4(packed, scales)
+    assert w.shape == (1, 64)
+    assert w[0, 0] == 0.5 * 8 and w[0, 1] == 6.0 * 8
+    assert w[0, 32] == -0.5 and w[0, 33] == 0.5
+    assert (w[0, 2:32] == 0).all() and (w[0, 34:] == 0).all()
