@@ -34,6 +34,14 @@
  *     x_scale [T,H/128] (one per token and 128 channels); expert weights are e4m3 with
  *     fp32 scales per 128x128 block ([E,I/128,H/128] for gate/up, [E,H/128,I/128] for
  *     down); W_r stays bf16; the output is bf16.
+ *     dtype MOE_DTYPE_FP8_FP4 (the FP8 x FP4 GEMM of "DeepGEMM质变…" §5.3, the Mega MoE
+ *     compute unit): x as for FP8; expert weights are e2m1 (OCP MX FP4), two per byte
+ *     (element 2j in the low nibble: W_gate, W_up [E,I,H/2] bytes, W_down [E,H,I/2]),
+ *     base pointers 32-byte aligned, with one UE8M0 scale (2^(byte-127)) per row and 32
+ *     consecutive K elements, passed as the atoms moe_prepare_fp4_scales() makes.  No
+ *     shared expert, block_m 128.
+ *   - Weight scale arguments (void*): fp32 block scales for MOE_DTYPE_FP8_E4M3, prepared
+ *     atoms for MOE_DTYPE_FP8_FP4, ignored (may be NULL) for MOE_DTYPE_BF16.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
@@ -45,7 +53,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 3
+#define MOE_ABI_VERSION 4
 
 typedef enum moe_status {
   MOE_OK = 0,
@@ -63,7 +71,7 @@ typedef enum moe_status {
                                     /* pairs; the pairs past it got no row (left out)       */
 
 enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 };
-enum { MOE_DTYPE_BF16 = 0, MOE_DTYPE_FP8_E4M3 = 1 };
+enum { MOE_DTYPE_BF16 = 0, MOE_DTYPE_FP8_E4M3 = 1, MOE_DTYPE_FP8_FP4 = 2 };
 
 typedef struct moe_params {
   int32_t T;            /* tokens                                                        */
@@ -78,7 +86,7 @@ typedef struct moe_params {
   int32_t renormalize;  /* 1: divide the chosen weights by their sum                     */
   float routed_scale;   /* factor applied to the (renormalised) weights                  */
   int32_t I_shared;     /* intermediate size of the shared expert, 0 = none              */
-  int32_t dtype;        /* MOE_DTYPE_BF16 or MOE_DTYPE_FP8_E4M3                          */
+  int32_t dtype;        /* MOE_DTYPE_BF16, MOE_DTYPE_FP8_E4M3 or MOE_DTYPE_FP8_FP4       */
   int32_t block_m;      /* row alignment of each expert's bucket: 128 (one-SM GEMM tiles), */
                         /* 256 (two-SM cta_group::2 tiles: a third less SM-side operand  */
                         /* traffic, more pad rows), 0 = default (128)                    */
@@ -202,8 +210,8 @@ moe_status_t moe_permute_noalloc(const moe_params_t* p, const int32_t* topk_ids,
 moe_status_t moe_expert_ffn(const moe_params_t* p, const void* x_perm, const float* x_perm_scale,
                             const int32_t* offsets_padded, const int32_t* counts,
                             const void* w_gate, const void* w_up, const void* w_down,
-                            const float* w_gate_scale, const float* w_up_scale,
-                            const float* w_down_scale, void* y_perm, void* ws, size_t ws_bytes,
+                            const void* w_gate_scale, const void* w_up_scale,
+                            const void* w_down_scale, void* y_perm, void* ws, size_t ws_bytes,
                             void* stream);
 
 /* Dense SwiGLU FFN of the always-active shared expert on all T tokens ("MoE" §0, §2.1):
@@ -231,8 +239,8 @@ moe_status_t moe_combine(const moe_params_t* p, const void* y_perm, const int32_
 /* ---------------------------------------------------------------------------------- */
 moe_status_t moe_layer_forward(const moe_params_t* p, const void* x, const float* x_scale,
                                const void* w_r, const float* bias, const void* w_gate,
-                               const void* w_up, const void* w_down, const float* w_gate_scale,
-                               const float* w_up_scale, const float* w_down_scale,
+                               const void* w_up, const void* w_down, const void* w_gate_scale,
+                               const void* w_up_scale, const void* w_down_scale,
                                const void* ws_gate, const void* ws_up, const void* ws_down,
                                void* out, int32_t* topk_ids_out, float* topk_w_out,
                                int32_t* counts_out, void* ws, size_t ws_bytes, void* stream);
@@ -245,11 +253,26 @@ moe_status_t moe_layer_forward(const moe_params_t* p, const void* x, const float
 moe_status_t moe_layer_forward_host(const moe_params_t* p, const void* x_host,
                                     const float* x_scale_host, const void* w_r,
                                     const float* bias, const void* w_gate, const void* w_up,
-                                    const void* w_down, const float* w_gate_scale,
-                                    const float* w_up_scale, const float* w_down_scale,
+                                    const void* w_down, const void* w_gate_scale,
+                                    const void* w_up_scale, const void* w_down_scale,
                                     const void* ws_gate, const void* ws_up,
                                     const void* ws_down, void* out_host, void* ws,
                                     size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------- */
+/* e2m1 weight scales ("DeepGEMM质变…" §5.3 FP8 x FP4 GEMM; §一 1.3 lays the UE8M0 scale */
+/* buffers out at the 128-element granularity of the tensor core's scale copy).         */
+/* Converts one weight tensor's scales, once, when the weights are loaded:              */
+/*   scale_words [rows, K/128] 32-bit words, byte j of word (r, kb) = UE8M0 scale of    */
+/*               K elements 128 kb + 32 j ... + 31 of row r (4-byte aligned).  A row-   */
+/*               major [rows, K/32] byte array of the scales is exactly this.           */
+/*   atoms       out, rows * K / 32 bytes, 16-byte aligned: the 512-byte per (128 rows, */
+/*               128 K) blocks that moe_expert_ffn / moe_layer_forward read.            */
+/* rows (all experts of the tensor stacked: E*I for gate/up, E*H for down) and K must   */
+/* be multiples of 128.  Asynchronous on `stream`; no workspace.                        */
+/* ---------------------------------------------------------------------------------- */
+moe_status_t moe_prepare_fp4_scales(const void* scale_words, int64_t rows, int32_t K, void* atoms,
+                                    void* stream);
 
 /* ---------------------------------------------------------------------------------- */
 /* Status, tracing                                                                      */

@@ -76,6 +76,7 @@ _SIGS = {
     "moe_clear_device_status": (ctypes.c_int, [_P, _P]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_abi_version": (ctypes.c_int32, []),
+    "moe_prepare_fp4_scales": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.c_int32, _P, _P]),
     "moe_trace_enable": (ctypes.c_int, [ctypes.c_uint32, ctypes.c_int32]),
     "moe_trace_disable": (ctypes.c_int, []),
     "moe_trace_collect": (ctypes.c_int32, [ctypes.POINTER(ctypes.c_int32),
@@ -237,6 +238,12 @@ def moe_status_string(s: int) -> str:
 
 def moe_abi_version() -> int:
     return lib(require_gpu=False).moe_abi_version()
+
+
+def moe_prepare_fp4_scales(scale_bytes, rows: int, K: int, atoms, stream=None) -> int:
+    """scale_bytes: UE8M0 bytes [rows, K/32] (read as [rows, K/128] 32-bit words);
+    atoms: rows*K/32 bytes, written."""
+    return lib().moe_prepare_fp4_scales(_ptr(scale_bytes), rows, K, _ptr(atoms), _stream(stream))
 
 
 def moe_trace_enable(kernel_mask: int, capacity: int) -> int:

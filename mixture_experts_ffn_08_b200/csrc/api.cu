@@ -69,7 +69,10 @@ struct Layout {
   long long max_rows;
 };
 
-bool is_fp8(const moe_params_t* p) { return p->dtype == MOE_DTYPE_FP8_E4M3; }
+// e4m3 activations (with e4m3 or e2m1 expert weights)
+bool is_fp8(const moe_params_t* p) { return p->dtype == MOE_DTYPE_FP8_E4M3 || p->dtype == MOE_DTYPE_FP8_FP4; }
+// e2m1 expert weights whose scale atoms the caller prepared (moe_prepare_fp4_scales)
+bool is_fp4(const moe_params_t* p) { return p->dtype == MOE_DTYPE_FP8_FP4; }
 
 // Bucket alignment: 128 rows (one-SM GEMM tiles) unless the caller asks for 256 (two-SM
 // cta_group::2 tiles).  Measured on B200, the pair tiles' third less SM-side traffic did
@@ -107,13 +110,14 @@ Layout layout(const moe_params_t* p) {
   L.h_sh = take(T * static_cast<long long>(p->I_shared) * 2);
   L.y_sh = take(p->I_shared > 0 || p->fused_combine ? T * H * 4 : 0);  // also the fused-combine accumulator
   const bool f8 = is_fp8(p);
+  const bool w8 = p->dtype == MOE_DTYPE_FP8_E4M3;  // e4m3 weights: atoms built per call
   // e4m3 scale atoms: 512 bytes per 128 rows and 4 K blocks of 128
   const long long hk4 = (H / 128 + 3) / 4, ik4 = (I / 128 + 3) / 4;
   L.x_atoms = take(f8 ? rows_t / 128 * hk4 * 512 : 0);
   L.h_atoms = take(f8 ? rows_t / 128 * ik4 * 512 : 0);
-  L.wg_atoms = take(f8 ? E * (I / 128) * hk4 * 512 : 0);
-  L.wu_atoms = take(f8 ? E * (I / 128) * hk4 * 512 : 0);
-  L.wd_atoms = take(f8 ? E * (H / 128) * ik4 * 512 : 0);
+  L.wg_atoms = take(w8 ? E * (I / 128) * hk4 * 512 : 0);
+  L.wu_atoms = take(w8 ? E * (I / 128) * hk4 * 512 : 0);
+  L.wd_atoms = take(w8 ? E * (H / 128) * ik4 * 512 : 0);
   L.total = o;
   L.x_stage = take(T * H * xelem);
   L.x_scale_stage = take(is_fp8(p) ? T * (H / 128) * 4 : 0);
@@ -132,7 +136,8 @@ moe_status_t validate(const moe_params_t* p) {
   if (p->T < 0 || p->H <= 0 || p->I <= 0 || p->E <= 0 || p->K <= 0) return MOE_ERR_INVALID_ARG;
   if (p->E > kMaxExperts || p->K > kMaxTopK || p->K > p->E) return MOE_ERR_INVALID_ARG;
   if (p->score_fn != MOE_SCORE_SOFTMAX && p->score_fn != MOE_SCORE_SIGMOID) return MOE_ERR_INVALID_ARG;
-  if (p->dtype != MOE_DTYPE_BF16 && p->dtype != MOE_DTYPE_FP8_E4M3) return MOE_ERR_INVALID_ARG;
+  if (p->dtype != MOE_DTYPE_BF16 && p->dtype != MOE_DTYPE_FP8_E4M3 && p->dtype != MOE_DTYPE_FP8_FP4)
+    return MOE_ERR_INVALID_ARG;
   if (p->n_group < 1 || p->n_group > 32 || p->E % p->n_group != 0) return MOE_ERR_INVALID_ARG;
   if (p->n_group > 1) {
     const int gs = p->E / p->n_group;
@@ -143,7 +148,8 @@ moe_status_t validate(const moe_params_t* p) {
   if (p->I_shared < 0) return MOE_ERR_INVALID_ARG;
   if (p->H % 128 != 0 || p->I % 128 != 0 || p->I_shared % 128 != 0) return MOE_ERR_UNSUPPORTED;
   if (p->block_m != 0 && p->block_m != kBlockM && p->block_m != kBlockM2) return MOE_ERR_UNSUPPORTED;
-  if (p->dtype == MOE_DTYPE_FP8_E4M3 && p->I_shared > 0) return MOE_ERR_UNSUPPORTED;
+  if (is_fp8(p) && p->I_shared > 0) return MOE_ERR_UNSUPPORTED;
+  if (is_fp4(p) && p->block_m == kBlockM2) return MOE_ERR_UNSUPPORTED;
   if (p->fused_combine != 0 && p->fused_combine != 1) return MOE_ERR_INVALID_ARG;
   if (p->fused_combine && (p->dtype != MOE_DTYPE_BF16 || p->block_m == kBlockM2)) return MOE_ERR_UNSUPPORTED;
   const long long rows = static_cast<long long>(p->T) * p->K + static_cast<long long>(p->E) * (kBlockM2 - 1);
@@ -157,6 +163,15 @@ moe_status_t validate(const moe_params_t* p) {
 }
 
 bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+bool aligned32(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 31u) == 0; }
+
+// Weight scales as the FFN reads them: fp32 block scales (e4m3 weights) or prepared
+// 512-byte atoms (e2m1 weights, read with 16-byte bulk copies).
+bool weight_scales_ok(const moe_params_t* p, const void* g, const void* u, const void* d) {
+  if (!is_fp8(p)) return true;
+  if (!g || !u || !d) return false;
+  return !is_fp4(p) || (aligned16(g) && aligned16(u) && aligned16(d));
+}
 
 moe_status_t check_ws(const moe_params_t* p, const void* ws, size_t ws_bytes, bool host) {
   if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return MOE_ERR_INVALID_ARG;
@@ -201,8 +216,8 @@ moe_status_t do_permute(const moe_params_t* p, const int32_t* ids, const void* x
 
 moe_status_t do_expert_ffn_fp8(const moe_params_t* p, const void* x_perm, const float* x_perm_scale,
                                const int32_t* offsets, const int32_t* counts, const void* w_gate,
-                               const void* w_up, const void* w_down, const float* wgs,
-                               const float* wus, const float* wds, void* y_perm, void* ws,
+                               const void* w_up, const void* w_down, const void* wgs,
+                               const void* wus, const void* wds, void* y_perm, void* ws,
                                cudaStream_t st) {
   const Layout L = layout(p);
   int32_t* status = at<int32_t>(ws, L.status);
@@ -213,27 +228,41 @@ moe_status_t do_expert_ffn_fp8(const moe_params_t* p, const void* x_perm, const 
     MOE_CUDA(launch_masked_schedule(counts, p->E, at<int32_t>(ws, L.sched), st));
     sched = at<int32_t>(ws, L.sched);
   }
-  const long long rows_gu = static_cast<long long>(p->E) * (p->I / 128);   // 128-row weight blocks
-  const long long rows_d = static_cast<long long>(p->E) * (p->H / 128);
-  MOE_CUDA(launch_sf_blocks_to_atoms(wgs, rows_gu, p->H / 128, at<uint8_t>(ws, L.wg_atoms), st));
-  MOE_CUDA(launch_sf_blocks_to_atoms(wus, rows_gu, p->H / 128, at<uint8_t>(ws, L.wu_atoms), st));
-  MOE_CUDA(launch_sf_blocks_to_atoms(wds, rows_d, p->I / 128, at<uint8_t>(ws, L.wd_atoms), st));
+  // weight scale atoms: e2m1 weights bring theirs (prepared once); e4m3 weights' fp32
+  // block scales are turned into atoms here
+  const bool w4 = is_fp4(p);
+  const uint8_t* wg_atoms = static_cast<const uint8_t*>(wgs);
+  const uint8_t* wu_atoms = static_cast<const uint8_t*>(wus);
+  const uint8_t* wd_atoms = static_cast<const uint8_t*>(wds);
+  if (!w4) {
+    const long long rows_gu = static_cast<long long>(p->E) * (p->I / 128);   // 128-row weight blocks
+    const long long rows_d = static_cast<long long>(p->E) * (p->H / 128);
+    MOE_CUDA(launch_sf_blocks_to_atoms(static_cast<const float*>(wgs), rows_gu, p->H / 128,
+                                       at<uint8_t>(ws, L.wg_atoms), st));
+    MOE_CUDA(launch_sf_blocks_to_atoms(static_cast<const float*>(wus), rows_gu, p->H / 128,
+                                       at<uint8_t>(ws, L.wu_atoms), st));
+    MOE_CUDA(launch_sf_blocks_to_atoms(static_cast<const float*>(wds), rows_d, p->I / 128,
+                                       at<uint8_t>(ws, L.wd_atoms), st));
+    wg_atoms = at<uint8_t>(ws, L.wg_atoms);
+    wu_atoms = at<uint8_t>(ws, L.wu_atoms);
+    wd_atoms = at<uint8_t>(ws, L.wd_atoms);
+  }
   MOE_CUDA(launch_sf_rows_to_atoms(x_perm_scale, p->H / 128, offsets, p->E, L.max_rows,
                                    at<uint8_t>(ws, L.x_atoms), st));
   void* h = at<void>(ws, L.h);
   if (block_m_of(p) == kBlockM2) {
     MOE_CUDA(gemm_pair_gateup_swiglu_fp8(x_perm, at<uint8_t>(ws, L.x_atoms), L.max_rows, offsets, counts, p->E,
-                                         w_gate, w_up, at<uint8_t>(ws, L.wg_atoms), at<uint8_t>(ws, L.wu_atoms),
+                                         w_gate, w_up, wg_atoms, wu_atoms,
                                          p->I, p->H, h, at<uint8_t>(ws, L.h_atoms), status, st));
     MOE_CUDA(gemm_pair_down_fp8(h, at<uint8_t>(ws, L.h_atoms), L.max_rows, offsets, counts, p->E, w_down,
-                                at<uint8_t>(ws, L.wd_atoms), p->H, p->I, y_perm, status, st));
+                                wd_atoms, p->H, p->I, y_perm, status, st));
     return MOE_OK;
   }
   MOE_CUDA(gemm_gateup_swiglu_fp8(x_perm, at<uint8_t>(ws, L.x_atoms), L.max_rows, sched, counts, p->E,
-                                  w_gate, w_up, at<uint8_t>(ws, L.wg_atoms), at<uint8_t>(ws, L.wu_atoms),
-                                  p->I, p->H, h, at<uint8_t>(ws, L.h_atoms), status, st, cap));
-  MOE_CUDA(gemm_down_fp8(h, at<uint8_t>(ws, L.h_atoms), L.max_rows, sched, counts, p->E, w_down,
-                         at<uint8_t>(ws, L.wd_atoms), p->H, p->I, y_perm, status, st, cap));
+                                  w_gate, w_up, wg_atoms, wu_atoms, p->I, p->H, h, at<uint8_t>(ws, L.h_atoms),
+                                  status, st, cap, w4));
+  MOE_CUDA(gemm_down_fp8(h, at<uint8_t>(ws, L.h_atoms), L.max_rows, sched, counts, p->E, w_down, wd_atoms,
+                         p->H, p->I, y_perm, status, st, cap, w4));
   return MOE_OK;
 }
 
@@ -276,7 +305,7 @@ moe_status_t do_shared(const moe_params_t* p, const void* x, const void* wsg, co
 
 moe_status_t do_layer(const moe_params_t* p, const void* x, const float* x_scale, const void* w_r,
                       const float* bias, const void* w_gate, const void* w_up, const void* w_down,
-                      const float* wgs, const float* wus, const float* wds, const void* wsg,
+                      const void* wgs, const void* wus, const void* wds, const void* wsg,
                       const void* wsu, const void* wsd, void* out, int32_t* ids_out, float* w_out,
                       int32_t* counts_out, void* ws, cudaStream_t st) {
   const Layout L = layout(p);
@@ -331,6 +360,7 @@ moe_status_t check_layer_args(const moe_params_t* p, const void* x, const float*
       !aligned16(out))
     return MOE_ERR_INVALID_ARG;
   if (is_fp8(p) && !x_scale) return MOE_ERR_INVALID_ARG;
+  if (is_fp4(p) && !(aligned32(w_gate) && aligned32(w_up) && aligned32(w_down))) return MOE_ERR_INVALID_ARG;
   if (p->I_shared > 0) {
     if (!wsg || !wsu || !wsd) return MOE_ERR_INVALID_ARG;
     if (!aligned16(wsg) || !aligned16(wsu) || !aligned16(wsd)) return MOE_ERR_INVALID_ARG;
@@ -405,8 +435,8 @@ moe_status_t moe_permute(const moe_params_t* p, const int32_t* topk_ids, const v
 
 moe_status_t moe_expert_ffn(const moe_params_t* p, const void* x_perm, const float* x_perm_scale,
                             const int32_t* offsets_padded, const int32_t* counts, const void* w_gate,
-                            const void* w_up, const void* w_down, const float* w_gate_scale,
-                            const float* w_up_scale, const float* w_down_scale, void* y_perm,
+                            const void* w_up, const void* w_down, const void* w_gate_scale,
+                            const void* w_up_scale, const void* w_down_scale, void* y_perm,
                             void* ws, size_t ws_bytes, void* stream) {
   MOE_TRY(validate(p));
   MOE_TRY(check_ws(p, ws, ws_bytes, false));
@@ -414,8 +444,9 @@ moe_status_t moe_expert_ffn(const moe_params_t* p, const void* x_perm, const flo
   if (p->masked_cap > 0 ? !counts : !offsets_padded) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x_perm) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down) || !aligned16(y_perm))
     return MOE_ERR_INVALID_ARG;
-  if (is_fp8(p) && (!x_perm_scale || !w_gate_scale || !w_up_scale || !w_down_scale))
-    return MOE_ERR_INVALID_ARG;
+  if (is_fp8(p) && !x_perm_scale) return MOE_ERR_INVALID_ARG;
+  if (!weight_scales_ok(p, w_gate_scale, w_up_scale, w_down_scale)) return MOE_ERR_INVALID_ARG;
+  if (is_fp4(p) && !(aligned32(w_gate) && aligned32(w_up) && aligned32(w_down))) return MOE_ERR_INVALID_ARG;
   if (p->T == 0) return MOE_OK;
   if (offsets_padded == nullptr) {  // masked layout: expert e's rows start at e*cap
     const Layout L = layout(p);
@@ -455,14 +486,14 @@ moe_status_t moe_combine(const moe_params_t* p, const void* y_perm, const int32_
 
 moe_status_t moe_layer_forward(const moe_params_t* p, const void* x, const float* x_scale, const void* w_r,
                                const float* bias, const void* w_gate, const void* w_up, const void* w_down,
-                               const float* w_gate_scale, const float* w_up_scale, const float* w_down_scale,
+                               const void* w_gate_scale, const void* w_up_scale, const void* w_down_scale,
                                const void* ws_gate, const void* ws_up, const void* ws_down, void* out,
                                int32_t* topk_ids_out, float* topk_w_out, int32_t* counts_out, void* ws,
                                size_t ws_bytes, void* stream) {
   MOE_TRY(validate(p));
   MOE_TRY(check_ws(p, ws, ws_bytes, false));
   MOE_TRY(check_layer_args(p, x, x_scale, w_r, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, out));
-  if (is_fp8(p) && (!w_gate_scale || !w_up_scale || !w_down_scale)) return MOE_ERR_INVALID_ARG;
+  if (!weight_scales_ok(p, w_gate_scale, w_up_scale, w_down_scale)) return MOE_ERR_INVALID_ARG;
   return do_layer(p, x, x_scale, w_r, bias, w_gate, w_up, w_down, w_gate_scale, w_up_scale, w_down_scale,
                   ws_gate, ws_up, ws_down, out, topk_ids_out,
                   topk_w_out, counts_out, ws, static_cast<cudaStream_t>(stream));
@@ -470,14 +501,15 @@ moe_status_t moe_layer_forward(const moe_params_t* p, const void* x, const float
 
 moe_status_t moe_layer_forward_host(const moe_params_t* p, const void* x_host, const float* x_scale_host,
                                     const void* w_r, const float* bias, const void* w_gate, const void* w_up,
-                                    const void* w_down, const float* w_gate_scale, const float* w_up_scale,
-                                    const float* w_down_scale, const void* ws_gate, const void* ws_up,
+                                    const void* w_down, const void* w_gate_scale, const void* w_up_scale,
+                                    const void* w_down_scale, const void* ws_gate, const void* ws_up,
                                     const void* ws_down, void* out_host, void* ws, size_t ws_bytes,
                                     void* stream) {
   MOE_TRY(validate(p));
   MOE_TRY(check_ws(p, ws, ws_bytes, true));
   if (!x_host || !out_host) return MOE_ERR_INVALID_ARG;
-  if (is_fp8(p) && (!x_scale_host || !w_gate_scale || !w_up_scale || !w_down_scale)) return MOE_ERR_INVALID_ARG;
+  if (is_fp8(p) && !x_scale_host) return MOE_ERR_INVALID_ARG;
+  if (!weight_scales_ok(p, w_gate_scale, w_up_scale, w_down_scale)) return MOE_ERR_INVALID_ARG;
   const Layout L = layout(p);
   void* x_dev = at<void>(ws, L.x_stage);
   float* xs_dev = is_fp8(p) ? at<float>(ws, L.x_scale_stage) : nullptr;
@@ -522,6 +554,14 @@ const char* moe_status_string(moe_status_t s) {
 
 int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
 
+moe_status_t moe_prepare_fp4_scales(const void* scale_words, int64_t rows, int32_t K, void* atoms, void* stream) {
+  if (!scale_words || !atoms || rows <= 0 || rows % 128 != 0 || K <= 0 || K % 128 != 0) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(scale_words) & 3u) != 0 || !aligned16(atoms)) return MOE_ERR_INVALID_ARG;
+  if (rows > (1LL << 40) / K) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_fp4_scale_atoms(static_cast<const uint32_t*>(scale_words), rows, K,
+                                            static_cast<uint8_t*>(atoms), static_cast<cudaStream_t>(stream)));
+}
+
 moe_status_t moe_trace_enable(uint32_t kernel_mask, int32_t capacity) {
   if (capacity <= 0 || capacity > (1 << 20)) return MOE_ERR_INVALID_ARG;
   Trace& t = g_trace;
@@ -563,7 +603,8 @@ int32_t moe_layer_launch_count(const moe_params_t* p) {
   if (validate(p) != MOE_OK) return -1;
   if (p->T == 0) return 0;
   int n = 2;                                 // router GEMM, top-k
-  if (is_fp8(p)) n += 5;                     // dequantise x for the router, 4 scale-atom passes
+  if (is_fp8(p)) n += is_fp4(p) ? 2 : 5;     // dequantise x for the router; scale atoms of x
+                                             // (and of the three e4m3 weights)
   n += (p->T * p->K > 0) ? 4 : 2;            // count, scan, rank, gather
   n += 2;                                    // gate/up, down
   if (p->I_shared > 0) n += 2;               // shared gate/up, down

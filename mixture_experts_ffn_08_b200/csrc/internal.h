@@ -20,6 +20,11 @@ void trace_before(int kid, cudaStream_t st);
 void trace_after(int kid, cudaStream_t st);
 int num_sms();
 
+// Activations (x, h) are e4m3 with 1x128 scales: the FP8 and the FP8 x FP4 layers.
+inline bool act_e4m3(const moe_params_t& p) {
+  return p.dtype == MOE_DTYPE_FP8_E4M3 || p.dtype == MOE_DTYPE_FP8_FP4;
+}
+
 // ---------------------------------------------------------------- routing (kernels.cu)
 cudaError_t launch_dequant_x(const uint8_t* xq, const float* xs, int T, int H, void* x_bf16,
                              cudaStream_t st);
@@ -83,12 +88,16 @@ cudaError_t gemm_gateup_swiglu_fp8(const void* A, const uint8_t* a_atoms, int64_
                                    const int32_t* offsets, const int32_t* counts, int G,
                                    const void* w_gate, const void* w_up, const uint8_t* gate_atoms,
                                    const uint8_t* up_atoms, int N, int K, void* h, uint8_t* h_atoms,
-                                   int32_t* status, cudaStream_t st, int masked_cap = 0);
+                                   int32_t* status, cudaStream_t st, int masked_cap = 0, bool w4 = false);
 // y [rows, N] bf16 = A W^T, block-scaled e4m3 GEMM.
 cudaError_t gemm_down_fp8(const void* A, const uint8_t* a_atoms, int64_t a_rows,
                           const int32_t* offsets, const int32_t* counts, int G, const void* w,
                           const uint8_t* w_atoms, int N, int K, void* y, int32_t* status,
-                          cudaStream_t st, int masked_cap = 0);
+                          cudaStream_t st, int masked_cap = 0, bool w4 = false);
+// w4: weights are packed e2m1 (cols/2 bytes per row, 32-byte aligned base) and the weight
+// atoms come from launch_fp4_scale_atoms.
+// e2m1 weight scale words [rows, K/128] (4 UE8M0 bytes each) -> atoms [rows/128][K/128][512].
+cudaError_t launch_fp4_scale_atoms(const uint32_t* words, long long rows, int K, uint8_t* atoms, cudaStream_t st);
 
 // ---------------------------------------------------------------- two-SM GEMMs (gemm_2cta.cu)
 cudaError_t gemm_pair_gateup_swiglu(const void* A, int64_t a_rows, const int32_t* offsets, const int32_t* counts,

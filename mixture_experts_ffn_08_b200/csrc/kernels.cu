@@ -498,7 +498,7 @@ cudaError_t launch_permute(const moe_params_t& p, int block_m, const int32_t* id
   const long long blocks = (max_rows + kGatherWarps - 1) / kGatherWarps;
   const int grid = static_cast<int>(blocks < num_sms() * 8LL ? (blocks > 0 ? blocks : 1) : num_sms() * 8LL);
   trace_before(MOE_K_PERM_GATHER, st);
-  if (p.dtype == MOE_DTYPE_FP8_E4M3)
+  if (act_e4m3(p))
     perm_gather_kernel<true><<<grid, 32 * kGatherWarps, 0, st>>>(x, x_scale, p.H, p.K, p.E, counts, offsets,
                                                    pair_of_row, x_perm, x_perm_scale, !masked);
   else
@@ -633,7 +633,7 @@ cudaError_t launch_combine(const moe_params_t& p, const void* y_perm, const int3
   if (p.T == 0) return cudaSuccess;
   const int grid = p.T < num_sms() * 16 ? p.T : num_sms() * 16;
   trace_before(MOE_K_COMBINE, st);
-  if (p.dtype == MOE_DTYPE_FP8_E4M3)
+  if (act_e4m3(p))
     combine_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(y_perm), row_of_pair,
                                                         w, y_shared, static_cast<__nv_bfloat16*>(out), p.T,
                                                         p.H, p.K);

@@ -77,12 +77,14 @@ MOE_DEVINL void umma_mxf8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint3
       : "memory");
 }
 
-// Instruction descriptor, kind::mxf8f6f4 block-scaled: e4m3 A and B (both K-major),
-// UE8M0 scale factors, fp32 accumulator; sf ids select the byte of each scale word.
+// Instruction descriptor, kind::mxf8f6f4 block-scaled: e4m3 A, e4m3 (b_fmt 0) or e2m1
+// (b_fmt 5) B, both K-major, UE8M0 scale factors, fp32 accumulator; sf ids select the
+// byte of each scale word.
+constexpr uint32_t kFmtE4M3 = 0, kFmtE2M1 = 5;
 __host__ __device__ constexpr uint32_t idesc_mxf8_e4m3(int M, int N, uint32_t a_sf_id,
-                                                       uint32_t b_sf_id) {
+                                                       uint32_t b_sf_id, uint32_t b_fmt = kFmtE4M3) {
   return (b_sf_id << 4)                             // B scale-factor byte
-         | (0u << 7) | (0u << 10)                   // A, B format: e4m3
+         | (kFmtE4M3 << 7) | (b_fmt << 10)          // A format e4m3, B format
          | (static_cast<uint32_t>(N >> 3) << 17)    // N / 8
          | (1u << 23)                               // scale format: UE8M0
          | (static_cast<uint32_t>(M >> 4) << 24)    // M / 16
@@ -102,7 +104,8 @@ struct Fp8Params {
   int K;                   // reduction length, multiple of 128
   int N;                   // output columns of one group
   const uint8_t* sfa;      // A scale atoms [m_tiles][ceil(K/512)][512]
-  const uint8_t* sfb0;     // B scale atoms [G][N/128][ceil(K/512)][512] (gate, or down weight)
+  const uint8_t* sfb0;     // B scale atoms (gate, or down weight): e4m3 [G][N/128][ceil(K/512)][512],
+                           // e2m1 [G][N/128][K/128][512]
   const uint8_t* sfb1;     // up-projection scale atoms (SwiGLU only)
   void* out;               // SwiGLU: e4m3 codes [rows, ldo]; BF16: bf16 [rows, ldo]
   int64_t ldo;             // elements
@@ -112,15 +115,20 @@ struct Fp8Params {
                            // at g * masked_cap), as in GemmParams
 };
 
-template <int BN_, int EPI_, int STAGES_>
+// W4_: B is e2m1 (FP4) with one UE8M0 scale per 32 K: TMA unpacks 16 packed values into
+// each 16-byte smem slot (8 data bytes, 8 gap bytes), so a 128-K B row fills 128 smem
+// bytes exactly like e4m3; B's scale atoms then change every K step (4 scales per row).
+template <int BN_, int EPI_, int STAGES_, bool W4_ = false>
 struct Fp8Cfg {
+  static constexpr bool W4 = W4_;
   static constexpr int BM = 128;
   static constexpr int BN = BN_;          // rows of B per tile (SwiGLU: 128 gate + 128 up)
   static constexpr int BK = 128;          // e4m3 elements (= bytes) per stage and row
   static constexpr int EPI = EPI_;
   static constexpr int STAGES = STAGES_;
   static constexpr int A_BYTES = BM * BK;
-  static constexpr int B_BYTES = BN * BK;
+  static constexpr int B_BYTES = BN * BK;                 // smem bytes of the B tile
+  static constexpr int B_TX_BYTES = W4 ? B_BYTES / 2 : B_BYTES;  // bytes the TMA counts: packed e2m1
   static constexpr int SFB_ATOMS = BN / 128;
   static constexpr int SF_BYTES = 512 * (1 + SFB_ATOMS);
   static constexpr int STAGE_BYTES = (A_BYTES + B_BYTES + SF_BYTES + 1023) / 1024 * 1024;
@@ -231,8 +239,10 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           uint8_t* sa = smem + s * Cfg::STAGE_BYTES;
           uint8_t* sb = sa + Cfg::A_BYTES;
           uint8_t* ssf = sb + Cfg::B_BYTES;
-          const bool new_sf = (kb & 3) == 0;
-          mbar_arrive_expect_tx(&full_bar[s], Cfg::A_BYTES + Cfg::B_BYTES + (new_sf ? Cfg::SF_BYTES : 0));
+          const bool new_sf = (kb & 3) == 0;            // A atoms: one per four K steps
+          const bool new_sfb = Cfg::W4 || new_sf;        // B atoms: every step for e2m1
+          mbar_arrive_expect_tx(&full_bar[s], Cfg::A_BYTES + Cfg::B_TX_BYTES + (new_sf ? 512 : 0) +
+                                                  (new_sfb ? 512 * Cfg::SFB_ATOMS : 0));
           tma_load_2d(sa, &tmA, kb * BK, a_row, &full_bar[s]);
           if (Cfg::EPI == EPI8_SWIGLU_Q) {
             tma_load_2d(sb, &tmB0, kb * BK, b_row, &full_bar[s]);
@@ -240,17 +250,19 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           } else {
             tma_load_2d(sb, &tmB0, kb * BK, b_row, &full_bar[s]);
           }
-          if (new_sf) {
-            const int kb4 = kb >> 2;
-            bulk_load(ssf, p.sfa + (static_cast<size_t>(t.row0 / BM) * KB4 + kb4) * 512, 512, &full_bar[s]);
-            const size_t wsf = (static_cast<size_t>(wblk) * KB4 + kb4) * 512;
+          if (new_sf)
+            bulk_load(ssf, p.sfa + (static_cast<size_t>(t.row0 / BM) * KB4 + (kb >> 2)) * 512, 512, &full_bar[s]);
+          if (new_sfb) {
+            // weight atoms [128-row block][K step (e2m1) or four K steps (e4m3)][512 B]
+            const int steps = Cfg::W4 ? KB : KB4;
+            const size_t wsf = (static_cast<size_t>(wblk) * steps + (Cfg::W4 ? kb : kb >> 2)) * 512;
             if (Cfg::EPI == EPI8_SWIGLU_Q) {
               bulk_load(ssf + 512, p.sfb0 + wsf, 512, &full_bar[s]);
               bulk_load(ssf + 1024, p.sfb1 + wsf, 512, &full_bar[s]);
             } else {
 #pragma unroll
               for (int a = 0; a < Cfg::SFB_ATOMS; ++a)
-                bulk_load(ssf + 512 * (1 + a), p.sfb0 + wsf + static_cast<size_t>(a) * KB4 * 512, 512,
+                bulk_load(ssf + 512 * (1 + a), p.sfb0 + wsf + static_cast<size_t>(a) * steps * 512, 512,
                           &full_bar[s]);
             }
           }
@@ -284,15 +296,20 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           const uint32_t a0 = smem_u32(smem + s * Cfg::STAGE_BYTES);
           const uint32_t b0 = a0 + Cfg::A_BYTES;
           const uint32_t sf0 = b0 + Cfg::B_BYTES;
-          if ((kb & 3) == 0) {  // new scale atoms (four K steps each) into TMEM
-            tmem_cp_32x128b_warpx4(sfa_t, smem_desc_rows16(sf0));
+          // new scale atoms into TMEM (tcgen05.cp and tcgen05.mma of one thread run in
+          // issue order, so the MMAs of earlier steps still read the old columns)
+          if ((kb & 3) == 0) tmem_cp_32x128b_warpx4(sfa_t, smem_desc_rows16(sf0));
+          if (Cfg::W4 || (kb & 3) == 0) {
 #pragma unroll
             for (int a = 0; a < Cfg::SFB_ATOMS; ++a)
               tmem_cp_32x128b_warpx4(sfb_t + 4 * a, smem_desc_rows16(sf0 + 512 * (1 + a)));
           }
-          const uint32_t idesc = idesc_mxf8_e4m3(BM, BN, kb & 3, kb & 3);
 #pragma unroll
           for (int kk = 0; kk < BK / 32; ++kk) {
+            // A: byte kb%4 (one scale per 128 K); B: byte kk of this step's atom (e2m1,
+            // one scale per 32 K) or byte kb%4 (e4m3)
+            const uint32_t idesc = Cfg::W4 ? idesc_mxf8_e4m3(BM, BN, kb & 3, kk, kFmtE2M1)
+                                           : idesc_mxf8_e4m3(BM, BN, kb & 3, kb & 3);
             umma_mxf8(d_tmem, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32), idesc, sfa_t, sfb_t,
                       (kb | kk) != 0);
           }

@@ -2,8 +2,8 @@
 
 This module only draws numbers: Gaussian activations and weights of the sizes a
 workload names, the selection bias, the Zipf-shaped router of the skew stress case
-and, for the FP8 workload, the e4m3 codes plus power-of-two block scales that the
-layer then consumes as given inputs. It computes no part of the layer (no routing,
+and, for the FP8 workloads, the e4m3 (and e2m1 weight) codes plus power-of-two block
+scales that the layer then consumes as given inputs. It computes no part of the layer (no routing,
 no permutation, no expert FFN, no combine), so both the CUDA path and the CPU
 oracle can be fed from it without sharing any of the method's arithmetic.
 
@@ -18,7 +18,7 @@ import math
 
 import torch
 
-from .workloads import Workload, DTYPE_FP8
+from .workloads import Workload, DTYPE_FP8, DTYPE_FP8_FP4
 
 _TAGS = {"x": 1, "w_r": 2, "bias": 3, "w_gate": 4, "w_up": 5, "w_down": 6,
          "ws_gate": 7, "ws_up": 8, "ws_down": 9, "skew_m": 10, "skew_rank": 11}
@@ -80,6 +80,47 @@ def quantize_blocks_e4m3(v: torch.Tensor, rows_per_block: int):
     return q.view(torch.uint8), s.contiguous()
 
 
+FP4_MAX = 6.0
+FP4_BLOCK = 32
+# The eight non-negative e2m1 values (OCP MX FP4), in code order 0..7.
+_E2M1_POS = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)
+
+
+def quantize_rows_e2m1(v: torch.Tensor):
+    """Encode a [R, C] fp32 matrix as e2m1 codes with one power-of-two scale per row and
+    32 columns (the smallest with amax / scale <= 6), nearest value with ties to the
+    even code.  Returns (packed uint8 [R, C/2] with element 2j in the low nibble, UE8M0
+    scale bytes uint8 [R, C/32] = log2(scale) + 127).  This is how the FP8 x FP4
+    workload's given weights are produced."""
+    R, C = v.shape
+    assert C % FP4_BLOCK == 0 and C % 2 == 0
+    b = v.reshape(R, C // FP4_BLOCK, FP4_BLOCK)
+    amax = b.abs().amax(dim=2)
+    mant, expo = torch.frexp(amax / FP4_MAX)
+    e = torch.where(mant == 0.5, expo - 1, expo)
+    e = torch.where(amax > 0, e, torch.zeros_like(e)).clamp(-127, 127)
+    a = (b.abs() / torch.ldexp(torch.ones_like(amax), e)[:, :, None]).clamp(max=FP4_MAX)
+    grid = torch.tensor(_E2M1_POS, device=v.device, dtype=a.dtype)
+    hi = torch.bucketize(a, grid).clamp(max=len(_E2M1_POS) - 1)      # first grid value >= a
+    lo = (hi - 1).clamp(min=0)
+    d_lo = a - grid[lo]
+    d_hi = grid[hi] - a
+    take_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    code = torch.where(take_hi, hi, lo) | torch.where(b < 0, 8, 0)
+    code = code.reshape(R, C).to(torch.uint8)
+    packed = code[:, 0::2] | (code[:, 1::2] << 4)
+    return packed.contiguous(), (e + 127).to(torch.uint8).contiguous()
+
+
+def _stacked_fp4(n, rows, cols, g, device):
+    packed = torch.empty((n, rows, cols // 2), dtype=torch.uint8, device=device)
+    scales = torch.empty((n, rows, cols // FP4_BLOCK), dtype=torch.uint8, device=device)
+    for e in range(n):
+        w = torch.randn((rows, cols), generator=g, device=device, dtype=torch.float32) * WEIGHT_STD
+        packed[e], scales[e] = quantize_rows_e2m1(w)
+    return packed, scales
+
+
 def _stacked_fp8(n, rows, cols, g, device):
     codes = torch.empty((n, rows, cols), dtype=torch.uint8, device=device)
     scales = torch.empty((n, rows // QBLOCK, cols // QBLOCK), dtype=torch.float32, device=device)
@@ -97,7 +138,9 @@ def make_inputs(wl: Workload, seed: int = 0, device="cpu", weights: bool = True)
     ws_gate/ws_up [I_sh,H], ws_down [H,I_sh] bf16.
     FP8 workload: x is replaced by x_q [T,H] uint8 (e4m3 codes) + x_scale
     [T,H/128] fp32, and each expert weight W by W_q uint8 + W_s fp32
-    [E, rows/128, cols/128].  With weights=False only x (and the router) are drawn.
+    [E, rows/128, cols/128].  FP8 x FP4 workload: x as for FP8; W_q is packed e2m1
+    uint8 [E, rows, cols/2] and W_s UE8M0 bytes uint8 [E, rows, cols/32].  With
+    weights=False only x (and the router) are drawn.
     """
     T, H, I, E = wl.T, wl.H, wl.I, wl.E
     out = {}
@@ -109,7 +152,7 @@ def make_inputs(wl: Workload, seed: int = 0, device="cpu", weights: bool = True)
         x = torch.randn((T, H), generator=g, device=device, dtype=torch.float32) + m
     else:
         x = torch.randn((T, H), generator=g, device=device, dtype=torch.float32)
-    if wl.dtype == DTYPE_FP8:
+    if wl.dtype in (DTYPE_FP8, DTYPE_FP8_FP4):
         out["x_q"], out["x_scale"] = quantize_blocks_e4m3(x, 1)
     else:
         out["x"] = x.to(torch.bfloat16)
@@ -136,6 +179,9 @@ def make_inputs(wl: Workload, seed: int = 0, device="cpu", weights: bool = True)
     if wl.dtype == DTYPE_FP8:
         for name, rows, cols in (("w_gate", I, H), ("w_up", I, H), ("w_down", H, I)):
             out[name + "_q"], out[name + "_s"] = _stacked_fp8(E, rows, cols, _gen(device, seed, name), device)
+    elif wl.dtype == DTYPE_FP8_FP4:
+        for name, rows, cols in (("w_gate", I, H), ("w_up", I, H), ("w_down", H, I)):
+            out[name + "_q"], out[name + "_s"] = _stacked_fp4(E, rows, cols, _gen(device, seed, name), device)
     else:
         out["w_gate"] = _stacked_normal(E, (I, H), WEIGHT_STD, _gen(device, seed, "w_gate"), device)
         out["w_up"] = _stacked_normal(E, (I, H), WEIGHT_STD, _gen(device, seed, "w_up"), device)

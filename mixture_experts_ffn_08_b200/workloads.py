@@ -17,6 +17,7 @@ SCORE_SIGMOID = 1
 
 DTYPE_BF16 = 0
 DTYPE_FP8 = 1
+DTYPE_FP8_FP4 = 2      # e4m3 activations, e2m1 weights with UE8M0 scales per 32 K elements
 
 
 @dataclass(frozen=True)
@@ -63,7 +64,14 @@ DSV3_DECODE = DSV3_PREFILL.with_(name="dsv3_decode", T=128)
 SKEWED_FP8 = Workload("skewed_fp8", T=16384, H=4096, I=1536, E=128, K=8,
                       dtype=DTYPE_FP8, skewed=True)
 
+# FP8 x FP4 expert GEMMs ("DeepGEMM质变" §5.3, the Mega MoE compute unit) on the
+# DeepSeek-V3 routed experts: decode (expert weights streamed from HBM at half the FP8
+# bytes) and prefill.  Routed experts only: the shared expert stays a bf16-only feature.
+DSV3_DECODE_FP4 = DSV3_DECODE.with_(name="dsv3_decode_fp4", dtype=DTYPE_FP8_FP4, I_shared=0)
+DSV3_PREFILL_FP4 = DSV3_PREFILL.with_(name="dsv3_prefill_fp4", dtype=DTYPE_FP8_FP4, I_shared=0)
+
 ALL = {w.name: w for w in (TINY, MIXTRAL_PREFILL, DSV3_PREFILL, DSV3_DECODE, SKEWED_FP8)}
+FP4 = {w.name: w for w in (DSV3_DECODE_FP4, DSV3_PREFILL_FP4)}
 
 # Stand-ins small enough for a full profiler capture (a few GB on the device) that keep
 # the tile structure of a full workload: DeepSeek-V3 expert shapes with 32 experts and

@@ -35,7 +35,7 @@ def f64(t) -> np.ndarray:
 
 def x_f64(d, wl, rows=None):
     """Exact values of x (dequantised for FP8) as float64, optionally a row subset."""
-    if wl.dtype == W.DTYPE_FP8:
+    if wl.dtype in (W.DTYPE_FP8, W.DTYPE_FP8_FP4):
         q, s = d["x_q"], d["x_scale"]
         if rows is not None:
             q, s = q[rows], s[rows]
@@ -56,6 +56,9 @@ def expert_weights_fn(d, wl):
                 cache[e] = tuple(
                     o.dequant_blocks(d[n + "_q"][e].cpu().numpy(), d[n + "_s"][e].cpu().numpy(), 128)
                     for n in ("w_gate", "w_up", "w_down"))
+            elif wl.dtype == W.DTYPE_FP8_FP4:
+                cache[e] = tuple(o.dequant_fp4(d[n + "_q"][e].cpu().numpy(), d[n + "_s"][e].cpu().numpy())
+                                 for n in ("w_gate", "w_up", "w_down"))
             else:
                 cache[e] = tuple(f64(d[n][e]) for n in ("w_gate", "w_up", "w_down"))
         return cache[e]
@@ -68,7 +71,24 @@ def shared_weights(d, wl):
     return tuple(f64(d[n]) for n in ("ws_gate", "ws_up", "ws_down"))
 
 
+def prepare_fp4_atoms(d, wl):
+    """Scale atoms of the three e2m1 weight tensors (moe_prepare_fp4_scales), stored in
+    d as <name>_atoms."""
+    for n, rows, K in (("w_gate", wl.E * wl.I, wl.H), ("w_up", wl.E * wl.I, wl.H), ("w_down", wl.E * wl.H, wl.I)):
+        if n + "_atoms" not in d:
+            atoms = torch.empty(rows * K // 32, dtype=torch.uint8, device="cuda")
+            B.check(B.moe_prepare_fp4_scales(d[n + "_s"], rows, K, atoms), "moe_prepare_fp4_scales")
+            d[n + "_atoms"] = atoms
+    return d
+
+
 def device_inputs_ptrs(d, wl):
+    if wl.dtype == W.DTYPE_FP8_FP4:
+        prepare_fp4_atoms(d, wl)
+        return dict(
+            x=d["x_q"], x_scale=d["x_scale"], w_r=d["w_r"], bias=d["bias"], w_gate=d["w_gate_q"],
+            w_up=d["w_up_q"], w_down=d["w_down_q"], w_gate_scale=d["w_gate_atoms"], w_up_scale=d["w_up_atoms"],
+            w_down_scale=d["w_down_atoms"], ws_gate=None, ws_up=None, ws_down=None)
     fp8 = wl.dtype == W.DTYPE_FP8
     return dict(
         x=d["x_q"] if fp8 else d["x"], x_scale=d.get("x_scale"), w_r=d["w_r"], bias=d["bias"],

@@ -44,3 +44,32 @@ def test_skew_router_makes_one_expert_hot():
     mean = wl.T * wl.K / wl.E
     assert counts.max() >= 0.85 * wl.T and counts.max() / mean >= 13
     assert (counts == 0).sum() >= 1
+
+
+def test_e2m1_weight_quantiser_is_nearest_with_minimal_scale():
+    """The FP8 x FP4 workload's weights: each value is the nearest e2m1 code times the
+    block's power-of-two scale (ties to the even code), and the scale is the smallest
+    power of two that keeps the block's largest magnitude within 6."""
+    torch.manual_seed(1)
+    w = torch.randn(6, 128) * 0.02
+    w[0, :4] = torch.tensor([0.0, 0.25, 0.75, -1.25]) * 2.0 ** -3   # exact ties on the grid
+    packed, sb = inputs.quantize_rows_e2m1(w)
+    assert packed.shape == (6, 64) and sb.shape == (6, 4)
+    deq = o.dequant_fp4(packed.numpy(), sb.numpy())
+    grid = o.decode_e2m1(np.arange(16))
+    wv = w.double().numpy().reshape(6, 4, 32)
+    scale = np.ldexp(1.0, sb.numpy().astype(np.int64) - 127)
+    amax = np.abs(wv).max(axis=2)
+    assert (amax / scale <= 6.0).all() and ((amax / (scale / 2) > 6.0) | (amax == 0)).all()
+    for r in range(6):
+        for b in range(4):
+            for j in range(32):
+                a = wv[r, b, j] / scale[r, b]
+                d = np.abs(grid - a)
+                best = np.flatnonzero(d == d.min())
+                vals = {float(grid[c]) for c in best}
+                got = deq[r, 32 * b + j] / scale[r, b]
+                assert got in vals
+                if len(vals) > 1:  # a tie: the even code wins
+                    even = [c for c in best if c % 2 == 0]
+                    assert got == grid[even[0]]
