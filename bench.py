@@ -91,7 +91,7 @@ def _describe(wl):
         s += f" block_m={wl.block_m}"
     if wl.masked_cap:
         s += f" masked-layout cap={wl.masked_cap}"
-    return s + (" fp8" if wl.dtype else " bf16")
+    return s + {W.DTYPE_BF16: " bf16", W.DTYPE_FP8: " fp8", W.DTYPE_FP8_FP4: " fp8 x fp4 weights"}[wl.dtype]
 
 
 def _dist():
@@ -150,7 +150,7 @@ def _oracle_sample(wl, d, n_tokens, seed=0):
     toks = np.sort(rng.choice(wl.T, size=min(n_tokens, wl.T), replace=False))
     idx = torch.as_tensor(toks, device=d["w_r"].device)
     # host copies of the inputs are not part of the timed oracle work
-    if wl.dtype == W.DTYPE_FP8:
+    if wl.dtype in (W.DTYPE_FP8, W.DTYPE_FP8_FP4):
         xq, xs = d["x_q"][idx].cpu().numpy(), d["x_scale"][idx].cpu().numpy()
         x_of = lambda: o.dequant_blocks(xq, xs, 1)  # noqa: E731
     else:
@@ -162,7 +162,7 @@ def _oracle_sample(wl, d, n_tokens, seed=0):
 
     def fetch(e):
         if e not in host_w:
-            if wl.dtype == W.DTYPE_FP8:
+            if wl.dtype in (W.DTYPE_FP8, W.DTYPE_FP8_FP4):
                 host_w[e] = tuple((d[n + "_q"][e].cpu().numpy(), d[n + "_s"][e].cpu().numpy())
                                   for n in ("w_gate", "w_up", "w_down"))
             else:
@@ -181,6 +181,8 @@ def _oracle_sample(wl, d, n_tokens, seed=0):
     def expert_weights(e):
         if wl.dtype == W.DTYPE_FP8:
             return tuple(o.dequant_blocks(q, s, 128) for q, s in fetch(e))
+        if wl.dtype == W.DTYPE_FP8_FP4:
+            return tuple(o.dequant_fp4(q, s) for q, s in fetch(e))
         return tuple(t.to(torch.float64).numpy() for t in fetch(e))
 
     t0 = time.perf_counter()
@@ -210,7 +212,7 @@ def run_ours(args):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
-    wl = {**W.ALL, **W.PROFILE}[args.workload]
+    wl = {**W.ALL, **W.PROFILE, **W.FP4}[args.workload]
     if args.fused_combine:
         wl = wl.with_(fused_combine=True)
     if args.block_m:
@@ -219,10 +221,19 @@ def run_ours(args):
         wl = wl.with_(masked_cap=args.masked_cap)
     p = B.params(wl)
     d = inputs.make_inputs(wl, seed=rank, device="cuda")
-    fp8 = wl.dtype == W.DTYPE_FP8
+    fp8 = wl.dtype in (W.DTYPE_FP8, W.DTYPE_FP8_FP4)     # e4m3 activations
+    w4 = wl.dtype == W.DTYPE_FP8_FP4                    # e2m1 expert weights
     a = dict(x=d["x_q"] if fp8 else d["x"], x_scale=d.get("x_scale"))
+    scales = [d.get("w_gate_s"), d.get("w_up_s"), d.get("w_down_s")]
+    if w4:  # weight-load step, once: UE8M0 scale bytes -> tensor-core scale atoms
+        scales = []
+        for n, rows, K in (("w_gate", wl.E * wl.I, wl.H), ("w_up", wl.E * wl.I, wl.H),
+                           ("w_down", wl.E * wl.H, wl.I)):
+            atoms = torch.empty(rows * K // 32, dtype=torch.uint8, device="cuda")
+            B.check(B.moe_prepare_fp4_scales(d[n + "_s"], rows, K, atoms), "moe_prepare_fp4_scales")
+            scales.append(atoms)
     wts = [d["w_gate_q"] if fp8 else d["w_gate"], d["w_up_q"] if fp8 else d["w_up"],
-           d["w_down_q"] if fp8 else d["w_down"], d.get("w_gate_s"), d.get("w_up_s"), d.get("w_down_s"),
+           d["w_down_q"] if fp8 else d["w_down"], *scales,
            d.get("ws_gate"), d.get("ws_up"), d.get("ws_down")]
     ws_bytes = B.moe_workspace_size_host(p)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
@@ -295,15 +306,16 @@ def run_ours(args):
     tokens_per_s = wl.T * world / (ms_step / 1e3)
 
     # algorithmic work (unpadded rows; weights of experts that received tokens)
-    wbytes = 1 if fp8 else 2
+    abytes = 1 if fp8 else 2                       # activation bytes per element
+    wbytes = (0.5 + 1 / 32) if w4 else abytes       # weight bytes per element (e2m1: + one scale byte per 32)
     active = int((counts_h > 0).sum())
     flops_gateup = 4.0 * P * wl.H * wl.I
     flops_down = 2.0 * P * wl.I * wl.H
     flops_shared = 6.0 * wl.T * wl.H * wl.I_shared
     gemm_flops = flops_gateup + flops_down + flops_shared
-    bytes_gateup = (active * 2 * wl.I * wl.H * wbytes + P * wl.H * wbytes + P * wl.I * wbytes)
+    bytes_gateup = (active * 2 * wl.I * wl.H * wbytes + P * wl.H * abytes + P * wl.I * abytes)
     layer_bytes = (active * 3 * wl.I * wl.H * wbytes + 3 * wl.I_shared * wl.H * 2 + wl.E * wl.H * 2
-                   + wl.T * wl.H * (wbytes + 2))
+                   + wl.T * wl.H * (abytes + 2))
     burst, sustained, hbm_peak, peak_kind = _peaks()
     # a kernel timed inside a long, power-capped run is held to the sustained figure
     capped = bool(clk and ("sw_power_cap" in clk.get("reasons", []) or
@@ -311,7 +323,7 @@ def run_ours(args):
                             clk["sm_mhz"] < 0.9 * clk["sm_max_mhz"])))
     ratio = FP8_OVER_BF16 if fp8 else 1.0
     tensor_peak = (sustained if capped else burst) * ratio
-    dt_name = "e4m3" if fp8 else "bf16"
+    dt_name = "e4m3 x e2m1" if w4 else ("e4m3" if fp8 else "bf16")
     dom_ms = [ms for k, ms in traced if k == dominant]
     dom_avg = statistics.mean(dom_ms) if dom_ms else None
     ridge = tensor_peak * 1e12 / (hbm_peak * 1e9)
@@ -380,7 +392,8 @@ def run_ours(args):
     line = {
         "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp8" if fp8 else "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8xfp4" if w4 else ("fp8" if fp8 else "bf16"),
         "data": "synthetic (seeded Gaussian activations and random-init weights)",
         "config": {"workload": f"{wl.name}: {_describe(wl)}", "global_batch": wl.T * world,
                    "seq_len": 1, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
@@ -411,7 +424,7 @@ def run_reference(args):
     world, rank, _ = _dist()
     if rank != 0:
         return
-    wl = {**W.ALL, **W.PROFILE}[args.workload]
+    wl = {**W.ALL, **W.PROFILE, **W.FP4}[args.workload]
     d = inputs.make_inputs(wl, seed=0, device="cpu" if not torch.cuda.is_available() else "cuda")
     n = max(2, _cpu_sample_tokens(wl) // 8)
     times, toks, threads = [], 0, 1
@@ -480,7 +493,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="mixtral_prefill", choices=sorted(W.ALL) + sorted(W.PROFILE))
+    ap.add_argument("--workload", default="mixtral_prefill", choices=sorted(W.ALL) + sorted(W.PROFILE) + sorted(W.FP4))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--fused-combine", action="store_true",
