@@ -40,12 +40,23 @@ FLUSH_BYTES = 512 << 20
 
 
 GEMM_SOURCES = ("csrc/tc_gemm.cuh", "csrc/common.cuh", "csrc/gemm.cu")
+FP8_GEMM_SOURCES = ("csrc/tc_gemm_fp8.cuh", "csrc/tc_gemm.cuh", "csrc/common.cuh", "csrc/gemm_fp8.cu")
+
+
+def sources_sha256(files):
+    """sha256 over the given source files of the package, in order."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "mixture_experts_ffn_08_b200", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
 
 
 def _profiled_traffic(workload):
     """DRAM bytes per launch of the gate/up kernel from the committed ncu summary of this
-    workload, or None if there is none or the kernel sources changed since it was taken."""
-    import hashlib
+    workload, or None if there is none or the kernel sources changed since it was taken.
+    The summary names the sources it covers (kernel_sources:, default the bf16 GEMM)."""
     import re
     path = os.path.join(ROOT, "profiles", f"gateup_swiglu_{workload}.md")
     if not os.path.exists(path):
@@ -53,13 +64,11 @@ def _profiled_traffic(workload):
     txt = open(path, encoding="utf-8").read()
     m_t = re.search(r"^traffic_bytes_per_launch:\s*(\d+)", txt, re.M)
     m_h = re.search(r"^kernel_source_sha256:\s*([0-9a-f]+)", txt, re.M)
+    m_s = re.search(r"^kernel_sources:\s*(.+)$", txt, re.M)
     if not (m_t and m_h):
         return None
-    h = hashlib.sha256()
-    for f in GEMM_SOURCES:
-        with open(os.path.join(ROOT, "mixture_experts_ffn_08_b200", f), "rb") as fh:
-            h.update(fh.read())
-    return int(m_t.group(1)) if h.hexdigest() == m_h.group(1) else None
+    files = [f.strip() for f in m_s.group(1).split(",")] if m_s else list(GEMM_SOURCES)
+    return int(m_t.group(1)) if sources_sha256(files) == m_h.group(1) else None
 
 
 def _peaks():
@@ -199,7 +208,7 @@ def _cpu_sample_tokens(wl):
     # about 10-30 s of fp64 work on a few host cores; with many experts each sampled
     # token brings K experts' weights to widen, which dominates, so sample fewer tokens
     per_token_flops = 6 * wl.K * wl.H * wl.I + 6 * wl.H * wl.I_shared
-    n = int(max(4, min(wl.T, 2.0e11 / max(per_token_flops, 1) / 4)))
+    n = int(max(4, min(wl.T, 2.5e12 / max(per_token_flops, 1) / 4)))
     return min(n, 8) if wl.E > 16 else n
 
 

@@ -100,8 +100,12 @@ struct TileCoord {
 };
 
 // Work item -> (M-tile, N-tile, group).  Items of group g occupy [mt0*NT, mt1*NT) where
-// [mt0, mt1) are g's M-tiles; inside that range N-tiles are outer, M-tiles inner.
-MOE_DEVINL TileCoord decode_item(int item, int NT, const GemmParams& p, int num_m_tiles) {
+// [mt0, mt1) are g's M-tiles.  Inside that range the operand with fewer rows is the one
+// re-read from L2 by the CTAs running side by side: N-tiles outer (each weight tile is
+// shared by all M-tiles in flight) when the group's weight rows NT*b_rows outnumber its
+// activation rows, M-tiles outer (each activation tile shared by all N-tiles) otherwise,
+// as for a hot expert of a skewed load or the dense shared expert.
+MOE_DEVINL TileCoord decode_item(int item, int NT, const GemmParams& p, int num_m_tiles, int b_rows) {
   const int v = item / NT;  // an M-tile of the same group
   int g = 0, mt0 = 0, cnt = num_m_tiles;
   if (p.offsets != nullptr) {
@@ -116,9 +120,10 @@ MOE_DEVINL TileCoord decode_item(int item, int NT, const GemmParams& p, int num_
     cnt = (__ldg(p.offsets + g + 1) >> 7) - mt0;
   }
   const int local = item - mt0 * NT;
+  const bool m_outer = cnt * 128 > NT * b_rows;
   TileCoord t;
-  t.m_tile = mt0 + local % cnt;
-  t.n_tile = local / cnt;
+  t.m_tile = mt0 + (m_outer ? local / NT : local % cnt);
+  t.n_tile = m_outer ? local % NT : local / cnt;
   t.group = g;
   t.local0 = (t.m_tile - mt0) * 128;
   t.row0 = p.masked_cap > 0 ? g * p.masked_cap + t.local0 : t.m_tile * 128;
@@ -187,7 +192,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       long long issued = 0;
       bool ok = true;
       for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
-        const TileCoord t = decode_item(item, NT, p, num_m_tiles);
+        const TileCoord t = decode_item(item, NT, p, num_m_tiles, BN);
         const int a_row = t.row0;
         const int b_row = t.group * p.b_rows_per_group + t.n_tile * Cfg::OUT_COLS;
         for (int kb = 0; kb < KB; ++kb) {
@@ -255,7 +260,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     int acc = 0;
     uint32_t acc_ph = 0;
     for (int item = blockIdx.x; item < total; item += gridDim.x) {
-      const TileCoord t = decode_item(item, NT, p, num_m_tiles);
+      const TileCoord t = decode_item(item, NT, p, num_m_tiles, BN);
       // every lane polls, then the warp agrees (tcgen05.ld below is warp-collective)
       const bool ready = __all_sync(0xffffffffu, mbar_wait_bounded(&tfull_bar[acc], acc_ph, &abort_flag));
       if (!ready) break;

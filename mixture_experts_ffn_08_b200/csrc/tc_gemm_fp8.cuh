@@ -230,7 +230,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       bool ok = true;
       const int nblk = p.N / 128;  // 128-row weight blocks per group
       for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
-        const TileCoord t = decode_item(item, NT, gp, num_m_tiles);
+        const TileCoord t = decode_item(item, NT, gp, num_m_tiles, BN);
         const int a_row = t.row0;
         const int b_row = t.group * p.N + t.n_tile * Cfg::OUT_COLS;
         const int wblk = t.group * nblk + (t.n_tile * Cfg::OUT_COLS) / 128;
@@ -331,7 +331,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     int acc = 0;
     uint32_t acc_ph = 0;
     for (int item = blockIdx.x; item < total; item += gridDim.x) {
-      const TileCoord t = decode_item(item, NT, gp, num_m_tiles);
+      const TileCoord t = decode_item(item, NT, gp, num_m_tiles, BN);
       const bool ready = __all_sync(0xffffffffu, mbar_wait_bounded(&tfull_bar[acc], acc_ph, &abort_flag));
       if (!ready) break;
       tc_fence_after();
