@@ -81,6 +81,7 @@ def _peaks():
     return 1590.0, 1400.0, 6650.0, "fallback"
 
 
+REFERENCE_BUDGET_S = 90.0   # oracle seconds for a whole --impl reference run
 FP8_OVER_BF16 = 2.0   # nominal dense e4m3 / bf16 tensor throughput (4.5 / 2.25 PFLOP/s)
 
 
@@ -150,9 +151,10 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ CPU oracle leg
-def _oracle_sample(wl, d, n_tokens, seed=0):
+def _oracle_sample(wl, d, n_tokens, seed=0, host_w=None):
     """Oracle forward (route + experts + combine) of a seeded token sample; returns
-    (tokens, seconds, threads)."""
+    (tokens, seconds, threads).  host_w caches host copies of expert weights across
+    calls (filled here, outside the timed part)."""
     from oracle import moe_oracle as o
     from threadpoolctl import threadpool_info
     rng = np.random.default_rng(seed)
@@ -167,7 +169,8 @@ def _oracle_sample(wl, d, n_tokens, seed=0):
         x_of = lambda: xh  # noqa: E731
     w_r = d["w_r"].cpu().to(torch.float64).numpy()
     bias = d["bias"].cpu().to(torch.float64).numpy() if d["bias"] is not None else None
-    host_w = {}
+    if host_w is None:
+        host_w = {}
 
     def fetch(e):
         if e not in host_w:
@@ -435,10 +438,19 @@ def run_reference(args):
         return
     wl = {**W.ALL, **W.PROFILE, **W.FP4}[args.workload]
     d = inputs.make_inputs(wl, seed=0, device="cpu" if not torch.cuda.is_available() else "cuda")
-    n = max(2, _cpu_sample_tokens(wl) // 8)
+    host_w = {}
+    # size each step's token sample so that all warm-up and timed steps together take about
+    # REFERENCE_BUDGET_S of oracle time.  A step costs about c0 + n*c1 (c0: widening the
+    # chosen experts' weights to fp64; c1: per token); two untimed samples fix c0 and c1.
+    k1, t1, _ = _oracle_sample(wl, d, 2, seed=10 ** 6, host_w=host_w)
+    k2, t2, _ = _oracle_sample(wl, d, 8, seed=10 ** 6 + 1, host_w=host_w)
+    c1 = max((t2 - t1) / max(k2 - k1, 1), 1e-6)
+    c0 = max(t1 - k1 * c1, 0.0)
+    per_step = REFERENCE_BUDGET_S / (args.warmup + args.steps)
+    n = int(max(1, min(wl.T, _cpu_sample_tokens(wl), (per_step - c0) / c1)))
     times, toks, threads = [], 0, 1
     for i in range(args.warmup + args.steps):
-        k, dt, threads = _oracle_sample(wl, d, n, seed=i)
+        k, dt, threads = _oracle_sample(wl, d, n, seed=i, host_w=host_w)
         if i >= args.warmup:
             times.append(dt)
             toks += k
