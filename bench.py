@@ -104,6 +104,23 @@ def _describe(wl):
     return s + {W.DTYPE_BF16: " bf16", W.DTYPE_FP8: " fp8", W.DTYPE_FP8_FP4: " fp8 x fp4 weights"}[wl.dtype]
 
 
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The largest value over all ranks (the slowest rank's time); the value itself on one
+    rank.  Every rank must call it at the same point."""
+    if world <= 1:
+        return float(value)
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(tokens_per_rank: int, world: int, ms_step: float) -> float:
+    """Whole-job tokens/s of `world` independent replicas, each processing tokens_per_rank
+    tokens per step, timed by the slowest rank's ms per step."""
+    return tokens_per_rank * world / (ms_step / 1e3)
+
+
 def _dist():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -308,14 +325,9 @@ def run_ours(args):
 
     counts_h = counts.cpu().numpy()
     P = wl.T * wl.K
-    ms_total = float(sum(step_ms))
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms_total], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(float(sum(step_ms)), world, "cuda")
     ms_step = ms_total / args.steps
-    tokens_per_s = wl.T * world / (ms_step / 1e3)
+    tokens_per_s = replica_throughput(wl.T, world, ms_step)
 
     # algorithmic work (unpadded rows; weights of experts that received tokens)
     abytes = 1 if fp8 else 2                       # activation bytes per element
@@ -379,13 +391,7 @@ def run_ours(args):
             e2e_step()
             ev2[i][1].record(stream)
         barrier()
-        e2e_ms = sum(s.elapsed_time(e) for s, e in ev2)
-        if world > 1:
-            import torch.distributed as dist
-            t = torch.tensor([e2e_ms], device="cuda", dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e_ms /= args.steps
+        e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in ev2), world, "cuda") / args.steps
     xbytes = wl.T * wl.H * (1 if fp8 else 2) + (wl.T * (wl.H // 128) * 4 if fp8 else 0)
 
     cpu = None
