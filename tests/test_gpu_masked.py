@@ -142,6 +142,19 @@ def test_masked_layer_matches_contiguous_layer(base):
     assert torch.equal(contig["out"], masked["out"])
 
 
+def test_masked_layer_with_fused_combine():
+    """Masked layout and the fused down + combine together: the same outputs as the
+    contiguous deterministic layer within the bf16 bounds (atomics reorder the sums)."""
+    wl = W.DSV3_PREFILL.with_(name="small_dsv3_fused", T=200, H=512, I=256, E=32, n_group=4, topk_group=2,
+                              I_shared=256)
+    d = inputs.make_inputs(wl, seed=5, device="cuda")
+    ref = P.run_layer(wl, d)
+    got = P.run_layer(wl.with_(masked_cap=256, fused_combine=True), d)
+    assert B.moe_get_device_status(got["ws"]) == 0
+    assert torch.equal(ref["ids"], got["ids"])
+    P.check_close(P.f64(got["out"]), P.f64(ref["out"]), P.BF16_MAX_TOL, "masked fused")
+
+
 def test_masked_layer_overflow_leaves_pairs_out():
     # a selection-only bias of +10 on expert 3 makes every token choose it: 400 pairs
     # for 128 rows (the weights still come from the unbiased scores)
