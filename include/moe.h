@@ -24,8 +24,10 @@
  *     launched.  Errors found by a kernel (an expert id out of range, a pipeline wait that
  *     timed out) are OR-ed into a status word inside `ws`; read it with
  *     moe_get_device_status().  No kernel traps.
- *   - Base pointers of bf16 / e4m3 matrices must be 16-byte aligned; H and I must be
- *     multiples of 128.
+ *   - Base pointers of bf16 / e4m3 matrices must be 16-byte aligned (e2m1 weights:
+ *     32-byte); H and I must be multiples of 128.
+ *   - "FP8" below means both dtypes with e4m3 activations (MOE_DTYPE_FP8_E4M3 and
+ *     MOE_DTYPE_FP8_FP4).
  *   - Weight layout is [out_features, in_features] (nn.Linear): W_r [E,H];
  *     W_gate, W_up [E,I,H]; W_down [E,H,I]; shared expert Ws_gate, Ws_up [I_shared,H],
  *     Ws_down [H,I_shared].
