@@ -228,7 +228,7 @@ def _cpu_sample_tokens(wl):
     # about 10-30 s of fp64 work on a few host cores; with many experts each sampled
     # token brings K experts' weights to widen, which dominates, so sample fewer tokens
     per_token_flops = 6 * wl.K * wl.H * wl.I + 6 * wl.H * wl.I_shared
-    n = int(max(4, min(wl.T, 2.5e12 / max(per_token_flops, 1) / 4)))
+    n = int(max(4, min(wl.T, 2.0e13 / max(per_token_flops, 1) / 4)))
     return min(n, 8) if wl.E > 16 else n
 
 
