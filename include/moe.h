@@ -55,7 +55,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 4
+#define MOE_ABI_VERSION 5
 
 typedef enum moe_status {
   MOE_OK = 0,
@@ -284,6 +284,14 @@ moe_status_t moe_prepare_fp4_scales(const void* scale_words, int64_t rows, int32
 moe_status_t moe_get_device_status(const void* ws, void* stream, int32_t* host_status);
 /* Clears the device status word of `ws` (asynchronous on `stream`). */
 moe_status_t moe_clear_device_status(void* ws, void* stream);
+
+/* Failure-path self-test (no counterpart on the pages).  One CTA waits on an mbarrier
+ * that nothing completes, using the same bounded wait as the GEMM pipelines, with a
+ * limit of limit_ms (1..2000) instead of the pipelines' 2 s.  When the limit runs out
+ * the wait gives up, MOE_DEV_TIMEOUT is OR-ed into the status word of `ws` (first 256
+ * bytes, 256-byte aligned), and the kernel returns: the context stays usable.
+ * Asynchronous on `stream`. */
+moe_status_t moe_selftest_bounded_wait(void* ws, int32_t limit_ms, void* stream);
 
 const char* moe_status_string(moe_status_t s);
 int32_t moe_abi_version(void);

@@ -77,6 +77,7 @@ _SIGS = {
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_abi_version": (ctypes.c_int32, []),
     "moe_prepare_fp4_scales": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.c_int32, _P, _P]),
+    "moe_selftest_bounded_wait": (ctypes.c_int, [_P, ctypes.c_int32, _P]),
     "moe_trace_enable": (ctypes.c_int, [ctypes.c_uint32, ctypes.c_int32]),
     "moe_trace_disable": (ctypes.c_int, []),
     "moe_trace_collect": (ctypes.c_int32, [ctypes.POINTER(ctypes.c_int32),
@@ -238,6 +239,10 @@ def moe_status_string(s: int) -> str:
 
 def moe_abi_version() -> int:
     return lib(require_gpu=False).moe_abi_version()
+
+
+def moe_selftest_bounded_wait(ws, limit_ms: int, stream=None) -> int:
+    return lib().moe_selftest_bounded_wait(_ptr(ws), limit_ms, _stream(stream))
 
 
 def moe_prepare_fp4_scales(scale_bytes, rows: int, K: int, atoms, stream=None) -> int:

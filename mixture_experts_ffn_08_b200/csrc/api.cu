@@ -554,6 +554,13 @@ const char* moe_status_string(moe_status_t s) {
 
 int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
 
+moe_status_t moe_selftest_bounded_wait(void* ws, int32_t limit_ms, void* stream) {
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0 || limit_ms < 1 || limit_ms > 2000)
+    return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_bounded_wait_selftest(static_cast<int32_t*>(ws), 1000000LL * limit_ms,
+                                                  static_cast<cudaStream_t>(stream)));
+}
+
 moe_status_t moe_prepare_fp4_scales(const void* scale_words, int64_t rows, int32_t K, void* atoms, void* stream) {
   if (!scale_words || !atoms || rows <= 0 || rows % 128 != 0 || K <= 0 || K % 128 != 0) return MOE_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(scale_words) & 3u) != 0 || !aligned16(atoms)) return MOE_ERR_INVALID_ARG;

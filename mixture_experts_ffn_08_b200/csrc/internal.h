@@ -39,6 +39,8 @@ cudaError_t launch_bias_update(const int32_t* counts, int E, float gamma, float*
 // `offsets` as the schedule, the 128-padded prefix sums of counts (masked_schedule), and
 // address group g's rows at g * masked_cap.
 cudaError_t launch_masked_schedule(const int32_t* counts, int E, int32_t* sched, cudaStream_t st);
+// One CTA waits on an mbarrier nothing completes, for limit_ns, then sets MOE_DEV_TIMEOUT.
+cudaError_t launch_bounded_wait_selftest(int32_t* status, long long limit_ns, cudaStream_t st);
 // offsets[e] = e * cap for e in [0, E] (masked layout row ranges).
 cudaError_t launch_masked_offsets(int E, int cap, int32_t* offsets, cudaStream_t st);
 cudaError_t launch_permute(const moe_params_t& p, int block_m, const int32_t* ids, const void* x,

@@ -310,6 +310,26 @@ cudaError_t launch_bias_update(const int32_t* counts, int E, float gamma, float*
   return cudaGetLastError();
 }
 
+// ================================================================== bounded-wait self-test
+// One thread waits on an mbarrier that nothing completes, with the same bounded wait
+// the GEMM pipelines use, and reports the give-up as MOE_DEV_TIMEOUT.
+__global__ void bounded_wait_selftest_kernel(int32_t* status, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ volatile int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !mbar_wait_bounded(&bar, 0, &abort_flag, limit_ns)) set_status(status, MOE_DEV_TIMEOUT);
+}
+
+cudaError_t launch_bounded_wait_selftest(int32_t* status, long long limit_ns, cudaStream_t st) {
+  bounded_wait_selftest_kernel<<<1, 32, 0, st>>>(status, static_cast<unsigned long long>(limit_ns));
+  return cudaGetLastError();
+}
+
 // ================================================================== permute
 // 1) per-chunk expert histogram
 __global__ void __launch_bounds__(kPermChunk) perm_count_kernel(

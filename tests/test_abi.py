@@ -38,7 +38,7 @@ def test_exports_every_declared_symbol(lib):
     for name in declared:
         assert hasattr(raw, name), name
     assert declared == set(B.EXPORTED), declared ^ set(B.EXPORTED)
-    assert lib.moe_abi_version() == 4
+    assert lib.moe_abi_version() == 5
 
 
 def test_params_struct_matches_header():
@@ -111,3 +111,10 @@ def test_binding_argument_counts_match_header(lib):
     for name, params in re.findall(r"\b(moe_[a-z0-9_]+)\s*\(([^)]*)\)\s*;", src):
         n = 0 if params.strip() in ("", "void") else params.count(",") + 1
         assert len(B._SIGS[name][1]) == n, (name, n, len(B._SIGS[name][1]))
+
+
+def test_selftest_argument_errors_need_no_gpu(lib):
+    import ctypes
+    assert lib.moe_selftest_bounded_wait(None, 50, None) == 1
+    assert lib.moe_selftest_bounded_wait(ctypes.c_void_p(4096), 0, None) == 1       # limit too small
+    assert lib.moe_selftest_bounded_wait(ctypes.c_void_p(4096 + 8), 50, None) == 1  # misaligned ws
