@@ -85,6 +85,44 @@ REFERENCE_BUDGET_S = 90.0   # oracle seconds for a whole --impl reference run
 FP8_OVER_BF16 = 2.0   # nominal dense e4m3 / bf16 tensor throughput (4.5 / 2.25 PFLOP/s)
 
 
+def power_capped(clk) -> bool:
+    """Whether the clock record says the power cap held the SM clock (sw_power_cap, or a
+    median under load below 90 % of the maximum)."""
+    return bool(clk and ("sw_power_cap" in clk.get("reasons", []) or
+                         (clk.get("sm_mhz") and clk.get("sm_max_mhz") and
+                          clk["sm_mhz"] < 0.9 * clk["sm_max_mhz"])))
+
+
+def roofline_record(flops, nbytes, launch_ms, clk, fp8, peaks):
+    """Roofline of one kernel from its algorithmic FLOPs and bytes per launch and its
+    launch times (ms): tensor-bound when flops/bytes reaches the ridge of the peaks,
+    else HBM-bound.  A power-capped run is held to the sustained tensor peak; e4m3 takes
+    twice the bf16 figure (the nominal dense ratio).  peaks = (bf16 burst TFLOP/s,
+    bf16 sustained TFLOP/s, HBM GB/s, kind)."""
+    burst, sustained, hbm_peak, peak_kind = peaks
+    capped = power_capped(clk)
+    ratio = FP8_OVER_BF16 if fp8 else 1.0
+    tensor_peak = (sustained if capped else burst) * ratio
+    avg = statistics.mean(launch_ms) if launch_ms else None
+    ridge = tensor_peak * 1e12 / (hbm_peak * 1e9)
+    if flops / nbytes >= ridge:
+        achieved = flops / (avg / 1e3) / 1e12 if avg else None
+        rec = {"bound": "tensor", "achieved": achieved, "peak": tensor_peak, "unit": "TFLOP/s",
+               "peak_kind": (f"{peak_kind} bf16 {'sustained' if capped else 'burst'}"
+                             + (" x2 (e4m3/bf16 nominal ratio)" if fp8 else "")),
+               "frac_of_burst": achieved / (burst * ratio) if achieved else None,
+               "frac_of_sustained": achieved / (sustained * ratio) if achieved else None}
+    else:
+        achieved = nbytes / (avg / 1e3) / 1e9 if avg else None
+        rec = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+               "peak_kind": f"{peak_kind} HBM copy"}
+    rec.update({"frac": achieved / rec["peak"] if achieved else None, "launches_timed": len(launch_ms),
+                "avg_ms": avg, "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": nbytes,
+                "tflops": flops / (avg / 1e3) / 1e12 if avg else None,
+                "gbs": nbytes / (avg / 1e3) / 1e9 if avg else None})
+    return rec
+
+
 def _describe(wl):
     s = (f"T={wl.T} H={wl.H} I={wl.I} E={wl.E} K={wl.K} "
          f"{'softmax' if wl.score_fn == 0 else 'sigmoid'}")
@@ -340,35 +378,11 @@ def run_ours(args):
     bytes_gateup = (active * 2 * wl.I * wl.H * wbytes + P * wl.H * abytes + P * wl.I * abytes)
     layer_bytes = (active * 3 * wl.I * wl.H * wbytes + 3 * wl.I_shared * wl.H * 2 + wl.E * wl.H * 2
                    + wl.T * wl.H * (abytes + 2))
-    burst, sustained, hbm_peak, peak_kind = _peaks()
-    # a kernel timed inside a long, power-capped run is held to the sustained figure
-    capped = bool(clk and ("sw_power_cap" in clk.get("reasons", []) or
-                           (clk.get("sm_mhz") and clk.get("sm_max_mhz") and
-                            clk["sm_mhz"] < 0.9 * clk["sm_max_mhz"])))
-    ratio = FP8_OVER_BF16 if fp8 else 1.0
-    tensor_peak = (sustained if capped else burst) * ratio
     dt_name = "e4m3 x e2m1" if w4 else ("e4m3" if fp8 else "bf16")
     dom_ms = [ms for k, ms in traced if k == dominant]
-    dom_avg = statistics.mean(dom_ms) if dom_ms else None
-    ridge = tensor_peak * 1e12 / (hbm_peak * 1e9)
-    if flops_gateup / bytes_gateup >= ridge:
-        achieved = flops_gateup / (dom_avg / 1e3) / 1e12 if dom_avg else None
-        roofline = {"bound": "tensor", "achieved": achieved, "peak": tensor_peak, "unit": "TFLOP/s",
-                    "peak_kind": (f"{peak_kind} bf16 {'sustained' if capped else 'burst'}"
-                                  + (" x2 (e4m3/bf16 nominal ratio)" if fp8 else "")),
-                    "frac_of_burst": achieved / (burst * ratio) if achieved else None,
-                    "frac_of_sustained": achieved / (sustained * ratio) if achieved else None}
-    else:
-        achieved = bytes_gateup / (dom_avg / 1e3) / 1e9 if dom_avg else None
-        roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                    "peak_kind": f"{peak_kind} HBM copy"}
-    roofline.update({
-        "kernel": f"gateup_swiglu (grouped GEMM, fused SwiGLU, {dt_name})",
-        "frac": achieved / roofline["peak"] if achieved else None,
-        "traffic": _profiled_traffic(wl.name), "launches_timed": len(dom_ms), "avg_ms": dom_avg,
-        "algorithmic_flops_per_launch": flops_gateup, "algorithmic_bytes_per_launch": bytes_gateup,
-        "tflops": flops_gateup / (dom_avg / 1e3) / 1e12 if dom_avg else None,
-        "gbs": bytes_gateup / (dom_avg / 1e3) / 1e9 if dom_avg else None})
+    roofline = roofline_record(flops_gateup, bytes_gateup, dom_ms, clk, fp8, _peaks())
+    roofline.update({"kernel": f"gateup_swiglu (grouped GEMM, fused SwiGLU, {dt_name})",
+                     "traffic": _profiled_traffic(wl.name)})
 
     # ---------------- end to end: host activations in, host output out
     x_host = (d["x_q"] if fp8 else d["x"]).cpu().pin_memory()

@@ -1,0 +1,42 @@
+"""The bench's roofline arithmetic on made-up numbers (no GPU): which bound applies,
+which peak a power-capped run is held to, and the fractions it reports."""
+import bench
+
+PEAKS = (1600.0, 1400.0, 6400.0, "measured")   # bf16 burst / sustained TFLOP/s, HBM GB/s
+
+
+def test_tensor_bound_kernel_at_burst_clocks():
+    # 2 TFLOP over 2.5 GB: 800 FLOP/B, above the 250 FLOP/B ridge
+    r = bench.roofline_record(2.0e12, 2.5e9, [1.25, 1.25], {"reasons": [], "sm_mhz": 1965, "sm_max_mhz": 1965},
+                              False, PEAKS)
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s" and r["peak"] == 1600.0
+    assert abs(r["achieved"] - 1600.0) < 1e-9 and abs(r["frac"] - 1.0) < 1e-12
+    assert abs(r["frac_of_sustained"] - 1600.0 / 1400.0) < 1e-12
+    assert r["launches_timed"] == 2 and r["avg_ms"] == 1.25
+
+
+def test_power_capped_run_is_held_to_the_sustained_peak():
+    clk = {"reasons": ["sw_power_cap"], "sm_mhz": 1965, "sm_max_mhz": 1965}
+    r = bench.roofline_record(2.0e12, 2.5e9, [1.25], clk, False, PEAKS)
+    assert r["peak"] == 1400.0 and "sustained" in r["peak_kind"]
+    # a clock stuck well below its maximum counts as capped as well
+    assert bench.power_capped({"reasons": [], "sm_mhz": 1500, "sm_max_mhz": 1965})
+    assert not bench.power_capped({"reasons": [], "sm_mhz": 1900, "sm_max_mhz": 1965})
+
+
+def test_e4m3_kernel_takes_twice_the_bf16_peak():
+    r = bench.roofline_record(4.0e12, 2.5e9, [1.25], None, True, PEAKS)
+    assert r["peak"] == 3200.0 and "x2" in r["peak_kind"]
+
+
+def test_decode_kernel_is_hbm_bound():
+    # 60 GFLOP over 7.7 GB: 7.8 FLOP/B, far below the ridge
+    r = bench.roofline_record(6.0e10, 7.7e9, [1.2], None, False, PEAKS)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["peak"] == 6400.0
+    assert abs(r["achieved"] - 7.7e9 / 1.2e-3 / 1e9) < 1e-6
+    assert abs(r["frac"] - r["achieved"] / 6400.0) < 1e-12
+
+
+def test_no_launches_gives_no_fraction():
+    r = bench.roofline_record(6.0e10, 7.7e9, [], None, False, PEAKS)
+    assert r["achieved"] is None and r["frac"] is None and r["launches_timed"] == 0
