@@ -44,6 +44,11 @@
  *     shared expert, block_m 128.
  *   - Weight scale arguments (void*): fp32 block scales for MOE_DTYPE_FP8_E4M3, prepared
  *     atoms for MOE_DTYPE_FP8_FP4, ignored (may be NULL) for MOE_DTYPE_BF16.
+ *   - Empty batch: T = 0 is valid.  After the parameter and workspace checks every call
+ *     returns MOE_OK, and arrays with a T or T*K dimension are not touched (they may be
+ *     NULL).  Outputs sized by E still describe the empty batch: moe_permute writes
+ *     counts (all 0), offsets_padded and, masked, pair_of_row (all -1);
+ *     moe_layer_forward zeroes counts_out when it is given.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H

@@ -400,17 +400,17 @@ moe_status_t moe_route(const moe_params_t* p, const void* x, const float* x_scal
                        void* stream) {
   MOE_TRY(validate(p));
   MOE_TRY(check_ws(p, ws, ws_bytes, false));
+  if (p->T == 0) return MOE_OK;  // empty batch: nothing to read or write
   if (!x || !w_r || !topk_ids || !topk_w || !aligned16(x) || !aligned16(w_r)) return MOE_ERR_INVALID_ARG;
   if (is_fp8(p) && !x_scale) return MOE_ERR_INVALID_ARG;
-  if (p->T == 0) return MOE_OK;
   return do_route(p, x, x_scale, w_r, bias, topk_ids, topk_w, ws, static_cast<cudaStream_t>(stream));
 }
 
 moe_status_t moe_grouped_topk(const moe_params_t* p, const float* logits, const float* bias,
                               int32_t* topk_ids, float* topk_w, void* stream) {
   MOE_TRY(validate(p));
-  if (!logits || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
   if (p->T == 0) return MOE_OK;
+  if (!logits || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
   return cuda_status(launch_topk(logits, *p, bias, topk_ids, topk_w, static_cast<cudaStream_t>(stream)));
 }
 
@@ -425,10 +425,13 @@ moe_status_t moe_permute(const moe_params_t* p, const int32_t* topk_ids, const v
                          void* x_perm, float* x_perm_scale, void* ws, size_t ws_bytes, void* stream) {
   MOE_TRY(validate(p));
   MOE_TRY(check_ws(p, ws, ws_bytes, false));
-  if (!topk_ids || !x || !counts || !offsets_padded || !row_of_pair || !pair_of_row || !x_perm)
+  // an empty batch still writes counts (all 0), offsets and, masked, pair_of_row (all -1);
+  // the [T,...] and [T*K] arrays are not touched and may be NULL
+  const bool empty = p->T == 0;
+  if ((!empty && (!topk_ids || !x || !row_of_pair)) || !counts || !offsets_padded || !pair_of_row || !x_perm)
     return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(x_perm)) return MOE_ERR_INVALID_ARG;
-  if (is_fp8(p) && (!x_scale || !x_perm_scale)) return MOE_ERR_INVALID_ARG;
+  if (is_fp8(p) && ((!empty && !x_scale) || !x_perm_scale)) return MOE_ERR_INVALID_ARG;
   return do_permute(p, topk_ids, x, x_scale, counts, offsets_padded, row_of_pair, pair_of_row, x_perm,
                     x_perm_scale, ws, static_cast<cudaStream_t>(stream));
 }
@@ -440,6 +443,7 @@ moe_status_t moe_expert_ffn(const moe_params_t* p, const void* x_perm, const flo
                             void* ws, size_t ws_bytes, void* stream) {
   MOE_TRY(validate(p));
   MOE_TRY(check_ws(p, ws, ws_bytes, false));
+  if (p->T == 0) return MOE_OK;
   if (!x_perm || !w_gate || !w_up || !w_down || !y_perm) return MOE_ERR_INVALID_ARG;
   if (p->masked_cap > 0 ? !counts : !offsets_padded) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x_perm) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down) || !aligned16(y_perm))
@@ -447,7 +451,6 @@ moe_status_t moe_expert_ffn(const moe_params_t* p, const void* x_perm, const flo
   if (is_fp8(p) && !x_perm_scale) return MOE_ERR_INVALID_ARG;
   if (!weight_scales_ok(p, w_gate_scale, w_up_scale, w_down_scale)) return MOE_ERR_INVALID_ARG;
   if (is_fp4(p) && !(aligned32(w_gate) && aligned32(w_up) && aligned32(w_down))) return MOE_ERR_INVALID_ARG;
-  if (p->T == 0) return MOE_OK;
   if (offsets_padded == nullptr) {  // masked layout: expert e's rows start at e*cap
     const Layout L = layout(p);
     int32_t* offs = at<int32_t>(ws, L.offsets);
@@ -468,16 +471,17 @@ moe_status_t moe_shared_expert_ffn(const moe_params_t* p, const void* x, const v
   MOE_TRY(validate(p));
   MOE_TRY(check_ws(p, ws, ws_bytes, false));
   if (p->I_shared <= 0 || is_fp8(p)) return MOE_ERR_UNSUPPORTED;
+  if (p->T == 0) return MOE_OK;
   if (!x || !ws_gate || !ws_up || !ws_down || !y_shared) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(ws_gate) || !aligned16(ws_up) || !aligned16(ws_down) || !aligned16(y_shared))
     return MOE_ERR_INVALID_ARG;
-  if (p->T == 0) return MOE_OK;
   return do_shared(p, x, ws_gate, ws_up, ws_down, y_shared, ws, static_cast<cudaStream_t>(stream));
 }
 
 moe_status_t moe_combine(const moe_params_t* p, const void* y_perm, const int32_t* row_of_pair,
                          const float* topk_w, const float* y_shared, void* out, void* stream) {
   MOE_TRY(validate(p));
+  if (p->T == 0) return MOE_OK;
   if (!y_perm || !row_of_pair || !topk_w || !out) return MOE_ERR_INVALID_ARG;
   if (!aligned16(y_perm) || !aligned16(out) || (y_shared && !aligned16(y_shared))) return MOE_ERR_INVALID_ARG;
   return cuda_status(launch_combine(*p, y_perm, row_of_pair, topk_w, y_shared, out,
@@ -492,6 +496,10 @@ moe_status_t moe_layer_forward(const moe_params_t* p, const void* x, const float
                                size_t ws_bytes, void* stream) {
   MOE_TRY(validate(p));
   MOE_TRY(check_ws(p, ws, ws_bytes, false));
+  if (p->T == 0)  // empty batch: no pairs, so the only output is an all-zero counts_out
+    return counts_out ? cuda_status(cudaMemsetAsync(counts_out, 0, static_cast<size_t>(p->E) * sizeof(int32_t),
+                                                    static_cast<cudaStream_t>(stream)))
+                      : MOE_OK;
   MOE_TRY(check_layer_args(p, x, x_scale, w_r, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, out));
   if (!weight_scales_ok(p, w_gate_scale, w_up_scale, w_down_scale)) return MOE_ERR_INVALID_ARG;
   return do_layer(p, x, x_scale, w_r, bias, w_gate, w_up, w_down, w_gate_scale, w_up_scale, w_down_scale,
@@ -507,6 +515,7 @@ moe_status_t moe_layer_forward_host(const moe_params_t* p, const void* x_host, c
                                     void* stream) {
   MOE_TRY(validate(p));
   MOE_TRY(check_ws(p, ws, ws_bytes, true));
+  if (p->T == 0) return MOE_OK;
   if (!x_host || !out_host) return MOE_ERR_INVALID_ARG;
   if (is_fp8(p) && !x_scale_host) return MOE_ERR_INVALID_ARG;
   if (!weight_scales_ok(p, w_gate_scale, w_up_scale, w_down_scale)) return MOE_ERR_INVALID_ARG;
@@ -515,7 +524,6 @@ moe_status_t moe_layer_forward_host(const moe_params_t* p, const void* x_host, c
   float* xs_dev = is_fp8(p) ? at<float>(ws, L.x_scale_stage) : nullptr;
   void* out_dev = at<void>(ws, L.out_stage);
   MOE_TRY(check_layer_args(p, x_dev, xs_dev, w_r, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, out_dev));
-  if (p->T == 0) return MOE_OK;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t xbytes = static_cast<size_t>(p->T) * p->H * (is_fp8(p) ? 1 : 2);
   MOE_CUDA(cudaMemcpyAsync(x_dev, x_host, xbytes, cudaMemcpyHostToDevice, st));

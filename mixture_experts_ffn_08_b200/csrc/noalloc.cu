@@ -65,10 +65,11 @@ extern "C" moe_status_t moe_permute_noalloc(const moe_params_t* p, const int32_t
                                             void* stream) {
   using namespace moe;
   if (moe_max_padded_rows(p) < 0) return MOE_ERR_INVALID_ARG;  // same parameter checks as moe_permute
-  if (!topk_ids || !x || !counts || !offsets_padded || !row_of_pair || !pair_of_row || !x_perm)
+  const bool empty = p->T == 0;  // same empty-batch rule as moe_permute
+  if ((!empty && (!topk_ids || !x || !row_of_pair)) || !counts || !offsets_padded || !pair_of_row || !x_perm)
     return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(x_perm)) return MOE_ERR_INVALID_ARG;
-  if (act_e4m3(*p) && (!x_scale || !x_perm_scale)) return MOE_ERR_INVALID_ARG;
+  if (act_e4m3(*p) && ((!empty && !x_scale) || !x_perm_scale)) return MOE_ERR_INVALID_ARG;
   const long long pairs = static_cast<long long>(p->T) * p->K;
   const long long chunks = (pairs + kPermChunk - 1) / kPermChunk;
   if ((chunks > 0 ? chunks : 1) * p->E > kNoAllocScratchInts) return MOE_ERR_UNSUPPORTED;

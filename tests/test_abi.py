@@ -118,3 +118,30 @@ def test_selftest_argument_errors_need_no_gpu(lib):
     assert lib.moe_selftest_bounded_wait(None, 50, None) == 1
     assert lib.moe_selftest_bounded_wait(ctypes.c_void_p(4096), 0, None) == 1       # limit too small
     assert lib.moe_selftest_bounded_wait(ctypes.c_void_p(4096 + 8), 50, None) == 1  # misaligned ws
+
+
+@pytest.mark.parametrize("dtype", [W.DTYPE_BF16, W.DTYPE_FP8])
+def test_empty_batch_returns_ok_without_touching_the_device(lib, dtype):
+    """T = 0: after the parameter and workspace checks every entry point returns MOE_OK,
+    with NULL for every array that has a T or T*K dimension.  None of these calls issues
+    a CUDA call (no counts_out given), so they run without a GPU."""
+    wl = W.DSV3_PREFILL.with_(name="empty", T=0, dtype=dtype,
+                              I_shared=W.DSV3_PREFILL.I_shared if dtype == W.DTYPE_BF16 else 0)
+    p = B.params(wl)
+    size, size_host = B.moe_workspace_size(p), lib.moe_workspace_size_host(ctypes.byref(p))
+    assert size > 0 and size_host >= size
+    ws = 4096  # never dereferenced
+    pp = ctypes.byref(p)
+    assert lib.moe_route(pp, None, None, None, None, None, None, ws, size, None) == 0
+    assert lib.moe_grouped_topk(pp, None, None, None, None, None) == 0
+    assert lib.moe_expert_ffn(pp, *([None] * 11), ws, size, None) == 0
+    assert lib.moe_combine(pp, None, None, None, None, None, None) == 0
+    assert lib.moe_layer_forward(pp, *([None] * 17), ws, size, None) == 0
+    assert lib.moe_layer_forward_host(pp, *([None] * 14), ws, size_host, None) == 0
+    if wl.I_shared > 0:
+        assert lib.moe_shared_expert_ffn(pp, None, None, None, None, None, ws, size, None) == 0
+    # the parameter and workspace checks still come first
+    assert lib.moe_route(pp, None, None, None, None, None, None, ws, size - 1, None) == 1
+    assert lib.moe_layer_forward(pp, *([None] * 17), ws + 8, size, None) == 1
+    bad = B.params(wl.with_(H=100))
+    assert lib.moe_combine(ctypes.byref(bad), None, None, None, None, None, None) == 2

@@ -122,6 +122,36 @@ def test_permute_bucket_edge_sizes():
     assert r["counts"].tolist() == sizes
 
 
+@pytest.mark.parametrize("cap", [0, 256])
+def test_permute_empty_batch(cap):
+    """T = 0: no pairs.  counts are all 0, offsets 0 (contiguous) or e*cap (masked),
+    every masked row is marked unused, and x_perm is left as it was."""
+    wl = W.Workload("empty", T=0, H=256, I=128, E=8, K=2, masked_cap=cap)
+    r = _permute(wl, np.zeros((0, wl.K), dtype=np.int32))
+    assert B.moe_get_device_status(r["ws"]) == 0
+    assert r["counts"].tolist() == [0] * wl.E
+    assert r["offs"].tolist() == [e * cap for e in range(wl.E + 1)]
+    assert (r["por"] == (-1 if cap else 12345)).all()
+    assert (r["xp"] == 7.0).all()
+
+
+def test_layer_empty_batch_zeroes_counts():
+    wl = W.DSV3_PREFILL.with_(name="empty_layer", T=0, H=512, I=256, E=32, I_shared=256)
+    d = inputs.make_inputs(wl, seed=0, device="cuda")
+    p = B.params(wl)
+    ws = _ws(wl)
+    a = P.device_inputs_ptrs(d, wl)
+    counts = torch.full((wl.E,), 77, dtype=torch.int32, device="cuda")
+    out = torch.empty((0, wl.H), dtype=torch.bfloat16, device="cuda")
+    B.check(B.moe_layer_forward(p, a["x"], a["x_scale"], a["w_r"], a["bias"], a["w_gate"], a["w_up"],
+                                a["w_down"], a["w_gate_scale"], a["w_up_scale"], a["w_down_scale"],
+                                a["ws_gate"], a["ws_up"], a["ws_down"], out, None, None, counts, ws,
+                                ws.numel()))
+    torch.cuda.synchronize()
+    assert counts.tolist() == [0] * wl.E
+    assert B.moe_get_device_status(ws) == 0
+
+
 def test_permute_page_bucket_example():
     from tests.conftest import load_golden
     g = load_golden("bucket_example.txt")
