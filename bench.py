@@ -41,6 +41,17 @@ FLUSH_BYTES = 512 << 20
 
 GEMM_SOURCES = ("csrc/tc_gemm.cuh", "csrc/common.cuh", "csrc/gemm.cu")
 FP8_GEMM_SOURCES = ("csrc/tc_gemm_fp8.cuh", "csrc/tc_gemm.cuh", "csrc/common.cuh", "csrc/gemm_fp8.cu")
+SWAP_GEMM_SOURCES = ("csrc/tc_gemm_swap.cuh", "csrc/tc_gemm_fp8.cuh", "csrc/tc_gemm.cuh", "csrc/common.cuh",
+                     "csrc/gemm_swap.cu")
+
+
+def gateup_sources(wl):
+    """Source files of the gate/up kernel the library runs for this workload: swap-A/B tiles
+    for FP8 x FP4 layers with at most 32 pairs per expert on average (the library's rule),
+    the block-scaled M-tile GEMM for other FP8 layers, the bf16 GEMM otherwise."""
+    if wl.dtype == W.DTYPE_FP8_FP4 and wl.T * wl.K <= 32 * wl.E:
+        return SWAP_GEMM_SOURCES
+    return FP8_GEMM_SOURCES if wl.dtype in (W.DTYPE_FP8, W.DTYPE_FP8_FP4) else GEMM_SOURCES
 
 
 def sources_sha256(files):
@@ -53,10 +64,11 @@ def sources_sha256(files):
     return h.hexdigest()
 
 
-def _profiled_traffic(workload):
+def _profiled_traffic(workload, sources=GEMM_SOURCES):
     """DRAM bytes per launch of the gate/up kernel from the committed ncu summary of this
-    workload, or None if there is none or the kernel sources changed since it was taken.
-    The summary names the sources it covers (kernel_sources:, default the bf16 GEMM)."""
+    workload, or None if there is none, it covers another kernel than `sources` (the
+    files of the kernel that runs now), or those sources changed since it was taken.  The
+    summary names the sources it covers (kernel_sources:, default the bf16 GEMM)."""
     import re
     path = os.path.join(ROOT, "profiles", f"gateup_swiglu_{workload}.md")
     if not os.path.exists(path):
@@ -68,6 +80,8 @@ def _profiled_traffic(workload):
     if not (m_t and m_h):
         return None
     files = [f.strip() for f in m_s.group(1).split(",")] if m_s else list(GEMM_SOURCES)
+    if files != list(sources):
+        return None
     return int(m_t.group(1)) if sources_sha256(files) == m_h.group(1) else None
 
 
@@ -379,10 +393,12 @@ def run_ours(args):
     layer_bytes = (active * 3 * wl.I * wl.H * wbytes + 3 * wl.I_shared * wl.H * 2 + wl.E * wl.H * 2
                    + wl.T * wl.H * (abytes + 2))
     dt_name = "e4m3 x e2m1" if w4 else ("e4m3" if fp8 else "bf16")
+    swap = gateup_sources(wl) == SWAP_GEMM_SOURCES
     dom_ms = [ms for k, ms in traced if k == dominant]
     roofline = roofline_record(flops_gateup, bytes_gateup, dom_ms, clk, fp8, _peaks())
-    roofline.update({"kernel": f"gateup_swiglu (grouped GEMM, fused SwiGLU, {dt_name})",
-                     "traffic": _profiled_traffic(wl.name)})
+    roofline.update({"kernel": (f"gateup_swiglu ({'swap-A/B ' if swap else ''}grouped GEMM, fused SwiGLU, "
+                                f"{dt_name})"),
+                     "traffic": _profiled_traffic(wl.name, gateup_sources(wl))})
 
     # ---------------- end to end: host activations in, host output out
     x_host = (d["x_q"] if fp8 else d["x"]).cpu().pin_memory()

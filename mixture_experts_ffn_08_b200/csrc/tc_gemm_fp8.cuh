@@ -147,9 +147,12 @@ struct Fp8Cfg {
   static_assert(EPI != EPI8_SWIGLU_Q || BN == 256, "SwiGLU tile = 128 gate + 128 up rows");
 };
 
-// Smallest e with amax <= 448 * 2^e (e = 0 when amax == 0), exactly in fp32.
+// Smallest e with amax <= 448 * 2^e (e = 0 when amax == 0), exactly in fp32.  A row with
+// no finite maximum (pad rows of the masked layout hold whatever the workspace held) gets
+// the largest exponent at once: the search below would otherwise walk down from ilogb(inf).
 MOE_DEVINL int e4m3_scale_exponent(float amax) {
   if (!(amax > 0.f)) return 0;
+  if (isinf(amax)) return 127;
   int e = ilogbf(amax) - 8;
   while (amax > ldexpf(448.f, e)) ++e;
   while (e > -126 && amax <= ldexpf(448.f, e - 1)) --e;

@@ -40,3 +40,28 @@ def test_decode_kernel_is_hbm_bound():
 def test_no_launches_gives_no_fraction():
     r = bench.roofline_record(6.0e10, 7.7e9, [], None, False, PEAKS)
     assert r["achieved"] is None and r["frac"] is None and r["launches_timed"] == 0
+
+
+def test_gate_up_kernel_sources_follow_the_library_rule():
+    from mixture_experts_ffn_08_b200 import workloads as W
+    assert bench.gateup_sources(W.MIXTRAL_PREFILL) == bench.GEMM_SOURCES
+    assert bench.gateup_sources(W.SKEWED_FP8) == bench.FP8_GEMM_SOURCES
+    assert bench.gateup_sources(W.FP4["dsv3_prefill_fp4"]) == bench.FP8_GEMM_SOURCES
+    assert bench.gateup_sources(W.FP4["dsv3_decode_fp4"]) == bench.SWAP_GEMM_SOURCES
+
+
+def test_profiled_traffic_only_for_the_kernel_it_covers(tmp_path, monkeypatch):
+    (tmp_path / "profiles").mkdir()
+    pkg = tmp_path / "mixture_experts_ffn_08_b200" / "csrc"
+    pkg.mkdir(parents=True)
+    for f in ("a.cuh", "b.cu"):
+        (pkg / f).write_text(f"// {f}\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    sha = bench.sources_sha256(["csrc/a.cuh", "csrc/b.cu"])
+    (tmp_path / "profiles" / "gateup_swiglu_w.md").write_text(
+        f"traffic_bytes_per_launch: 1234\nkernel_sources: csrc/a.cuh, csrc/b.cu\nkernel_source_sha256: {sha}\n")
+    assert bench._profiled_traffic("w", ("csrc/a.cuh", "csrc/b.cu")) == 1234
+    assert bench._profiled_traffic("w", ("csrc/a.cuh",)) is None          # another kernel runs now
+    (pkg / "b.cu").write_text("// changed\n")
+    assert bench._profiled_traffic("w", ("csrc/a.cuh", "csrc/b.cu")) is None  # sources changed
+    assert bench._profiled_traffic("none", ("csrc/a.cuh",)) is None
