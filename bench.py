@@ -41,16 +41,11 @@ FLUSH_BYTES = 512 << 20
 
 GEMM_SOURCES = ("csrc/tc_gemm.cuh", "csrc/common.cuh", "csrc/gemm.cu")
 FP8_GEMM_SOURCES = ("csrc/tc_gemm_fp8.cuh", "csrc/tc_gemm.cuh", "csrc/common.cuh", "csrc/gemm_fp8.cu")
-SWAP_GEMM_SOURCES = ("csrc/tc_gemm_swap.cuh", "csrc/tc_gemm_fp8.cuh", "csrc/tc_gemm.cuh", "csrc/common.cuh",
-                     "csrc/gemm_swap.cu")
 
 
 def gateup_sources(wl):
-    """Source files of the gate/up kernel the library runs for this workload: swap-A/B tiles
-    for FP8 x FP4 layers with at most 32 pairs per expert on average (the library's rule),
-    the block-scaled M-tile GEMM for other FP8 layers, the bf16 GEMM otherwise."""
-    if wl.dtype == W.DTYPE_FP8_FP4 and wl.T * wl.K <= 32 * wl.E:
-        return SWAP_GEMM_SOURCES
+    """Source files of the gate/up kernel the library runs for this workload: the
+    block-scaled GEMM for e4m3 activations, the bf16 GEMM otherwise."""
     return FP8_GEMM_SOURCES if wl.dtype in (W.DTYPE_FP8, W.DTYPE_FP8_FP4) else GEMM_SOURCES
 
 
@@ -393,11 +388,9 @@ def run_ours(args):
     layer_bytes = (active * 3 * wl.I * wl.H * wbytes + 3 * wl.I_shared * wl.H * 2 + wl.E * wl.H * 2
                    + wl.T * wl.H * (abytes + 2))
     dt_name = "e4m3 x e2m1" if w4 else ("e4m3" if fp8 else "bf16")
-    swap = gateup_sources(wl) == SWAP_GEMM_SOURCES
     dom_ms = [ms for k, ms in traced if k == dominant]
     roofline = roofline_record(flops_gateup, bytes_gateup, dom_ms, clk, fp8, _peaks())
-    roofline.update({"kernel": (f"gateup_swiglu ({'swap-A/B ' if swap else ''}grouped GEMM, fused SwiGLU, "
-                                f"{dt_name})"),
+    roofline.update({"kernel": f"gateup_swiglu (grouped GEMM, fused SwiGLU, {dt_name})",
                      "traffic": _profiled_traffic(wl.name, gateup_sources(wl))})
 
     # ---------------- end to end: host activations in, host output out

@@ -64,7 +64,7 @@ size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 struct Layout {
   size_t status, logits, xb, ids, w, counts, offsets, sched, row_of_pair, pair_of_row, chunk_counts;
   size_t x_perm, x_perm_scale, h, y_perm, h_sh, y_sh, total;
-  size_t x_atoms, h_atoms, wg_atoms, wu_atoms, wd_atoms, tsched, tok_atoms;
+  size_t x_atoms, h_atoms, wg_atoms, wu_atoms, wd_atoms;
   size_t x_stage, x_scale_stage, out_stage, total_host;
   long long max_rows;
 };
@@ -73,11 +73,6 @@ struct Layout {
 bool is_fp8(const moe_params_t* p) { return p->dtype == MOE_DTYPE_FP8_E4M3 || p->dtype == MOE_DTYPE_FP8_FP4; }
 // e2m1 expert weights whose scale atoms the caller prepared (moe_prepare_fp4_scales)
 bool is_fp4(const moe_params_t* p) { return p->dtype == MOE_DTYPE_FP8_FP4; }
-// Decode-sized FP8 x FP4 layers (at most 32 pairs per expert on average) run gate/up with
-// swap-A/B tiles: the weights as the 128-row M operand, 32-token tiles as N.
-bool use_swap(const moe_params_t* p) {
-  return is_fp4(p) && static_cast<long long>(p->T) * p->K <= 32LL * p->E;
-}
 
 // Bucket alignment: 128 rows (one-SM GEMM tiles) unless the caller asks for 256 (two-SM
 // cta_group::2 tiles).  Measured on B200, the pair tiles' third less SM-side traffic did
@@ -123,9 +118,6 @@ Layout layout(const moe_params_t* p) {
   L.wg_atoms = take(w8 ? E * (I / 128) * hk4 * 512 : 0);
   L.wu_atoms = take(w8 ? E * (I / 128) * hk4 * 512 : 0);
   L.wd_atoms = take(w8 ? E * (H / 128) * ik4 * 512 : 0);
-  const bool swap = use_swap(p);  // token-tile schedule and the tokens' padded scale atoms
-  L.tsched = take(swap ? (E + 1) * 4 : 0);
-  L.tok_atoms = take(swap ? swap_max_token_tiles(P, p->E) * hk4 * 512 : 0);
   L.total = o;
   L.x_stage = take(T * H * xelem);
   L.x_scale_stage = take(is_fp8(p) ? T * (H / 128) * 4 : 0);
@@ -255,20 +247,9 @@ moe_status_t do_expert_ffn_fp8(const moe_params_t* p, const void* x_perm, const 
     wu_atoms = at<uint8_t>(ws, L.wu_atoms);
     wd_atoms = at<uint8_t>(ws, L.wd_atoms);
   }
-  void* h = at<void>(ws, L.h);
-  if (use_swap(p) && counts != nullptr) {
-    // few tokens per expert: gate/up with the weights as M and 32-token tiles as N; it
-    // writes h and its scale atoms exactly as the M-tile kernel does, for the down GEMM
-    MOE_CUDA(gemm_gateup_swiglu_swap(x_perm, x_perm_scale, L.max_rows, offsets, counts, p->E,
-                                     swap_max_token_tiles(static_cast<long long>(p->T) * p->K, p->E), w_gate,
-                                     w_up, wg_atoms, wu_atoms, p->I, p->H, h, at<uint8_t>(ws, L.h_atoms),
-                                     at<int32_t>(ws, L.tsched), at<uint8_t>(ws, L.tok_atoms), status, st));
-    MOE_CUDA(gemm_down_fp8(h, at<uint8_t>(ws, L.h_atoms), L.max_rows, sched, counts, p->E, w_down, wd_atoms,
-                           p->H, p->I, y_perm, status, st, cap, w4));
-    return MOE_OK;
-  }
   MOE_CUDA(launch_sf_rows_to_atoms(x_perm_scale, p->H / 128, offsets, p->E, L.max_rows,
                                    at<uint8_t>(ws, L.x_atoms), st));
+  void* h = at<void>(ws, L.h);
   if (block_m_of(p) == kBlockM2) {
     MOE_CUDA(gemm_pair_gateup_swiglu_fp8(x_perm, at<uint8_t>(ws, L.x_atoms), L.max_rows, offsets, counts, p->E,
                                          w_gate, w_up, wg_atoms, wu_atoms,
@@ -637,9 +618,8 @@ int32_t moe_layer_launch_count(const moe_params_t* p) {
   if (validate(p) != MOE_OK) return -1;
   if (p->T == 0) return 0;
   int n = 2;                                 // router GEMM, top-k
-  if (is_fp8(p)) n += is_fp4(p) ? (use_swap(p) ? 3 : 2) : 5;  // dequantise x for the router;
-                                             // scale atoms of x (and of the three e4m3 weights),
-                                             // or the token-tile schedule and token atoms (swap-A/B)
+  if (is_fp8(p)) n += is_fp4(p) ? 2 : 5;     // dequantise x for the router; scale atoms of x
+                                             // (and of the three e4m3 weights)
   n += (p->T * p->K > 0) ? 4 : 2;            // count, scan, rank, gather
   n += 2;                                    // gate/up, down
   if (p->I_shared > 0) n += 2;               // shared gate/up, down

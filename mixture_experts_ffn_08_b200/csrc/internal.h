@@ -101,20 +101,6 @@ cudaError_t gemm_down_fp8(const void* A, const uint8_t* a_atoms, int64_t a_rows,
 // e2m1 weight scale words [rows, K/128] (4 UE8M0 bytes each) -> atoms [rows/128][K/128][512].
 cudaError_t launch_fp4_scale_atoms(const uint32_t* words, long long rows, int K, uint8_t* atoms, cudaStream_t st);
 
-// ---------------------------------------------------------------- swap-A/B gate/up (gemm_swap.cu)
-// Upper bound on the 32-token tiles of `pairs` pairs over E experts: ceil(pairs/32) + E.
-long long swap_max_token_tiles(long long pairs, int E);
-// h (e4m3 [rows, N] + scale atoms, as gemm_gateup_swiglu_fp8 writes them) for e2m1 weights
-// with the weights as the 128-row M operand and each expert's tokens, 32 at a time, as N.
-// offsets: first bucket row of each expert (contiguous offsets, or e*cap); counts required;
-// tsched [G+1] and tok_atoms [max_tiles][ceil(K/512)][512] are scratch.
-cudaError_t gemm_gateup_swiglu_swap(const void* x_perm, const float* x_scale, int64_t x_rows,
-                                    const int32_t* offsets, const int32_t* counts, int G,
-                                    long long max_tiles, const void* w_gate, const void* w_up,
-                                    const uint8_t* gate_atoms, const uint8_t* up_atoms, int N, int K,
-                                    void* h, uint8_t* h_atoms, int32_t* tsched, uint8_t* tok_atoms,
-                                    int32_t* status, cudaStream_t st);
-
 // ---------------------------------------------------------------- two-SM GEMMs (gemm_2cta.cu)
 cudaError_t gemm_pair_gateup_swiglu(const void* A, int64_t a_rows, const int32_t* offsets, const int32_t* counts,
                                     int G, const void* w_gate, const void* w_up, int N, int K, void* h,

@@ -147,11 +147,8 @@ def test_empty_batch_returns_ok_without_touching_the_device(lib, dtype):
     assert lib.moe_combine(ctypes.byref(bad), None, None, None, None, None, None) == 2
 
 
-def test_fp4_launch_counts_follow_the_gate_up_tiling(lib):
-    """FP8 x FP4 layers with at most 32 pairs per expert on average use swap-A/B gate/up
-    tiles (token-tile schedule + token scale atoms); larger ones the 128-row M-tiles
-    (token scale atoms of x).  Both dequantise x for the router."""
-    dec, pre = W.FP4["dsv3_decode_fp4"], W.FP4["dsv3_prefill_fp4"]
-    assert dec.T * dec.K <= 32 * dec.E < pre.T * pre.K
-    assert B.moe_layer_launch_count(B.params(dec)) == 9 + 3
-    assert B.moe_layer_launch_count(B.params(pre)) == 9 + 2
+def test_fp4_launch_counts(lib):
+    """FP8 x FP4 layers add two launches to the bf16 layer's nine: x dequantised for the
+    router and the scale atoms of x (the weights bring theirs)."""
+    for wl in W.FP4.values():
+        assert B.moe_layer_launch_count(B.params(wl)) == 9 + 2

@@ -47,7 +47,7 @@ def test_gate_up_kernel_sources_follow_the_library_rule():
     assert bench.gateup_sources(W.MIXTRAL_PREFILL) == bench.GEMM_SOURCES
     assert bench.gateup_sources(W.SKEWED_FP8) == bench.FP8_GEMM_SOURCES
     assert bench.gateup_sources(W.FP4["dsv3_prefill_fp4"]) == bench.FP8_GEMM_SOURCES
-    assert bench.gateup_sources(W.FP4["dsv3_decode_fp4"]) == bench.SWAP_GEMM_SOURCES
+    assert bench.gateup_sources(W.FP4["dsv3_decode_fp4"]) == bench.FP8_GEMM_SOURCES
 
 
 def test_profiled_traffic_only_for_the_kernel_it_covers(tmp_path, monkeypatch):

@@ -137,9 +137,9 @@ def test_fp4_layer_full_size_decode_sampled():
     P.check_close(got, ref, P.FP8_MAX_TOL, wl.name)
 
 
-# ---------------------------------------------------------------- swap-A/B gate/up
-# Layers with at most 32 pairs per expert on average (T*K <= 32*E) run the FP8 x FP4 gate/up
-# with the weights as the 128-row M operand and each expert's tokens, 32 at a time, as N.
+# ---------------------------------------------------------------- few tokens per expert
+# Decode-like shapes (at most 32 pairs per expert on average): M-tiles that are mostly pad
+# rows, experts with no token, and buckets of one or two partial 32-row groups.
 
 def _ids_from_counts(counts, seed):
     ids = np.concatenate([np.full(n, e) for e, n in enumerate(counts)]).astype(np.int32)
@@ -148,21 +148,19 @@ def _ids_from_counts(counts, seed):
 
 
 @pytest.mark.parametrize("E,K,T,H,I", [(32, 4, 64, 512, 384), (16, 2, 200, 256, 256), (64, 6, 100, 1024, 768)])
-def test_fp4_swap_expert_ffn(E, K, T, H, I):
+def test_fp4_few_tokens_expert_ffn(E, K, T, H, I):
     wl = W.Workload("f4s", T=T, H=H, I=I, E=E, K=K, dtype=W.DTYPE_FP8_FP4)
-    assert T * K <= 32 * E  # the swap-A/B shape
     d = inputs.make_inputs(wl, seed=8, device="cuda")
     ids = _ids(wl, 8)
     r, y = _expert_ffn(wl, d, ids)
     _check_ffn(wl, d, ids, r, y)
 
 
-def test_fp4_swap_token_tile_edges():
-    """Experts with 0, 1, 31, 32, 33, 64 and 65 tokens: empty experts, a partial tile,
-    exactly one and two full tiles, and a tile with one token past them."""
+def test_fp4_bucket_edges():
+    """Experts with 0, 1, 31, 32, 33, 64 and 65 tokens: empty buckets and buckets just
+    under, at and over multiples of 32 rows inside one 128-row M-tile."""
     counts = [0, 1, 31, 32, 33, 64, 65, 0]
     wl = W.Workload("f4e", T=sum(counts), H=256, I=256, E=len(counts), K=1, dtype=W.DTYPE_FP8_FP4)
-    assert wl.T * wl.K <= 32 * wl.E
     d = inputs.make_inputs(wl, seed=9, device="cuda")
     ids = _ids_from_counts(counts, 9)
     r, y = _expert_ffn(wl, d, ids)
@@ -171,9 +169,8 @@ def test_fp4_swap_token_tile_edges():
 
 
 @pytest.mark.parametrize("masked", [False, True])
-def test_fp4_swap_layer_small_all_elements(masked):
-    wl = SMALL_FP4.with_(name="dsv3_fp4_swap_small", T=100, masked_cap=128 if masked else 0)
-    assert wl.T * wl.K <= 32 * wl.E
+def test_fp4_decode_like_layer_small_all_elements(masked):
+    wl = SMALL_FP4.with_(name="dsv3_fp4_decode_small", T=100, masked_cap=128 if masked else 0)
     d = inputs.make_inputs(wl, seed=10, device="cuda")
     res = P.run_layer(wl, d)
     assert B.moe_get_device_status(res["ws"]) == 0
