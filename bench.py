@@ -176,10 +176,44 @@ def _dist():
 
 
 # ------------------------------------------------------------------ clocks
+def _is_num(v):
+    return v.replace(".", "", 1).isdigit()
+
+
+def summarize_clock_rows(lines, window=None):
+    """Summary of nvidia-smi samples (ClockSampler.FIELDS, csv, noheader, nounits): median SM
+    clock under load, maximum SM clock, and the throttle reasons seen.  It is taken over the
+    samples whose timestamps fall inside window = (t0, t1), host time.time() values around
+    the timed region, or over all samples when none does (a region shorter than the
+    sampling interval); samples_in_window says which."""
+    from datetime import datetime
+    rows = []
+    for line in lines:
+        r = [c.strip() for c in line.split(",")]
+        if len(r) < 10:
+            continue
+        try:
+            ts = datetime.strptime(r[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+        except ValueError:
+            ts = None
+        rows.append((ts, r))
+    inside = [r for ts, r in rows if window and ts is not None and window[0] <= ts <= window[1]]
+    use = inside or [r for _, r in rows]
+    sm = [float(r[2]) for r in use if _is_num(r[2])]
+    smax = [float(r[3]) for _, r in rows if _is_num(r[3])]
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    reasons = sorted({names[i] for r in use for i in range(4) if r[6 + i] == "Active"})
+    loaded = [v for v in sm if smax and v > 0.5 * max(smax)] or sm
+    return {"sm_mhz": statistics.median(loaded) if loaded else None,
+            "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+            "samples": len(rows), "samples_in_window": len(inside)}
+
+
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    INTERVAL_MS = 50
 
     def __init__(self, device):
         self.proc = None
@@ -191,27 +225,20 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", self.uuid, f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", str(self.INTERVAL_MS)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
         time.sleep(0.3)
 
-    def stop(self):
+    def stop(self, window=None):
+        """window: (t0, t1) host time.time() values around the timed region."""
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         time.sleep(0.3)
         self.proc.terminate()
         out, _ = self.proc.communicate(timeout=10)
-        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8]
-        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
-        smax = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip() == "Active"})
-        loaded = [v for v in sm if smax and v > 0.5 * max(smax)] or sm
-        return {"sm_mhz": statistics.median(loaded) if loaded else None,
-                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
-                "samples": len(rows)}
+        return summarize_clock_rows(out.strip().splitlines(), window)
 
 
 # ------------------------------------------------------------------ CPU oracle leg
@@ -344,16 +371,18 @@ def run_ours(args):
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
     barrier()
+    t_region = time.time()
     for i in range(args.steps):
         flush.fill_(i & 0xFF)
         ev[i][0].record(stream)
         step()
         ev[i][1].record(stream)
     barrier()
+    t_region = (t_region, time.time())
     step_ms = [s.elapsed_time(e) for s, e in ev]
     traced = B.moe_trace_collect()
     B.moe_trace_disable()
-    clk = clocks.stop() if clocks else None
+    clk = clocks.stop(t_region) if clocks else None
     status = B.moe_get_device_status(ws)
     if status != 0:
         raise B.MoEError(f"device status {status:#x} after the timed steps")

@@ -65,3 +65,30 @@ def test_profiled_traffic_only_for_the_kernel_it_covers(tmp_path, monkeypatch):
     (pkg / "b.cu").write_text("// changed\n")
     assert bench._profiled_traffic("w", ("csrc/a.cuh", "csrc/b.cu")) is None  # sources changed
     assert bench._profiled_traffic("none", ("csrc/a.cuh",)) is None
+
+
+def _smi_line(ts, sm, reason_cap="Not Active", smax=1965):
+    # ClockSampler.FIELDS order: timestamp, index, clocks.sm, clocks.max.sm, power.draw,
+    # reasons.active, hw_slowdown, hw_thermal_slowdown, sw_thermal_slowdown, sw_power_cap
+    return f"{ts}, 0, {sm}, {smax}, 900.5, 0x0000000000000004, Not Active, Not Active, Not Active, {reason_cap}"
+
+
+def test_clock_summary_uses_the_samples_inside_the_timed_window():
+    from datetime import datetime
+    t = lambda s: datetime.strptime(s, "%Y/%m/%d %H:%M:%S.%f").timestamp()
+    lines = [_smi_line("2026/12/02 10:00:00.000", 1965),                      # idle, before
+             _smi_line("2026/12/02 10:00:00.250", 1372, "Active"),            # timed region
+             _smi_line("2026/12/02 10:00:00.300", 1380, "Active"),
+             _smi_line("2026/12/02 10:00:00.350", 1390, "Active"),
+             _smi_line("2026/12/02 10:00:00.700", 1965),                      # idle, after
+             "garbage line"]
+    win = (t("2026/12/02 10:00:00.200"), t("2026/12/02 10:00:00.400"))
+    c = bench.summarize_clock_rows(lines, win)
+    assert c["sm_mhz"] == 1380 and c["sm_max_mhz"] == 1965 and c["reasons"] == ["sw_power_cap"]
+    assert c["samples"] == 5 and c["samples_in_window"] == 3
+    assert bench.power_capped(c)
+    # a region shorter than the sampling interval: all samples, flagged as such
+    short = (t("2026/12/02 10:00:00.400"), t("2026/12/02 10:00:00.450"))
+    c = bench.summarize_clock_rows(lines, short)
+    assert c["samples_in_window"] == 0 and c["samples"] == 5 and c["sm_mhz"] == 1390
+    assert bench.summarize_clock_rows([], None)["sm_mhz"] is None
