@@ -372,8 +372,9 @@ def forward_given_routing(x, ids, w, expert_weights, E: int, shared=None,
 
 
 def activation_format(dtype: int):
-    """Storage format of h for a workload dtype (0 = bf16, 1 = FP8 e4m3)."""
-    return "e4m3" if dtype == 1 else "bf16"
+    """Storage format of h for a workload dtype: 0 = bf16; 1 (FP8) and 2 (FP8 x FP4, whose
+    FP4 operand is the weights) have e4m3 activations, so h is e4m3 with 1x128 scales."""
+    return "e4m3" if dtype in (1, 2) else "bf16"
 
 
 def layer_forward(x, w_r, bias, expert_weights, wl, shared=None, h_format="auto"):

@@ -179,7 +179,35 @@ def _masked_keeps_last(ids, E, cap):
             por.astype(np.int32), int(np.maximum(n - cap, 0).sum()))
 
 
+def _route_groups_on_unbiased(s, K, bias=None, n_group=1, topk_group=1, group_topn=1, renormalize=True,
+                              routed_scale=1.0):
+    s = np.asarray(s, np.float64)
+    T, E = s.shape
+    c = s + (np.asarray(bias, np.float64)[None, :] if bias is not None else 0.0)
+    ids = np.empty((T, K), dtype=np.int32)
+    w = np.empty((T, K))
+    for t in range(T):
+        cc = c[t].copy()
+        if n_group > 1:
+            gs = E // n_group
+            g = np.sort(s[t].reshape(n_group, gs), axis=1)[:, ::-1][:, :group_topn].sum(axis=1)  # unbiased s
+            allowed = np.zeros(E, dtype=bool)
+            for j in np.argsort(-g, kind="stable")[:topk_group]:
+                allowed[j * gs:(j + 1) * gs] = True
+            cc = np.where(allowed, cc, -np.inf)
+        ids[t] = np.argsort(-cc, kind="stable")[:K]
+        wt = s[t, ids[t]]
+        w[t] = (wt / wt.sum() if renormalize else wt) * routed_scale
+    return ids, w
+
+
+def _dequant_scales_transposed(codes, scales, rows_per_block):
+    sc = np.asarray(scales, np.float64)
+    return _dequant_blocks_orig(codes, sc.T if sc.shape[0] == sc.shape[1] else sc, rows_per_block)
+
+
 _select_orig = o.select_experts
+_dequant_blocks_orig = o.dequant_blocks
 _permute_orig = o.permute
 _combine_orig = o.combine
 _e2m1_orig = o.decode_e2m1
@@ -201,6 +229,8 @@ MUTATIONS = {
     "e2m1 nibbles swapped": ("dequant_fp4", _fp4_nibbles_swapped),
     "bf16 rounding truncates": ("round_bf16", _bf16_truncate),
     "masked layout keeps the last pairs": ("permute_masked", _masked_keeps_last),
+    "groups ranked on the unbiased scores": ("route_from_scores", _route_groups_on_unbiased),
+    "128x128 block scales transposed": ("dequant_blocks", _dequant_scales_transposed),
 }
 
 

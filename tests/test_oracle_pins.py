@@ -205,6 +205,21 @@ def test_bias_only_chooses_and_scale_applies_after_renorm():
     np.testing.assert_allclose(w[0], [2.5 * 0.2 / 0.7, 2.5 * 0.5 / 0.7], rtol=1e-14)
 
 
+def test_group_stage_ranks_groups_by_the_biased_scores():
+    """The selection-only bias steers every selection step, the group stage included:
+    groups are ranked on c = s + b.  Worked by hand on 4 experts in 2 groups, one group
+    kept, group score = group maximum, K = 1.  s = [.5, .1, .45, .2], b = [0, 0, .1, 0]:
+    biased group maxima are .5 and .55, so group {2, 3} stays and expert 2 (c = .55) wins.
+    Ranking the groups on s instead (.5 and .45) would keep group {0, 1} and pick expert 0.
+    The weight comes from the unbiased score and renormalises to the routed scale."""
+    s = np.array([[0.5, 0.1, 0.45, 0.2]])
+    b = np.array([0.0, 0.0, 0.1, 0.0])
+    ids, w = o.route_from_scores(s, 1, b, n_group=2, topk_group=1, group_topn=1, routed_scale=2.5)
+    assert ids.tolist() == [[2]] and w[0, 0] == pytest.approx(2.5)
+    ids, _ = o.route_from_scores(s, 1, None, n_group=2, topk_group=1, group_topn=1)
+    assert ids.tolist() == [[0]]  # without the bias the other group wins
+
+
 def test_weights_sum_to_routed_scale():
     rng = np.random.default_rng(4)
     s = scipy.special.expit(rng.normal(size=(30, 64)))
@@ -352,6 +367,31 @@ def test_e4m3_quantize_is_nearest_even_by_search():
     inr = np.abs(v) < 448
     tq = torch.from_numpy(v[inr]).to(torch.float32).to(torch.float8_e4m3fn).to(torch.float64).numpy()
     np.testing.assert_array_equal(np.abs(q[inr]), np.abs(tq))
+
+
+def test_block_dequant_of_constant_codes_is_the_scale_grid():
+    """Codes that all decode to 1.0 dequantise to the block-scale grid itself: element
+    (r, c) takes scales[r // 128, c // 128].  A non-symmetric 2 x 2 grid tells rows from
+    columns."""
+    codes = np.full((256, 256), 0x38, dtype=np.uint8)  # e4m3 1.0
+    assert o.decode_e4m3(np.array([0x38]))[0] == 1.0
+    scales = np.array([[1.0, 2.0], [4.0, 8.0]])
+    got = o.dequant_blocks(codes, scales, 128)
+    assert got[0, 0] == 1.0 and got[0, 255] == 2.0 and got[255, 0] == 4.0 and got[255, 255] == 8.0
+    assert got[127, 127] == 1.0 and got[128, 127] == 4.0 and got[127, 128] == 2.0
+    # one scale per row and 128 columns (rows_per_block = 1) for activations
+    x_scales = np.array([[1.0, 0.5]] * 3 + [[2.0, 4.0]])
+    got = o.dequant_blocks(np.full((4, 256), 0x38, dtype=np.uint8), x_scales, 1)
+    assert got[0, 0] == 1.0 and got[0, 128] == 0.5 and got[3, 0] == 2.0 and got[3, 255] == 4.0
+
+
+def test_activation_format_of_each_dtype():
+    """h is stored in the activation format of the layer: bf16 for the bf16 layer, and
+    e4m3 with 1 x 128 scales whenever the activations are e4m3 (the FP8 layer and the
+    FP8 x FP4 layer, whose FP4 operand is the weights only)."""
+    assert o.activation_format(0) == "bf16"
+    assert o.activation_format(1) == "e4m3"
+    assert o.activation_format(2) == "e4m3"
 
 
 def test_pow2_scale_definition():
