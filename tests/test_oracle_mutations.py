@@ -206,6 +206,12 @@ def _dequant_scales_transposed(codes, scales, rows_per_block):
     return _dequant_blocks_orig(codes, sc.T if sc.shape[0] == sc.shape[1] else sc, rows_per_block)
 
 
+def _requant_one_scale_per_row(h):
+    h = np.asarray(h, np.float64)
+    s = o.pow2_scale(np.abs(h).max(axis=1))[:, None]                          # whole row, not 1 x 128
+    return o.quantize_e4m3(h / s) * s
+
+
 _select_orig = o.select_experts
 _dequant_blocks_orig = o.dequant_blocks
 _permute_orig = o.permute
@@ -231,6 +237,7 @@ MUTATIONS = {
     "masked layout keeps the last pairs": ("permute_masked", _masked_keeps_last),
     "groups ranked on the unbiased scores": ("route_from_scores", _route_groups_on_unbiased),
     "128x128 block scales transposed": ("dequant_blocks", _dequant_scales_transposed),
+    "h re-quantised with one scale per row": ("quantize_rows_1x128", _requant_one_scale_per_row),
 }
 
 

@@ -418,6 +418,18 @@ def test_rowwise_requant_error_bound():
     assert (err <= bound + 1e-300).all()
 
 
+def test_requant_scales_each_128_column_block_on_its_own():
+    """Values that are e4m3 codes times a power of two come back exactly when each 1 x 128
+    block gets its own scale: block 0 holds codes x 2^-20 (its maximum 448 x 2^-20 makes
+    the scale 2^-20), block 1 codes x 1.  One scale for the whole row (1) would flush
+    block 0 below e4m3's smallest subnormal, 2^-9."""
+    codes = o.decode_e4m3(np.arange(0, 0x7F, dtype=np.uint8))      # every finite positive code and 0
+    row0 = np.resize(codes, 128) * np.where(np.arange(128) % 2, -1.0, 1.0)
+    row0[5] = 448.0
+    h = np.concatenate([row0 * 2.0 ** -20, row0])[None, :]
+    np.testing.assert_array_equal(o.quantize_rows_1x128(h), h)
+
+
 # ------------------------------------------------------------------ bf16 activations
 def test_round_bf16_matches_torch_on_fp32_values():
     rng = np.random.default_rng(12)
