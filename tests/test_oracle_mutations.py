@@ -212,7 +212,12 @@ def _requant_one_scale_per_row(h):
     return o.quantize_e4m3(h / s) * s
 
 
+def _route_ignores_bias(x, w_r, bias, wl):
+    return _route_orig(x, w_r, None, wl)                                       # bias never reaches selection
+
+
 _select_orig = o.select_experts
+_route_orig = o.route
 _dequant_blocks_orig = o.dequant_blocks
 _permute_orig = o.permute
 _combine_orig = o.combine
@@ -238,6 +243,7 @@ MUTATIONS = {
     "groups ranked on the unbiased scores": ("route_from_scores", _route_groups_on_unbiased),
     "128x128 block scales transposed": ("dequant_blocks", _dequant_scales_transposed),
     "h re-quantised with one scale per row": ("quantize_rows_1x128", _requant_one_scale_per_row),
+    "route drops the selection bias": ("route", _route_ignores_bias),
 }
 
 

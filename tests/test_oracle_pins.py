@@ -220,6 +220,22 @@ def test_group_stage_ranks_groups_by_the_biased_scores():
     assert ids.tolist() == [[0]]  # without the bias the other group wins
 
 
+def test_route_applies_the_selection_bias_end_to_end():
+    """Logits through sigmoid, the bias steering the choice, the weight from the unbiased
+    score.  x = [1, 0] and W_r rows [1, 0], [.9, 0], [0, 1] give logits [1, .9, 0] and
+    scores expit(.) = [.731, .711, .5]; a bias of +.1 on expert 1 makes it the top-1
+    (.811 > .731); without the bias expert 0 wins."""
+    from types import SimpleNamespace
+    wl = SimpleNamespace(K=1, score_fn=1, n_group=1, topk_group=1, group_topn=1, renormalize=False,
+                         routed_scale=1.0)
+    x = np.array([[1.0, 0.0]])
+    w_r = np.array([[1.0, 0.0], [0.9, 0.0], [0.0, 1.0]])
+    ids, w, s = o.route(x, w_r, np.array([0.0, 0.1, 0.0]), wl)
+    assert ids.tolist() == [[1]] and w[0, 0] == pytest.approx(scipy.special.expit(0.9), rel=1e-15)
+    ids, _, _ = o.route(x, w_r, None, wl)
+    assert ids.tolist() == [[0]]
+
+
 def test_weights_sum_to_routed_scale():
     rng = np.random.default_rng(4)
     s = scipy.special.expit(rng.normal(size=(30, 64)))
