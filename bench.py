@@ -9,12 +9,19 @@ With N > 1 (torchrun, one process per GPU) every rank runs an independent replic
 the layer on its own inputs (the layer has no cross-GPU exchange on one node's data
 path): the reported value is all ranks' tokens over the slowest rank's time.
 
-`value` is tokens/s; the line also carries the grouped-GEMM TFLOP/s, an end-to-end
-number through moe_layer_forward_host (host activations copied in and the output
-copied back inside the timed region), the roofline of the dominant kernel from CUDA
-events recorded around its launches, the SM clocks sampled during the timed region,
-and the fp64 CPU oracle timed on a bounded sample of the same workload.
-`--impl reference` times that oracle alone, per step, on the host cores.
+The headline workload is the DeepSeek-V3-shaped prefill layer (T=8192, H=7168, I=2048,
+256 routed experts, top-8, plus a shared expert), the largest of the five workloads.
+On one GPU the line also carries, under "configs", the same record for each of the
+other four workloads (tiny, Mixtral-shaped prefill, DeepSeek-V3-shaped decode, skewed
+FP8), each timed over enough steps to fill a few hundred ms.
+
+Each record has `value` (tokens/s), the grouped-GEMM TFLOP/s and each GEMM kernel's
+fraction of the measured bf16 burst peak, an end-to-end number through
+moe_layer_forward_host (host activations copied in and the output copied back inside
+the timed region), the roofline of the dominant kernel from CUDA events recorded around
+its launches, the SM clocks sampled (NVML, every 5 ms) during the timed region, and the
+fp64 CPU oracle timed on a bounded sample of the same workload.  `--impl reference`
+times that oracle alone, per step, on the host cores.
 """
 from __future__ import annotations
 
@@ -95,31 +102,39 @@ FP8_OVER_BF16 = 2.0   # nominal dense e4m3 / bf16 tensor throughput (4.5 / 2.25 
 
 
 def power_capped(clk) -> bool:
-    """Whether the clock record says the power cap held the SM clock (sw_power_cap, or a
-    median under load below 90 % of the maximum)."""
-    return bool(clk and ("sw_power_cap" in clk.get("reasons", []) or
-                         (clk.get("sm_mhz") and clk.get("sm_max_mhz") and
-                          clk["sm_mhz"] < 0.9 * clk["sm_max_mhz"])))
+    """Whether the clock record says the power cap held the SM clock (sw_power_cap in at
+    least a fifth of the in-window samples, or a median under load below 90 % of the
+    maximum).  Reported beside the roofline; the fraction itself is always taken
+    against the burst peak."""
+    if not clk:
+        return False
+    n = clk.get("samples_in_window") or clk.get("samples") or 0
+    capped_samples = clk.get("sw_power_cap_samples")
+    if capped_samples is None:
+        by_reason = "sw_power_cap" in clk.get("reasons", [])
+    else:
+        by_reason = n > 0 and capped_samples >= 0.2 * n
+    low = bool(clk.get("sm_mhz") and clk.get("sm_max_mhz") and clk["sm_mhz"] < 0.9 * clk["sm_max_mhz"])
+    return bool(by_reason or low)
 
 
 def roofline_record(flops, nbytes, launch_ms, clk, fp8, peaks):
     """Roofline of one kernel from its algorithmic FLOPs and bytes per launch and its
     launch times (ms): tensor-bound when flops/bytes reaches the ridge of the peaks,
-    else HBM-bound.  A power-capped run is held to the sustained tensor peak; e4m3 takes
-    twice the bf16 figure (the nominal dense ratio).  peaks = (bf16 burst TFLOP/s,
-    bf16 sustained TFLOP/s, HBM GB/s, kind)."""
+    else HBM-bound.  `frac` is taken against the measured burst tensor peak (these
+    kernels run for milliseconds inside steps of milliseconds); frac_of_sustained is
+    the same figure against the seconds-long power-capped loop.  e4m3 takes twice the
+    bf16 figure (the nominal dense ratio).  peaks = (bf16 burst TFLOP/s, bf16 sustained
+    TFLOP/s, HBM GB/s, kind)."""
     burst, sustained, hbm_peak, peak_kind = peaks
-    capped = power_capped(clk)
     ratio = FP8_OVER_BF16 if fp8 else 1.0
-    tensor_peak = (sustained if capped else burst) * ratio
+    tensor_peak = burst * ratio
     avg = statistics.mean(launch_ms) if launch_ms else None
     ridge = tensor_peak * 1e12 / (hbm_peak * 1e9)
     if flops / nbytes >= ridge:
         achieved = flops / (avg / 1e3) / 1e12 if avg else None
         rec = {"bound": "tensor", "achieved": achieved, "peak": tensor_peak, "unit": "TFLOP/s",
-               "peak_kind": (f"{peak_kind} bf16 {'sustained' if capped else 'burst'}"
-                             + (" x2 (e4m3/bf16 nominal ratio)" if fp8 else "")),
-               "frac_of_burst": achieved / (burst * ratio) if achieved else None,
+               "peak_kind": f"{peak_kind} bf16 burst" + (" x2 (e4m3/bf16 nominal ratio)" if fp8 else ""),
                "frac_of_sustained": achieved / (sustained * ratio) if achieved else None}
     else:
         achieved = nbytes / (avg / 1e3) / 1e9 if avg else None
@@ -128,7 +143,8 @@ def roofline_record(flops, nbytes, launch_ms, clk, fp8, peaks):
     rec.update({"frac": achieved / rec["peak"] if achieved else None, "launches_timed": len(launch_ms),
                 "avg_ms": avg, "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": nbytes,
                 "tflops": flops / (avg / 1e3) / 1e12 if avg else None,
-                "gbs": nbytes / (avg / 1e3) / 1e9 if avg else None})
+                "gbs": nbytes / (avg / 1e3) / 1e9 if avg else None,
+                "power_capped": power_capped(clk)})
     return rec
 
 
@@ -205,8 +221,73 @@ def summarize_clock_rows(lines, window=None):
     reasons = sorted({names[i] for r in use for i in range(4) if r[6 + i] == "Active"})
     loaded = [v for v in sm if smax and v > 0.5 * max(smax)] or sm
     return {"sm_mhz": statistics.median(loaded) if loaded else None,
+            "sm_mhz_min": min(loaded) if loaded else None,
             "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+            "sw_power_cap_samples": sum(1 for r in use if r[9] == "Active"),
             "samples": len(rows), "samples_in_window": len(inside)}
+
+
+class NvmlClockSampler:
+    """Samples the SM clock, power and throttle reasons through NVML every 5 ms on a host
+    thread (reading only), producing rows in ClockSampler's csv format."""
+    INTERVAL_S = 0.005
+    # NVML clocks-event reason bits: sw power cap, hw slowdown, sw thermal, hw thermal
+    _CAP, _HW, _SWT, _HWT = 0x4, 0x8, 0x20, 0x40
+
+    def __init__(self, device):
+        import pynvml
+        self.nv = pynvml
+        pynvml.nvmlInit()
+        uuid = str(torch.cuda.get_device_properties(device).uuid)
+        if not uuid.startswith("GPU-"):
+            uuid = "GPU-" + uuid
+        self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+        self.rows, self.thread, self.stop_flag = [], None, False
+
+    def _reasons(self):
+        nv = self.nv
+        fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        return int(fn(self.h))
+
+    def _loop(self):
+        from datetime import datetime
+        nv = self.nv
+        smax = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+        act = lambda bits, b: "Active" if bits & b else "Not Active"  # noqa: E731
+        while not self.stop_flag:
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                pw = nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+                r = self._reasons()
+            except Exception:  # noqa: BLE001 - a failed read ends the sampling
+                break
+            ts = datetime.fromtimestamp(time.time()).strftime("%Y/%m/%d %H:%M:%S.%f")
+            self.rows.append(f"{ts}, 0, {sm}, {smax}, {pw:.1f}, {r:#x}, {act(r, self._HW)}, "
+                             f"{act(r, self._HWT)}, {act(r, self._SWT)}, {act(r, self._CAP)}")
+            time.sleep(self.INTERVAL_S)
+
+    def start(self):
+        import threading
+        self.thread = threading.Thread(target=self._loop, daemon=True)
+        self.thread.start()
+        time.sleep(0.05)
+
+    def stop(self, window=None):
+        time.sleep(0.05)
+        self.stop_flag = True
+        self.thread.join(timeout=5)
+        rec = summarize_clock_rows(self.rows, window)
+        rec["sampler"] = f"nvml every {self.INTERVAL_S * 1e3:g} ms"
+        return rec
+
+
+def clock_sampler(device):
+    """NVML sampler where pynvml works, else nvidia-smi."""
+    try:
+        return NvmlClockSampler(device)
+    except Exception:  # noqa: BLE001
+        return ClockSampler(device)
 
 
 class ClockSampler:
@@ -242,16 +323,71 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ CPU oracle leg
+def _expert_f64_bytes(wl):
+    return 3 * wl.H * wl.I * 8
+
+
+def _host_cache_bytes():
+    """fp64 expert weights the oracle leg may keep on the host: half the available RAM,
+    at most 120 GiB."""
+    try:
+        import psutil
+        avail = psutil.virtual_memory().available
+    except Exception:  # noqa: BLE001
+        avail = 32 << 30
+    return int(min(avail // 2, 120 << 30))
+
+
+class HostWeights:
+    """Expert weights for the oracle leg as exact fp64 values (bf16 widened, e4m3 codes
+    times their block scales, e2m1 through the oracle's decoder), loaded when the oracle
+    first asks for an expert and kept up to a host-memory cap, oldest first out.  Loading
+    is reading the layer's inputs, not layer work: its time is accumulated in load_s and
+    taken out of the oracle's measured time."""
+
+    def __init__(self, wl, d, cap_bytes=None):
+        self.wl, self.d, self.cache, self.load_s = wl, d, {}, 0.0
+        cap = _host_cache_bytes() if cap_bytes is None else cap_bytes
+        self.cap = max(1, cap // _expert_f64_bytes(wl))
+        self.shared = None
+        if wl.I_shared:
+            self.shared = tuple(d[n].to(torch.float64).cpu().numpy() for n in ("ws_gate", "ws_up", "ws_down"))
+
+    def _load(self, e):
+        from oracle import moe_oracle as o
+        wl, d = self.wl, self.d
+        if wl.dtype == W.DTYPE_FP8:
+            def deq(n):
+                q = d[n + "_q"][e].view(torch.float8_e4m3fn).to(torch.float64)
+                s = d[n + "_s"][e].to(torch.float64).repeat_interleave(128, 0).repeat_interleave(128, 1)
+                return (q * s).cpu().numpy()
+            return tuple(deq(n) for n in ("w_gate", "w_up", "w_down"))
+        if wl.dtype == W.DTYPE_FP8_FP4:
+            return tuple(o.dequant_fp4(d[n + "_q"][e].cpu().numpy(), d[n + "_s"][e].cpu().numpy())
+                         for n in ("w_gate", "w_up", "w_down"))
+        return tuple(d[n][e].to(torch.float64).cpu().numpy() for n in ("w_gate", "w_up", "w_down"))
+
+    def __call__(self, e):
+        e = int(e)
+        if e not in self.cache:
+            t0 = time.perf_counter()
+            while self.cache and len(self.cache) >= self.cap:
+                self.cache.pop(next(iter(self.cache)))
+            self.cache[e] = self._load(e)
+            self.load_s += time.perf_counter() - t0
+        return self.cache[e]
+
+
 def _oracle_sample(wl, d, n_tokens, seed=0, host_w=None):
     """Oracle forward (route + experts + combine) of a seeded token sample; returns
-    (tokens, seconds, threads).  host_w caches host copies of expert weights across
-    calls (filled here, outside the timed part)."""
+    (tokens, seconds, threads).  Host copies of the sampled activations are made before
+    the clock starts; the time spent loading expert weights on first use (host_w, a
+    HostWeights, which keeps them across calls) is taken out."""
     from oracle import moe_oracle as o
     from threadpoolctl import threadpool_info
     rng = np.random.default_rng(seed)
     toks = np.sort(rng.choice(wl.T, size=min(n_tokens, wl.T), replace=False))
     idx = torch.as_tensor(toks, device=d["w_r"].device)
-    # host copies of the inputs are not part of the timed oracle work
     if wl.dtype in (W.DTYPE_FP8, W.DTYPE_FP8_FP4):
         xq, xs = d["x_q"][idx].cpu().numpy(), d["x_scale"][idx].cpu().numpy()
         x_of = lambda: o.dequant_blocks(xq, xs, 1)  # noqa: E731
@@ -261,67 +397,44 @@ def _oracle_sample(wl, d, n_tokens, seed=0, host_w=None):
     w_r = d["w_r"].cpu().to(torch.float64).numpy()
     bias = d["bias"].cpu().to(torch.float64).numpy() if d["bias"] is not None else None
     if host_w is None:
-        host_w = {}
-
-    def fetch(e):
-        if e not in host_w:
-            if wl.dtype in (W.DTYPE_FP8, W.DTYPE_FP8_FP4):
-                host_w[e] = tuple((d[n + "_q"][e].cpu().numpy(), d[n + "_s"][e].cpu().numpy())
-                                  for n in ("w_gate", "w_up", "w_down"))
-            else:
-                host_w[e] = tuple(d[n][e].cpu() for n in ("w_gate", "w_up", "w_down"))
-        return host_w[e]
-
-    # routing decides which experts the sample needs; fetch them before the clock starts
-    x0 = x_of()
-    ids0, _, _ = o.route(x0, w_r, bias, wl)
-    for e in np.unique(ids0):
-        fetch(int(e))
-    shared = None
-    if wl.I_shared:
-        sh = [d[n].cpu() for n in ("ws_gate", "ws_up", "ws_down")]
-
-    def expert_weights(e):
-        if wl.dtype == W.DTYPE_FP8:
-            return tuple(o.dequant_blocks(q, s, 128) for q, s in fetch(e))
-        if wl.dtype == W.DTYPE_FP8_FP4:
-            return tuple(o.dequant_fp4(q, s) for q, s in fetch(e))
-        return tuple(t.to(torch.float64).numpy() for t in fetch(e))
-
+        host_w = HostWeights(wl, d)
+    load0 = host_w.load_s
     t0 = time.perf_counter()
-    x = x_of()
-    if wl.I_shared:
-        shared = tuple(t.to(torch.float64).numpy() for t in sh)
-    o.layer_forward(x, w_r, bias, expert_weights, wl, shared)
-    dt = time.perf_counter() - t0
+    o.layer_forward(x_of(), w_r, bias, host_w, wl, host_w.shared)
+    dt = time.perf_counter() - t0 - (host_w.load_s - load0)
     threads = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
     return len(toks), dt, threads
 
 
 def _cpu_sample_tokens(wl):
-    # about 10-30 s of fp64 work on a few host cores; with many experts each sampled
-    # token brings K experts' weights to widen, which dominates, so sample fewer tokens
+    """Tokens in one oracle sample: about 2e12 fp64 FLOP of expert work (a few seconds on
+    the host cores), at least 4, at most the batch."""
     per_token_flops = 6 * wl.K * wl.H * wl.I + 6 * wl.H * wl.I_shared
-    n = int(max(4, min(wl.T, 2.0e13 / max(per_token_flops, 1) / 4)))
-    return min(n, 8) if wl.E > 16 else n
+    return int(max(4, min(wl.T, 2.0e12 / max(per_token_flops, 1))))
+
+
+def cpu_baseline_record(wl, d):
+    n, dt, threads = _oracle_sample(wl, d, _cpu_sample_tokens(wl))
+    return {"value": n / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n} seeded tokens of {wl.name} through the fp64 oracle (route, experts, "
+                      f"combine; the time to load expert weights as fp64 is not counted); {dt:.2f} s"}
 
 
 # ------------------------------------------------------------------ our arm
-def run_ours(args):
-    world, rank, local = _dist()
-    torch.cuda.set_device(local)
-    if world > 1:
-        import torch.distributed as dist
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    wl = {**W.ALL, **W.PROFILE, **W.FP4}[args.workload]
-    if args.fused_combine:
-        wl = wl.with_(fused_combine=True)
-    if args.block_m:
-        wl = wl.with_(block_m=args.block_m)
-    if args.masked_cap:
-        wl = wl.with_(masked_cap=args.masked_cap)
+def _steps_for(ms_one, min_steps, target_ms=300.0, max_steps=1000):
+    """Steps that fill about target_ms of device time, at least min_steps."""
+    return int(min(max(min_steps, -(-target_ms // max(ms_one, 1e-3))), max(max_steps, min_steps)))
+
+
+def _gemm_peak(wl):
+    burst = _peaks()[0]
+    return burst * (FP8_OVER_BF16 if wl.dtype in (W.DTYPE_FP8, W.DTYPE_FP8_FP4) else 1.0)
+
+
+def measure(wl, steps, warmup, world=1, rank=0, local=0, cpu=True, adapt_steps=False):
+    """One workload: W warm-up steps, then the timed steps (L2 flushed before each),
+    the per-kernel breakdown, the end-to-end run through the host entry point, and
+    (rank 0, one GPU) the oracle's CPU baseline.  Returns the record (rank 0) or None."""
     p = B.params(wl)
     d = inputs.make_inputs(wl, seed=rank, device="cuda")
     fp8 = wl.dtype in (W.DTYPE_FP8, W.DTYPE_FP8_FP4)     # e4m3 activations
@@ -352,9 +465,16 @@ def run_ours(args):
         B.check(B.moe_layer_forward(p, a["x"], a["x_scale"], d["w_r"], d["bias"], *wts, out, ids, wgt,
                                     counts, ws, ws_bytes), "moe_layer_forward")
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         step()
     torch.cuda.synchronize()
+    if adapt_steps:  # fill a few hundred ms, so the clock record has many in-window samples
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        step()
+        s1.record(stream)
+        torch.cuda.synchronize()
+        steps = _steps_for(s0.elapsed_time(s1), steps)
 
     def barrier():
         if world > 1:
@@ -363,16 +483,15 @@ def run_ours(args):
         torch.cuda.synchronize()
 
     # ---------------- timed region: device-resident inputs
-    clocks = ClockSampler(local) if rank == 0 else None
+    clocks = clock_sampler(local) if rank == 0 else None
     if clocks:
         clocks.start()
     dominant = B.K_GATEUP
-    B.check(B.moe_trace_enable(1 << dominant, 4 * args.steps))
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
+    B.check(B.moe_trace_enable(1 << dominant, 4 * steps))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     barrier()
     t_region = time.time()
-    for i in range(args.steps):
+    for i in range(steps):
         flush.fill_(i & 0xFF)
         ev[i][0].record(stream)
         step()
@@ -385,7 +504,7 @@ def run_ours(args):
     clk = clocks.stop(t_region) if clocks else None
     status = B.moe_get_device_status(ws)
     if status != 0:
-        raise B.MoEError(f"device status {status:#x} after the timed steps")
+        raise B.MoEError(f"device status {status:#x} after the timed steps of {wl.name}")
 
     # per-kernel breakdown: a few more steps, every kernel of the library bracketed by
     # events (outside the timed region, so the events do not perturb the headline)
@@ -402,90 +521,125 @@ def run_ours(args):
     counts_h = counts.cpu().numpy()
     P = wl.T * wl.K
     ms_total = max_over_ranks(float(sum(step_ms)), world, "cuda")
-    ms_step = ms_total / args.steps
+    ms_step = ms_total / steps
     tokens_per_s = replica_throughput(wl.T, world, ms_step)
 
     # algorithmic work (unpadded rows; weights of experts that received tokens)
     abytes = 1 if fp8 else 2                       # activation bytes per element
     wbytes = (0.5 + 1 / 32) if w4 else abytes       # weight bytes per element (e2m1: + one scale byte per 32)
     active = int((counts_h > 0).sum())
-    flops_gateup = 4.0 * P * wl.H * wl.I
-    flops_down = 2.0 * P * wl.I * wl.H
-    flops_shared = 6.0 * wl.T * wl.H * wl.I_shared
-    gemm_flops = flops_gateup + flops_down + flops_shared
+    flops = {"gateup_swiglu": 4.0 * P * wl.H * wl.I, "down": 2.0 * P * wl.I * wl.H,
+             "shared_gateup": 4.0 * wl.T * wl.H * wl.I_shared, "shared_down": 2.0 * wl.T * wl.H * wl.I_shared}
+    gemm_flops = sum(flops.values())
     bytes_gateup = (active * 2 * wl.I * wl.H * wbytes + P * wl.H * abytes + P * wl.I * abytes)
     layer_bytes = (active * 3 * wl.I * wl.H * wbytes + 3 * wl.I_shared * wl.H * 2 + wl.E * wl.H * 2
                    + wl.T * wl.H * (abytes + 2))
     dt_name = "e4m3 x e2m1" if w4 else ("e4m3" if fp8 else "bf16")
     dom_ms = [ms for k, ms in traced if k == dominant]
-    roofline = roofline_record(flops_gateup, bytes_gateup, dom_ms, clk, fp8, _peaks())
+    roofline = roofline_record(flops["gateup_swiglu"], bytes_gateup, dom_ms, clk, fp8, _peaks())
     roofline.update({"kernel": f"gateup_swiglu (grouped GEMM, fused SwiGLU, {dt_name})",
                      "traffic": _profiled_traffic(wl.name, gateup_sources(wl))})
+    peak_t = _gemm_peak(wl)
+    hbm_peak = _peaks()[2]
+    gemm_ms = sum(kernel_ms.get(k, 0.0) for k in flops)
 
     # ---------------- end to end: host activations in, host output out
     x_host = (d["x_q"] if fp8 else d["x"]).cpu().pin_memory()
     xs_host = d["x_scale"].cpu().pin_memory() if fp8 else None
     out_host = torch.empty((wl.T, wl.H), dtype=torch.bfloat16).pin_memory()
-    e2e_ms = None
-    if True:
-        def e2e_step():
-            B.check(B.moe_layer_forward_host(p, x_host, xs_host, d["w_r"], d["bias"], *wts, out_host, ws,
-                                             ws_bytes), "moe_layer_forward_host")
-        for _ in range(2):
-            e2e_step()
-        torch.cuda.synchronize()
-        ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(args.steps)]
-        barrier()
-        for i in range(args.steps):
-            flush.fill_(i & 0xFF)
-            ev2[i][0].record(stream)
-            e2e_step()
-            ev2[i][1].record(stream)
-        barrier()
-        e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in ev2), world, "cuda") / args.steps
+
+    def e2e_step():
+        B.check(B.moe_layer_forward_host(p, x_host, xs_host, d["w_r"], d["bias"], *wts, out_host, ws,
+                                         ws_bytes), "moe_layer_forward_host")
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    barrier()
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        ev2[i][0].record(stream)
+        e2e_step()
+        ev2[i][1].record(stream)
+    barrier()
+    e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in ev2), world, "cuda") / steps
     xbytes = wl.T * wl.H * (1 if fp8 else 2) + (wl.T * (wl.H // 128) * 4 if fp8 else 0)
 
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n, dt, threads = _oracle_sample(wl, d, _cpu_sample_tokens(wl))
-        cpu = {"value": n / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-               "sample": f"{n} seeded tokens of {wl.name} through the fp64 oracle "
-                         f"(route, experts, combine); {dt:.1f} s"}
+    base = cpu_baseline_record(wl, d) if (cpu and rank == 0 and world == 1) else None
+    del d, ws, flush
+    torch.cuda.empty_cache()
+    if rank != 0:
+        return None
+    return {
+        "workload": f"{wl.name}: {_describe(wl)}",
+        "value": tokens_per_s, "unit": "tokens/s", "ms_per_step": ms_step, "steps": steps,
+        "dtype": "fp8xfp4" if w4 else ("fp8" if fp8 else "bf16"),
+        "grouped_gemm_tflops": gemm_flops / (ms_step / 1e3) / 1e12 * world,
+        "gemm_kernel_tflops": {k: f / (kernel_ms[k] / 1e3) / 1e12 for k, f in flops.items() if kernel_ms.get(k)},
+        "gemm_kernel_frac_of_burst": {k: f / (kernel_ms[k] / 1e3) / 1e12 / peak_t
+                                      for k, f in flops.items() if kernel_ms.get(k)},
+        "gemm_kernels_frac_of_burst": (gemm_flops / (gemm_ms / 1e3) / 1e12 / peak_t) if gemm_ms else None,
+        "layer_hbm_gbs": layer_bytes / (ms_step / 1e3) / 1e9 * world,
+        "layer_hbm_frac": layer_bytes / (ms_step / 1e3) / 1e9 / hbm_peak,
+        "layer_algorithmic_bytes": layer_bytes,
+        "active_experts": active,
+        "e2e": {"value": wl.T * world / (e2e_ms / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": xbytes, "d2h_bytes_per_step": wl.T * wl.H * 2},
+        "roofline": roofline,
+        "clocks": clk,
+        "gpu_launches": B.moe_layer_launch_count(p) * steps,
+        "cpu_baseline": base,
+        "kernel_ms_per_step": kernel_ms,
+        "expert_load": {"max": int(counts_h.max()), "min": int(counts_h.min()), "mean": P / wl.E},
+    }
 
+
+SUB_CONFIGS = ("tiny", "mixtral_prefill", "dsv3_decode", "skewed_fp8", "dsv3_prefill")
+
+
+def run_ours(args):
+    world, rank, local = _dist()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    wl = {**W.ALL, **W.PROFILE, **W.FP4}[args.workload]
+    if args.fused_combine:
+        wl = wl.with_(fused_combine=True)
+    if args.block_m:
+        wl = wl.with_(block_m=args.block_m)
+    if args.masked_cap:
+        wl = wl.with_(masked_cap=args.masked_cap)
+    rec = measure(wl, args.steps, args.warmup, world, rank, local, cpu=not args.no_cpu_baseline)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
         dist.destroy_process_group()
+    configs = None
+    if world == 1 and not args.no_configs:
+        configs = {}
+        for name in SUB_CONFIGS:
+            if name == wl.name:
+                continue
+            configs[name] = measure(W.ALL[name], args.steps, args.warmup, cpu=not args.no_cpu_baseline,
+                                    adapt_steps=True)
     if rank != 0:
         return
     line = {
-        "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "fp8xfp4" if w4 else ("fp8" if fp8 else "bf16"),
+        "metric": METRIC, "value": rec["value"], "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": rec["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": rec["dtype"],
         "data": "synthetic (seeded Gaussian activations and random-init weights)",
-        "config": {"workload": f"{wl.name}: {_describe(wl)}", "global_batch": wl.T * world,
+        "config": {"workload": rec["workload"], "global_batch": wl.T * world,
                    "seq_len": 1, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "flushed before every timed step (512 MiB write, outside the events)"},
-        "grouped_gemm_tflops": gemm_flops / (ms_step / 1e3) / 1e12 * world,
-        "gemm_kernel_tflops": {k: f / (kernel_ms[k] / 1e3) / 1e12 for k, f in
-                               (("gateup_swiglu", flops_gateup), ("down", flops_down),
-                                ("shared_gateup", 4.0 * wl.T * wl.H * wl.I_shared),
-                                ("shared_down", 2.0 * wl.T * wl.H * wl.I_shared))
-                               if kernel_ms.get(k)},
-        "layer_hbm_gbs": layer_bytes / (ms_step / 1e3) / 1e9 * world,
-        "active_experts": active,
-        "e2e": {"value": wl.T * world / (e2e_ms / 1e3) if e2e_ms else None, "unit": "tokens/s",
-                "h2d_bytes_per_step": xbytes, "d2h_bytes_per_step": wl.T * wl.H * 2},
-        "roofline": roofline,
-        "clocks": clk,
-        "gpu_launches": B.moe_layer_launch_count(p) * args.steps,
-        "cpu_baseline": cpu,
-        "kernel_ms_per_step": kernel_ms,
-        "expert_load": {"max": int(counts_h.max()), "min": int(counts_h.min()),
-                        "mean": P / wl.E},
     }
+    line.update({k: v for k, v in rec.items() if k not in ("workload", "value", "unit", "ms_per_step",
+                                                           "steps", "dtype")})
+    if configs is not None:
+        line["configs"] = configs
     print(json.dumps(line), flush=True)
 
 
@@ -496,19 +650,19 @@ def run_reference(args):
         return
     wl = {**W.ALL, **W.PROFILE, **W.FP4}[args.workload]
     d = inputs.make_inputs(wl, seed=0, device="cpu" if not torch.cuda.is_available() else "cuda")
-    host_w = {}
-    # size each step's token sample so that all warm-up and timed steps together take about
-    # REFERENCE_BUDGET_S of oracle time.  A step costs about c0 + n*c1 (c0: widening the
-    # chosen experts' weights to fp64; c1: per token); two untimed samples fix c0 and c1.
-    k1, t1, _ = _oracle_sample(wl, d, 2, seed=10 ** 6, host_w=host_w)
-    k2, t2, _ = _oracle_sample(wl, d, 8, seed=10 ** 6 + 1, host_w=host_w)
-    c1 = max((t2 - t1) / max(k2 - k1, 1), 1e-6)
-    c0 = max(t1 - k1 * c1, 0.0)
+    host_w = HostWeights(wl, d)
+    # Every step runs the same seeded token sample (as the GPU arm re-runs one batch);
+    # expert weights are loaded as fp64 on first use, kept while host memory allows, and
+    # their load time is not counted.  The sample makes all warm-up and timed steps
+    # together take about REFERENCE_BUDGET_S of oracle time, at most the cpu sample.
+    cap = min(wl.T, _cpu_sample_tokens(wl))
+    k0, t0, _ = _oracle_sample(wl, d, min(cap, 64), seed=0, host_w=host_w)
+    c1 = max(t0 / k0, 1e-6)
     per_step = REFERENCE_BUDGET_S / (args.warmup + args.steps)
-    n = int(max(1, min(wl.T, _cpu_sample_tokens(wl), (per_step - c0) / c1)))
+    n = int(max(1, min(cap, per_step / c1)))
     times, toks, threads = [], 0, 1
     for i in range(args.warmup + args.steps):
-        k, dt, threads = _oracle_sample(wl, d, n, seed=i, host_w=host_w)
+        k, dt, threads = _oracle_sample(wl, d, n, seed=0, host_w=host_w)
         if i >= args.warmup:
             times.append(dt)
             toks += k
@@ -521,7 +675,9 @@ def run_reference(args):
         "config": {"workload": f"{wl.name}: {_describe(wl)}", "global_batch": wl.T, "seq_len": 1,
                    "parallelism": "host cores"},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                         "sample": f"{n} seeded tokens per step through the fp64 oracle"},
+                         "sample": f"the same {n} seeded tokens every step through the fp64 oracle "
+                                   f"(route, experts, combine; the time to load expert weights as "
+                                   f"fp64 is not counted)"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -572,9 +728,11 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="mixtral_prefill", choices=sorted(W.ALL) + sorted(W.PROFILE) + sorted(W.FP4))
+    ap.add_argument("--workload", default="dsv3_prefill", choices=sorted(W.ALL) + sorted(W.PROFILE) + sorted(W.FP4))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="time only --workload (no per-config records of the other workloads)")
     ap.add_argument("--fused-combine", action="store_true",
                     help="down projection adds into the output with fp32 atomics (non-deterministic)")
     ap.add_argument("--block-m", type=int, default=0, choices=[0, 128, 256],

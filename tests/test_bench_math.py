@@ -15,13 +15,19 @@ def test_tensor_bound_kernel_at_burst_clocks():
     assert r["launches_timed"] == 2 and r["avg_ms"] == 1.25
 
 
-def test_power_capped_run_is_held_to_the_sustained_peak():
+def test_power_capped_run_keeps_the_burst_peak_and_is_flagged():
     clk = {"reasons": ["sw_power_cap"], "sm_mhz": 1965, "sm_max_mhz": 1965}
     r = bench.roofline_record(2.0e12, 2.5e9, [1.25], clk, False, PEAKS)
-    assert r["peak"] == 1400.0 and "sustained" in r["peak_kind"]
+    assert r["peak"] == 1600.0 and "burst" in r["peak_kind"] and r["power_capped"]
+    assert abs(r["frac_of_sustained"] - 1600.0 / 1400.0) < 1e-12
     # a clock stuck well below its maximum counts as capped as well
     assert bench.power_capped({"reasons": [], "sm_mhz": 1500, "sm_max_mhz": 1965})
     assert not bench.power_capped({"reasons": [], "sm_mhz": 1900, "sm_max_mhz": 1965})
+    # with per-sample counts, one capped sample among many in the window is not a cap
+    one = {"reasons": ["sw_power_cap"], "sw_power_cap_samples": 1, "samples_in_window": 40,
+           "sm_mhz": 1965, "sm_max_mhz": 1965}
+    assert not bench.power_capped(one)
+    assert bench.power_capped({**one, "sw_power_cap_samples": 12})
 
 
 def test_e4m3_kernel_takes_twice_the_bf16_peak():
@@ -85,10 +91,38 @@ def test_clock_summary_uses_the_samples_inside_the_timed_window():
     win = (t("2026/12/02 10:00:00.200"), t("2026/12/02 10:00:00.400"))
     c = bench.summarize_clock_rows(lines, win)
     assert c["sm_mhz"] == 1380 and c["sm_max_mhz"] == 1965 and c["reasons"] == ["sw_power_cap"]
-    assert c["samples"] == 5 and c["samples_in_window"] == 3
+    assert c["samples"] == 5 and c["samples_in_window"] == 3 and c["sw_power_cap_samples"] == 3
     assert bench.power_capped(c)
     # a region shorter than the sampling interval: all samples, flagged as such
     short = (t("2026/12/02 10:00:00.400"), t("2026/12/02 10:00:00.450"))
     c = bench.summarize_clock_rows(lines, short)
     assert c["samples_in_window"] == 0 and c["samples"] == 5 and c["sm_mhz"] == 1390
     assert bench.summarize_clock_rows([], None)["sm_mhz"] is None
+
+
+def test_steps_fill_the_target_time():
+    assert bench._steps_for(7.5, 20) == 40          # 300 ms / 7.5 ms
+    assert bench._steps_for(100.0, 20) == 20        # never below the asked steps
+    assert bench._steps_for(0.01, 20) == 1000       # capped
+    assert bench._steps_for(0.01, 2000) == 2000
+
+
+def test_cpu_sample_sizes():
+    from mixture_experts_ffn_08_b200 import workloads as W
+    assert bench._cpu_sample_tokens(W.TINY) == 64                  # whole batch
+    assert bench._cpu_sample_tokens(W.MIXTRAL_PREFILL) == 2838     # 2e12 / (6*2*4096*14336), floored
+    assert bench._cpu_sample_tokens(W.DSV3_DECODE) == 128
+    n = bench._cpu_sample_tokens(W.DSV3_PREFILL)
+    assert 2000 < n < 3000
+
+
+def test_host_weights_load_time_is_kept_apart_and_cache_is_bounded():
+    import torch
+    from mixture_experts_ffn_08_b200 import workloads as W
+    wl = W.Workload("hw", T=4, H=128, I=128, E=4, K=2)
+    d = {n: torch.randn(wl.E, 128, 128).to(torch.bfloat16) for n in ("w_gate", "w_up", "w_down")}
+    hw = bench.HostWeights(wl, d, cap_bytes=2 * bench._expert_f64_bytes(wl))
+    for e in (0, 1, 2, 0):
+        g, u, dn = hw(e)
+        assert g.dtype.name == "float64" and (g == d["w_gate"][e].double().numpy()).all()
+    assert len(hw.cache) <= 2 and hw.load_s > 0

@@ -129,12 +129,11 @@ def test_fp4_layer_full_size_decode_sampled():
     s = o.scores(o.router_logits(x, P.f64(d["w_r"])), wl.score_fn)
     n_mism, w_or = P.check_routing(gpu_ids, res["w"].cpu().numpy(), s, P.f64(d["bias"]), wl)
     assert n_mism <= 2
-    rng = np.random.default_rng(0)
-    toks = np.sort(rng.choice(wl.T, size=6, replace=False))
+    toks = P.stratified_tokens(gpu_ids, wl.E, np.random.default_rng(0), n_random=8, n_tail_experts=8, hot_rows=4)
     ref = o.forward_given_routing(x[toks], gpu_ids[toks], w_or[toks], P.expert_weights_fn(d, wl), wl.E, None,
                                   h_format="e4m3")
     got = P.f64(res["out"][torch.as_tensor(toks, device="cuda")])
-    P.check_close(got, ref, P.FP8_MAX_TOL, wl.name)
+    P.check_close(got, ref, P.FP8_MAX_TOL, f"{wl.name} ({len(toks)} tokens)")
 
 
 # ---------------------------------------------------------------- few tokens per expert

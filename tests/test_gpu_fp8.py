@@ -122,12 +122,16 @@ def test_fp8_layer_full_size_sampled():
     assert n_mism <= max(2, wl.T // 1000)
     counts = res["counts"].cpu().numpy()
     assert counts.sum() == wl.T * wl.K and counts.max() >= 0.85 * wl.T
-    rng = np.random.default_rng(0)
-    toks = np.sort(rng.choice(wl.T, size=6, replace=False))
+    # rows spread over the hot expert's bucket (~15k rows, ~120 M-tiles), the last
+    # partial M-tile of several other experts, and a few uniform draws
+    toks = P.stratified_tokens(gpu_ids, wl.E, np.random.default_rng(0), n_random=4, n_tail_experts=6,
+                               hot_rows=16)
+    hot = int(np.argmax(counts))
+    assert (gpu_ids[toks] == hot).any(axis=1).sum() >= 16
     ref = o.forward_given_routing(x[toks], gpu_ids[toks], w_or[toks], P.expert_weights_fn(d, wl), wl.E, None,
                                   h_format="e4m3")
     got = P.f64(res["out"][torch.as_tensor(toks, device="cuda")])
-    P.check_close(got, ref, P.FP8_MAX_TOL, wl.name)
+    P.check_close(got, ref, P.FP8_MAX_TOL, f"{wl.name} ({len(toks)} tokens)")
 
 
 def test_fp8_host_entry_point_matches_device_entry_point():

@@ -3,7 +3,16 @@
 Small workloads keep the shapes' features (routing rules, several M/N/K tiles, ragged
 buckets) at sizes the oracle finishes in seconds and are compared on every element.
 The full workloads run in the configuration the benchmark times and are compared on the
-whole routing decision and permutation, plus sampled output rows.
+whole routing decision and permutation, plus output rows: every token of the decode
+workload, and for the prefill workloads a stratified sample that includes tokens in
+several experts' last, partially filled M-tiles and rows spread over the most loaded
+expert's bucket.
+
+Every output is judged against two oracles: h stored in bf16 between the projections
+(the bf16 expert FFN, routing primer §8.4), where both bounds are asserted, and h kept
+exact, where the mean relative bound is asserted and the max bound wherever it holds
+(every case but those in EXACT_MAX_EXCEEDS); both errors are printed and, with
+MOE_PARITY_REPORT set, appended to that file.
 """
 import numpy as np
 import pytest
@@ -36,6 +45,20 @@ SMALL = {
 }
 
 
+# Cases whose max|err| against the exact-h oracle is above 2e-2 * RMS: measured 0.0208
+# (0.0159 against the bf16-h oracle), of which 0.0159 is the floor that rounding the
+# exact output once to bf16 already costs on these 512,000 outputs.  Every other case
+# asserts the max bound against the exact-h oracle as well.
+EXACT_MAX_EXCEEDS = {"mixtral_small", "mixtral_small_pair", "mixtral_small_fused"}
+
+
+def _both(x, ids, w, d, wl):
+    """Oracle outputs with h in bf16 and with h exact, on the given routing."""
+    sh = P.shared_weights(d, wl)
+    ew = P.expert_weights_fn(d, wl)
+    return tuple(o.forward_given_routing(x, ids, w, ew, wl.E, sh, h_format=f) for f in ("bf16", None))
+
+
 def _oracle_full(d, wl, gpu_ids):
     x = P.x_f64(d, wl)
     s = o.scores(o.router_logits(x, P.f64(d["w_r"])), wl.score_fn)
@@ -53,9 +76,9 @@ def test_layer_small_all_elements(name):
     x, s, bias = _oracle_full(d, wl, gpu_ids)
     _, w_or = P.check_routing(gpu_ids, r["w"].cpu().numpy(), s, bias, wl)
     np.testing.assert_array_equal(r["counts"].cpu().numpy(), np.bincount(gpu_ids.ravel(), minlength=wl.E))
-    ref = o.forward_given_routing(x, gpu_ids, w_or, P.expert_weights_fn(d, wl), wl.E,
-                                  P.shared_weights(d, wl), h_format=o.activation_format(wl.dtype))
-    P.check_close(P.f64(r["out"]), ref, P.BF16_MAX_TOL, name)
+    ref, ref_exact = _both(x, gpu_ids, w_or, d, wl)
+    P.check_both_oracles(P.f64(r["out"]), ref, ref_exact, P.BF16_MAX_TOL, name,
+                         exact_max=name not in EXACT_MAX_EXCEEDS)
 
 
 def test_layer_is_deterministic():
@@ -85,13 +108,16 @@ def test_layer_full_size_sampled(name):
     assert counts.sum() == wl.T * wl.K
     np.testing.assert_array_equal(counts, np.bincount(gpu_ids.ravel(), minlength=wl.E))
     rng = np.random.default_rng(0)
-    n_sample = 12 if wl.E <= 8 else 4
-    toks = np.sort(rng.choice(wl.T, size=n_sample, replace=False))
-    ref = o.forward_given_routing(x[toks], gpu_ids[toks], w_or[toks], P.expert_weights_fn(d, wl),
-                                  wl.E, P.shared_weights(d, wl) if wl.I_shared else None,
-                                  h_format=o.activation_format(wl.dtype))
+    if wl.T <= 128:
+        toks = np.arange(wl.T)                     # decode: every token
+    elif wl.E <= 8:
+        toks = P.stratified_tokens(gpu_ids, wl.E, rng, n_random=8, n_tail_experts=wl.E, hot_rows=8)
+    else:
+        toks = P.stratified_tokens(gpu_ids, wl.E, rng, n_random=4, n_tail_experts=8, hot_rows=4)
+    ref, ref_exact = _both(x[toks], gpu_ids[toks], w_or[toks], d, wl)
     got = P.f64(r["out"][torch.as_tensor(toks, device="cuda")])
-    P.check_close(got, ref, P.BF16_MAX_TOL, name)
+    P.check_both_oracles(got, ref, ref_exact, P.BF16_MAX_TOL, f"{name} ({len(toks)} tokens)",
+                         exact_max=name not in EXACT_MAX_EXCEEDS)
     del d, r
     torch.cuda.empty_cache()
 

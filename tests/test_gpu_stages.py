@@ -198,8 +198,9 @@ def test_expert_ffn_grouped_gemm(E, K, T, H, I, bm):
     rows = B.moe_max_padded_rows(p)
     offs = torch.as_tensor(r["offs"], device="cuda")
     counts = torch.as_tensor(r["counts"], device="cuda")
-    ref, _ = o.expert_outputs(P.f64(d["x"]), ids, P.expert_weights_fn(d, wl), E,
-                              B.moe_effective_block_m(p), h_format="bf16")
+    ew = P.expert_weights_fn(d, wl)
+    ref, _ = o.expert_outputs(P.f64(d["x"]), ids, ew, E, B.moe_effective_block_m(p), h_format="bf16")
+    ref_exact, _ = o.expert_outputs(P.f64(d["x"]), ids, ew, E, B.moe_effective_block_m(p), h_format=None)
     total = r["offs"][E]
     real = r["por"][:total] >= 0
     # with counts: pad rows are left untouched; without: they are computed (zero input -> 0)
@@ -210,7 +211,9 @@ def test_expert_ffn_grouped_gemm(E, K, T, H, I, bm):
         torch.cuda.synchronize()
         assert B.moe_get_device_status(r["ws"]) == 0
         got = P.f64(y[:total])
-        P.check_close(got[real], ref[real], P.BF16_MAX_TOL, "y_perm")
+        # y_perm is fp32: against the exact-h oracle only h's bf16 storage separates them
+        P.check_both_oracles(got[real], ref[real], ref_exact[real], P.BF16_MAX_TOL,
+                             f"y_perm E{E} K{K} T{T} H{H} I{I} bm{bm}", exact_max=True)
         if cnt is None:
             assert np.all(got[~real] == 0)
         else:
@@ -226,7 +229,8 @@ def test_shared_expert_dense_ffn_ragged_T():
     B.check(B.moe_shared_expert_ffn(p, d["x"], d["ws_gate"], d["ws_up"], d["ws_down"], y, ws, ws.numel()))
     torch.cuda.synchronize()
     ref = o.swiglu_ffn(P.f64(d["x"]), *P.shared_weights(d, wl), h_format="bf16")
-    P.check_close(P.f64(y), ref, P.BF16_MAX_TOL, "shared")
+    ref_exact = o.swiglu_ffn(P.f64(d["x"]), *P.shared_weights(d, wl), h_format=None)
+    P.check_both_oracles(P.f64(y), ref, ref_exact, P.BF16_MAX_TOL, "shared expert y (fp32)", exact_max=True)
 
 
 # ------------------------------------------------------------------ combine
