@@ -542,6 +542,8 @@ def measure(wl, steps, warmup, world=1, rank=0, local=0, cpu=True, adapt_steps=F
     peak_t = _gemm_peak(wl)
     hbm_peak = _peaks()[2]
     gemm_ms = sum(kernel_ms.get(k, 0.0) for k in flops)
+    bm = B.moe_effective_block_m(p)
+    mma_rows = int(sum(-(-int(c) // bm) * bm for c in counts_h))   # bucket rows the routed GEMMs compute
 
     # ---------------- end to end: host activations in, host output out
     x_host = (d["x_q"] if fp8 else d["x"]).cpu().pin_memory()
@@ -583,6 +585,8 @@ def measure(wl, steps, warmup, world=1, rank=0, local=0, cpu=True, adapt_steps=F
         "layer_hbm_frac": layer_bytes / (ms_step / 1e3) / 1e9 / hbm_peak,
         "layer_algorithmic_bytes": layer_bytes,
         "active_experts": active,
+        "routed_gemm_rows": {"real": P, "computed": mma_rows,
+                             "pad_frac": (mma_rows - P) / mma_rows if mma_rows else 0.0},
         "e2e": {"value": wl.T * world / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": xbytes, "d2h_bytes_per_step": wl.T * wl.H * 2},
         "roofline": roofline,

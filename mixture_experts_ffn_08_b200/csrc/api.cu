@@ -2,6 +2,8 @@
 // workspace layout, stage orchestration on one stream, device status word and tracing.
 #include <cuda_runtime.h>
 
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
 #include <vector>
 
@@ -22,6 +24,14 @@ int num_sms() {
     cached[dev] = n;
   }
   return cached[dev];
+}
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* v = std::getenv("MOE_DISABLE_PDL");
+    return v == nullptr || v[0] == '\0' || std::strcmp(v, "0") == 0;
+  }();
+  return on;
 }
 
 // ------------------------------------------------------------------ tracing
@@ -93,7 +103,7 @@ Layout layout(const moe_params_t* p) {
   auto take = [&](size_t bytes) { size_t at = o; o += up(bytes); return at; };
   L.max_rows = rows;
   L.status = take(256);
-  L.logits = take(T * E * 4);
+  L.logits = take(router_k_splits(T, p->H, p->E) * T * E * 4);  // one [T,E] slice per K-slice
   L.xb = take(is_fp8(p) ? T * H * 2 : 0);
   L.ids = take(P * 4);
   L.w = take(P * 4);
@@ -202,7 +212,7 @@ moe_status_t do_route(const moe_params_t* p, const void* x, const float* x_scale
   }
   float* logits = at<float>(ws, L.logits);
   MOE_CUDA(gemm_router(xb, w_r, p->T, p->H, p->E, logits, status, st));
-  MOE_CUDA(launch_topk(logits, *p, bias, ids, w, st));
+  MOE_CUDA(launch_topk(logits, *p, bias, ids, w, st, router_k_splits(p->T, p->H, p->E)));
   return MOE_OK;
 }
 

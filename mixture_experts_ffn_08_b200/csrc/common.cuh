@@ -234,6 +234,16 @@ MOE_DEVINL uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Programmatic dependent launch.  Every kernel of the layer is launched so that the
+// next kernel in the stream may start while it runs (cudaLaunchAttribute
+// ProgrammaticStreamSerialization).  Each kernel first lets its dependents launch, then
+// waits, before its first global-memory access, until the kernel before it has
+// finished and its writes are visible: the dependents' CTAs take SMs as this kernel's
+// CTAs leave and do their set-up (barriers, TMEM, descriptor prefetch) in the gap.
+// Both instructions are no-ops for a kernel launched without the attribute.
+MOE_DEVINL void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+MOE_DEVINL void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 MOE_DEVINL void set_status(int32_t* status, int32_t bits) {
   if (status) atomicOr(status, bits);
 }

@@ -49,9 +49,9 @@ cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMa
   const long long sms = num_sms();
   const int grid = static_cast<int>(max_items < sms ? (max_items > 0 ? max_items : 1) : sms);
   trace_before(kid, st);
-  kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, st>>>(a, b0, b1, gp);
+  err = launch_k(kern, grid, Cfg::THREADS, Cfg::SMEM_BYTES, st, a, b0, b1, gp);
   trace_after(kid, st);
-  return cudaGetLastError();
+  return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 long long ceil_div(long long a, long long b) { return (a + b - 1) / b; }
@@ -76,7 +76,9 @@ cudaError_t gemm_router(const void* x, const void* w_r, int T, int H, int E, flo
   gp.out = logits;
   gp.ldo = E;
   gp.status = status;
-  const long long items = ceil_div(T, 128) * ceil_div(E, bn);
+  gp.k_splits = router_k_splits(T, H, E);
+  gp.split_stride = static_cast<long long>(T) * E;
+  const long long items = ceil_div(T, 128) * ceil_div(E, bn) * gp.k_splits;
 #define MOE_ROUTER_CASE(BN, ST) \
   return launch<GemmCfg<BN, EPI_F32, ST>>(ta, tb, tb, gp, items, MOE_K_ROUTER_GEMM, st)
   switch (bn) {

@@ -65,9 +65,9 @@ cudaError_t launch8(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorM
   const long long sms = num_sms();
   const int grid = static_cast<int>(max_items < sms ? (max_items > 0 ? max_items : 1) : sms);
   trace_before(kid, st);
-  kern<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, st>>>(a, b0, b1, fp);
+  err = launch_k(kern, grid, Cfg::THREADS, Cfg::SMEM_BYTES, st, a, b0, b1, fp);
   trace_after(kid, st);
-  return cudaGetLastError();
+  return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 // UE8M0 byte of a power-of-two fp32 scale: its biased exponent field.
@@ -79,6 +79,8 @@ __device__ __forceinline__ uint32_t ue8m0_of(float s) { return (__float_as_uint(
 __global__ void sf_rows_to_atoms_kernel(const float* __restrict__ scales, int nk,
                                         const int32_t* __restrict__ offsets, int G,
                                         uint8_t* __restrict__ atoms) {
+  pdl_launch_dependents();
+  pdl_wait();
   const long long n = static_cast<long long>(__ldg(offsets + G)) * nk;
   const int nk4 = (nk + 3) / 4;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
@@ -94,6 +96,8 @@ __global__ void sf_rows_to_atoms_kernel(const float* __restrict__ scales, int nk
 // whose 128 words all hold the scales of four consecutive K blocks.
 __global__ void sf_blocks_to_atoms_kernel(const float* __restrict__ scales, long long nblk, int nk,
                                           uint8_t* __restrict__ atoms) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int nk4 = (nk + 3) / 4;
   const long long n = nblk * nk4 * 32;  // 32 x 16 bytes per atom
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
@@ -120,9 +124,9 @@ cudaError_t launch_sf_rows_to_atoms(const float* scales, int nk, const int32_t* 
   const long long n = max_rows * nk;
   const int grid = static_cast<int>(cdiv(n, 256) < num_sms() * 8LL ? cdiv(n, 256) : num_sms() * 8LL);
   trace_before(MOE_K_SCALE_ATOMS, st);
-  sf_rows_to_atoms_kernel<<<grid > 0 ? grid : 1, 256, 0, st>>>(scales, nk, offsets, G, atoms);
+  const cudaError_t err = launch_k(sf_rows_to_atoms_kernel, grid > 0 ? grid : 1, 256, 0, st, scales, nk, offsets, G, atoms);
   trace_after(MOE_K_SCALE_ATOMS, st);
-  return cudaGetLastError();
+  return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 cudaError_t launch_sf_blocks_to_atoms(const float* scales, long long nblk, int nk, uint8_t* atoms,
@@ -130,9 +134,9 @@ cudaError_t launch_sf_blocks_to_atoms(const float* scales, long long nblk, int n
   const long long n = nblk * ((nk + 3) / 4) * 32;
   const int grid = static_cast<int>(cdiv(n, 256) < num_sms() * 8LL ? cdiv(n, 256) : num_sms() * 8LL);
   trace_before(MOE_K_SCALE_ATOMS, st);
-  sf_blocks_to_atoms_kernel<<<grid > 0 ? grid : 1, 256, 0, st>>>(scales, nblk, nk, atoms);
+  const cudaError_t err = launch_k(sf_blocks_to_atoms_kernel, grid > 0 ? grid : 1, 256, 0, st, scales, nblk, nk, atoms);
   trace_after(MOE_K_SCALE_ATOMS, st);
-  return cudaGetLastError();
+  return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 cudaError_t gemm_gateup_swiglu_fp8(const void* A, const uint8_t* a_atoms, int64_t a_rows,

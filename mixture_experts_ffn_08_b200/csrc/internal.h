@@ -15,6 +15,41 @@ constexpr int kMaxExperts = 1024;
 constexpr int kMaxTopK = 32;
 constexpr int kPermChunk = 256;  // pairs per chunk of the stable bucket ranking
 
+// Programmatic dependent launch of the layer's kernels (api.cu): on unless the
+// environment sets MOE_DISABLE_PDL to a non-empty value other than "0".
+bool pdl_enabled();
+
+// Launches kern<<<grid, block, smem, st>>>(args...) with programmatic stream
+// serialization when pdl_enabled(); every kernel launched this way calls pdl_wait()
+// before it reads or writes global memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                     Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+// K-slices of the router GEMM.  With few output tiles (small T) the reduction over H is
+// split so that about 128 CTAs work; slice s writes its own fp32 partial logits at
+// s * T * E, and the top-k kernel adds the slices in order s = 0, 1, ... (the same sum
+// on every run).  At least 4 K-blocks of 64 per slice.
+inline int router_k_splits(long long T, int H, int E) {
+  const long long tiles = ((T + 127) / 128) * ((E + 255) / 256);
+  const long long kb = H / 64;
+  long long s = tiles > 0 ? 128 / tiles : 1;
+  if (s > kb / 4) s = kb / 4;
+  return s < 1 ? 1 : static_cast<int>(s);
+}
+
 // Tracing (api.cu): brackets a launch of kernel `kid` with events when enabled.
 void trace_before(int kid, cudaStream_t st);
 void trace_after(int kid, cudaStream_t st);
@@ -28,8 +63,9 @@ inline bool act_e4m3(const moe_params_t& p) {
 // ---------------------------------------------------------------- routing (kernels.cu)
 cudaError_t launch_dequant_x(const uint8_t* xq, const float* xs, int T, int H, void* x_bf16,
                              cudaStream_t st);
+// logits: n_part slices of [T, E] fp32 partial sums, summed in slice order.
 cudaError_t launch_topk(const float* logits, const moe_params_t& p, const float* bias,
-                        int32_t* ids, float* w, cudaStream_t st);
+                        int32_t* ids, float* w, cudaStream_t st, int n_part = 1);
 
 // b_e += gamma * sign(mean load - load_e) (aux-free balancing bias).
 cudaError_t launch_bias_update(const int32_t* counts, int E, float gamma, float* bias, cudaStream_t st);
@@ -55,7 +91,8 @@ cudaError_t launch_combine(const moe_params_t& p, const void* y_perm, const int3
                            const float* w, const float* y_shared, void* out, cudaStream_t st);
 
 // ---------------------------------------------------------------- GEMMs (gemm.cu)
-// Router logits [T, E] fp32 = x [T,H] bf16 @ W_r[E,H]^T.
+// Router logits x [T,H] bf16 @ W_r[E,H]^T as router_k_splits(T, H, E) fp32 partial
+// slices [T, E], slice s at logits + s*T*E.
 cudaError_t gemm_router(const void* x, const void* w_r, int T, int H, int E, float* logits,
                         int32_t* status, cudaStream_t st);
 // h [rows, N] bf16 = SiLU(A Wg^T) * (A Wu^T), grouped by offsets (or dense when null);

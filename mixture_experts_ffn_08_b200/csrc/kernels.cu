@@ -22,6 +22,8 @@ constexpr unsigned kFull = 0xffffffffu;
 // Each e4m3 value times its power-of-two scale is exactly representable in bf16.
 __global__ void dequant_x_kernel(const uint8_t* __restrict__ xq, const float* __restrict__ xs,
                                  int T, int H, __nv_bfloat16* __restrict__ xb) {
+  pdl_launch_dependents();
+  pdl_wait();
   const long long n16 = static_cast<long long>(T) * H / 16;
   for (long long v = blockIdx.x * (long long)blockDim.x + threadIdx.x; v < n16;
        v += (long long)gridDim.x * blockDim.x) {
@@ -52,9 +54,10 @@ cudaError_t launch_dequant_x(const uint8_t* xq, const float* xs, int T, int H, v
   const long long n16 = static_cast<long long>(T) * H / 16;
   const int grid = static_cast<int>(n16 / 256 + 1 < num_sms() * 8 ? n16 / 256 + 1 : num_sms() * 8);
   trace_before(MOE_K_DEQUANT_X, st);
-  dequant_x_kernel<<<grid, 256, 0, st>>>(xq, xs, T, H, static_cast<__nv_bfloat16*>(x_bf16));
+  const cudaError_t err = launch_k(dequant_x_kernel, grid, 256, 0, st, xq, xs, T, H,
+                                   static_cast<__nv_bfloat16*>(x_bf16));
   trace_after(MOE_K_DEQUANT_X, st);
-  return cudaGetLastError();
+  return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 // ================================================================== top-k
@@ -94,19 +97,30 @@ MOE_DEVINL float warp_max(float v) {
 // every one of the K rounds is a single warp argmax over the lanes' heads.
 template <int EPL>
 __global__ void __launch_bounds__(128) topk_kernel(
-    const float* __restrict__ logits, int T, int E, int K, int n_group, int topk_group,
+    const float* __restrict__ logits, int n_part, int T, int E, int K, int n_group, int topk_group,
     int group_topn, int score_fn, int renorm, float scale, const float* __restrict__ bias,
     int32_t* __restrict__ ids, float* __restrict__ wout) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int token = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (token >= T) return;  // warp-uniform
   const float* z = logits + static_cast<long long>(token) * E;
+  const long long part_stride = static_cast<long long>(T) * E;
 
+  // logits: the sum of n_part partial slices, added in slice order
   float s[EPL], c[EPL];
 #pragma unroll
   for (int j = 0; j < EPL; ++j) {
     const int e = j * 32 + lane;
     s[j] = e < E ? __ldg(z + e) : -CUDART_INF_F;
+  }
+  for (int part = 1; part < n_part; ++part) {
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) {
+      const int e = j * 32 + lane;
+      if (e < E) s[j] += __ldg(z + part * part_stride + e);
+    }
   }
   if (score_fn == MOE_SCORE_SOFTMAX) {
     float m = -CUDART_INF_F;
@@ -264,15 +278,16 @@ __global__ void __launch_bounds__(128) topk_kernel(
 }
 
 cudaError_t launch_topk(const float* logits, const moe_params_t& p, const float* bias,
-                        int32_t* ids, float* w, cudaStream_t st) {
+                        int32_t* ids, float* w, cudaStream_t st, int n_part) {
   const int grid = (p.T + 3) / 4;
   if (grid == 0) return cudaSuccess;
   const int epl = (p.E + 31) / 32;
   trace_before(MOE_K_TOPK, st);
-#define MOE_TOPK_CASE(N)                                                                   \
-  topk_kernel<N><<<grid, 128, 0, st>>>(logits, p.T, p.E, p.K, p.n_group, p.topk_group,    \
-                                       p.group_topn, p.score_fn, p.renormalize,            \
-                                       p.routed_scale, bias, ids, w)
+  cudaError_t err;
+#define MOE_TOPK_CASE(N)                                                                             \
+  err = launch_k(topk_kernel<N>, grid, 128, 0, st, logits, n_part, p.T, p.E, p.K, p.n_group,         \
+                 p.topk_group, p.group_topn, static_cast<int>(p.score_fn), p.renormalize,            \
+                 p.routed_scale, bias, ids, w)
   if (epl <= 1) MOE_TOPK_CASE(1);
   else if (epl <= 2) MOE_TOPK_CASE(2);
   else if (epl <= 4) MOE_TOPK_CASE(4);
@@ -281,7 +296,7 @@ cudaError_t launch_topk(const float* logits, const moe_params_t& p, const float*
   else MOE_TOPK_CASE(32);
 #undef MOE_TOPK_CASE
   trace_after(MOE_K_TOPK, st);
-  return cudaGetLastError();
+  return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 // ================================================================== aux-free bias
@@ -335,6 +350,8 @@ cudaError_t launch_bounded_wait_selftest(int32_t* status, long long limit_ns, cu
 __global__ void __launch_bounds__(kPermChunk) perm_count_kernel(
     const int32_t* __restrict__ ids, int P, int E, int32_t* __restrict__ chunk_counts,
     int32_t* status) {
+  pdl_launch_dependents();
+  pdl_wait();
   extern __shared__ int hist[];
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
@@ -357,6 +374,8 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t* __restrict__ c
                                                          int32_t* __restrict__ counts,
                                                          int32_t* __restrict__ offsets,
                                                          int32_t* status) {
+  pdl_launch_dependents();
+  pdl_wait();
   __shared__ int warp_tot[32];
   const int e = threadIdx.x, lane = e & 31, w = e >> 5;
   int total = 0;
@@ -406,6 +425,8 @@ constexpr int kRankWarps = 4;
 __global__ void __launch_bounds__(32 * kRankWarps) perm_rank_kernel(
     const int32_t* __restrict__ ids, int P, int E, int cap, const int32_t* __restrict__ chunk_base,
     int32_t* __restrict__ row_of_pair, int32_t* __restrict__ pair_of_row) {
+  pdl_launch_dependents();
+  pdl_wait();
   extern __shared__ int run_cnt[];  // [kRankWarps][E]
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int* my = run_cnt + w * E;
@@ -447,6 +468,8 @@ __global__ void __launch_bounds__(32 * kGatherWarps) perm_gather_kernel(
     const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets,
     int32_t* __restrict__ pair_of_row, void* __restrict__ x_perm,
     float* __restrict__ x_perm_scale, bool zero_pad) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int total = __ldg(offsets + E);
   const int row_bytes = FP8 ? H : 2 * H;
@@ -496,21 +519,23 @@ cudaError_t launch_permute(const moe_params_t& p, int block_m, const int32_t* id
   cudaError_t err;
   if (nchunks > 0) {
     trace_before(MOE_K_PERM_COUNT, st);
-    perm_count_kernel<<<nchunks, kPermChunk, p.E * sizeof(int), st>>>(ids, P, p.E, chunk_counts, status);
+    err = launch_k(perm_count_kernel, nchunks, kPermChunk, p.E * sizeof(int), st, ids, P, p.E, chunk_counts,
+                   status);
     trace_after(MOE_K_PERM_COUNT, st);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    if (err != cudaSuccess || (err = cudaGetLastError()) != cudaSuccess) return err;
   }
   trace_before(MOE_K_PERM_SCAN, st);
-  perm_scan_kernel<<<1, 1024, 0, st>>>(chunk_counts, nchunks, p.E, bm, p.masked_cap, counts, offsets, status);
+  err = launch_k(perm_scan_kernel, 1, 1024, 0, st, chunk_counts, nchunks, p.E, bm, p.masked_cap, counts, offsets,
+                 status);
   trace_after(MOE_K_PERM_SCAN, st);
-  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  if (err != cudaSuccess || (err = cudaGetLastError()) != cudaSuccess) return err;
   if (nchunks > 0) {
     trace_before(MOE_K_PERM_RANK, st);
     const int blocks = (nchunks + kRankWarps - 1) / kRankWarps;
-    perm_rank_kernel<<<blocks, 32 * kRankWarps, kRankWarps * p.E * sizeof(int), st>>>(
-        ids, P, p.E, p.masked_cap, chunk_counts, row_of_pair, pair_of_row);
+    err = launch_k(perm_rank_kernel, blocks, 32 * kRankWarps, kRankWarps * p.E * sizeof(int), st, ids, P, p.E,
+                   p.masked_cap, chunk_counts, row_of_pair, pair_of_row);
     trace_after(MOE_K_PERM_RANK, st);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    if (err != cudaSuccess || (err = cudaGetLastError()) != cudaSuccess) return err;
   }
   const bool masked = p.masked_cap > 0;
   const long long max_rows = masked ? static_cast<long long>(p.E) * p.masked_cap
@@ -519,18 +544,20 @@ cudaError_t launch_permute(const moe_params_t& p, int block_m, const int32_t* id
   const int grid = static_cast<int>(blocks < num_sms() * 8LL ? (blocks > 0 ? blocks : 1) : num_sms() * 8LL);
   trace_before(MOE_K_PERM_GATHER, st);
   if (act_e4m3(p))
-    perm_gather_kernel<true><<<grid, 32 * kGatherWarps, 0, st>>>(x, x_scale, p.H, p.K, p.E, counts, offsets,
-                                                   pair_of_row, x_perm, x_perm_scale, !masked);
+    err = launch_k(perm_gather_kernel<true>, grid, 32 * kGatherWarps, 0, st, x, x_scale, p.H, p.K, p.E, counts,
+                   offsets, pair_of_row, x_perm, x_perm_scale, !masked);
   else
-    perm_gather_kernel<false><<<grid, 32 * kGatherWarps, 0, st>>>(x, x_scale, p.H, p.K, p.E, counts, offsets,
-                                                    pair_of_row, x_perm, x_perm_scale, !masked);
+    err = launch_k(perm_gather_kernel<false>, grid, 32 * kGatherWarps, 0, st, x, x_scale, p.H, p.K, p.E, counts,
+                   offsets, pair_of_row, x_perm, x_perm_scale, !masked);
   trace_after(MOE_K_PERM_GATHER, st);
-  return cudaGetLastError();
+  return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 // sched[e] = sum over j < e of counts[j] rounded up to 128 (one block, E <= 1024).
 __global__ void __launch_bounds__(1024) masked_schedule_kernel(const int32_t* __restrict__ counts, int E,
                                                                int32_t* __restrict__ sched) {
+  pdl_launch_dependents();
+  pdl_wait();
   __shared__ int warp_tot[32];
   const int e = threadIdx.x, lane = e & 31, w = e >> 5;
   const int padded = e < E ? (__ldg(counts + e) + 127) / 128 * 128 : 0;
@@ -558,17 +585,19 @@ __global__ void __launch_bounds__(1024) masked_schedule_kernel(const int32_t* __
 }
 
 cudaError_t launch_masked_schedule(const int32_t* counts, int E, int32_t* sched, cudaStream_t st) {
-  masked_schedule_kernel<<<1, 1024, 0, st>>>(counts, E, sched);
-  return cudaGetLastError();
+  const cudaError_t err = launch_k(masked_schedule_kernel, 1, 1024, 0, st, counts, E, sched);
+  return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 __global__ void masked_offsets_kernel(int E, int cap, int32_t* __restrict__ offsets) {
+  pdl_launch_dependents();
+  pdl_wait();
   for (int e = blockIdx.x * blockDim.x + threadIdx.x; e <= E; e += gridDim.x * blockDim.x) offsets[e] = e * cap;
 }
 
 cudaError_t launch_masked_offsets(int E, int cap, int32_t* offsets, cudaStream_t st) {
-  masked_offsets_kernel<<<(E + 256) / 256, 256, 0, st>>>(E, cap, offsets);
-  return cudaGetLastError();
+  const cudaError_t err = launch_k(masked_offsets_kernel, (E + 256) / 256, 256, 0, st, E, cap, offsets);
+  return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 // ================================================================== combine
@@ -594,6 +623,8 @@ __global__ void __launch_bounds__(128) combine_kernel(
     const YT* __restrict__ y_perm, const int32_t* __restrict__ row_of_pair,
     const float* __restrict__ w, const float* __restrict__ y_sh,
     __nv_bfloat16* __restrict__ out, int T, int H, int K) {
+  pdl_launch_dependents();
+  pdl_wait();
   __shared__ int rows[kMaxTopK];
   __shared__ float wk[kMaxTopK];
   const int nvec = H / 8;  // 8 outputs (one 16-byte store) per thread step
@@ -629,6 +660,8 @@ __global__ void __launch_bounds__(128) combine_kernel(
 }
 
 __global__ void f32_to_bf16_kernel(const float* __restrict__ acc, long long n8, __nv_bfloat16* __restrict__ out) {
+  pdl_launch_dependents();
+  pdl_wait();
   for (long long v = blockIdx.x * (long long)blockDim.x + threadIdx.x; v < n8; v += (long long)gridDim.x * blockDim.x) {
     const float4 a = __ldg(reinterpret_cast<const float4*>(acc) + 2 * v);
     const float4 b = __ldg(reinterpret_cast<const float4*>(acc) + 2 * v + 1);
@@ -643,9 +676,9 @@ cudaError_t launch_f32_to_bf16(const float* acc, long long n, void* out, cudaStr
   const long long want = (n8 + 255) / 256;
   const int grid = static_cast<int>(want < num_sms() * 8LL ? want : num_sms() * 8LL);
   trace_before(MOE_K_COMBINE, st);
-  f32_to_bf16_kernel<<<grid, 256, 0, st>>>(acc, n8, static_cast<__nv_bfloat16*>(out));
+  const cudaError_t err = launch_k(f32_to_bf16_kernel, grid, 256, 0, st, acc, n8, static_cast<__nv_bfloat16*>(out));
   trace_after(MOE_K_COMBINE, st);
-  return cudaGetLastError();
+  return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 cudaError_t launch_combine(const moe_params_t& p, const void* y_perm, const int32_t* row_of_pair,
@@ -653,15 +686,15 @@ cudaError_t launch_combine(const moe_params_t& p, const void* y_perm, const int3
   if (p.T == 0) return cudaSuccess;
   const int grid = p.T < num_sms() * 16 ? p.T : num_sms() * 16;
   trace_before(MOE_K_COMBINE, st);
+  cudaError_t err;
   if (act_e4m3(p))
-    combine_kernel<__nv_bfloat16><<<grid, 128, 0, st>>>(static_cast<const __nv_bfloat16*>(y_perm), row_of_pair,
-                                                        w, y_shared, static_cast<__nv_bfloat16*>(out), p.T,
-                                                        p.H, p.K);
+    err = launch_k(combine_kernel<__nv_bfloat16>, grid, 128, 0, st, static_cast<const __nv_bfloat16*>(y_perm),
+                   row_of_pair, w, y_shared, static_cast<__nv_bfloat16*>(out), p.T, p.H, p.K);
   else
-    combine_kernel<float><<<grid, 128, 0, st>>>(static_cast<const float*>(y_perm), row_of_pair, w, y_shared,
-                                                static_cast<__nv_bfloat16*>(out), p.T, p.H, p.K);
+    err = launch_k(combine_kernel<float>, grid, 128, 0, st, static_cast<const float*>(y_perm), row_of_pair, w,
+                   y_shared, static_cast<__nv_bfloat16*>(out), p.T, p.H, p.K);
   trace_after(MOE_K_COMBINE, st);
-  return cudaGetLastError();
+  return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 }  // namespace moe

@@ -10,7 +10,7 @@
 //   out[r, n] = epilogue( sum_k A[r, k] * B[g*b_rows + n, k] )   for rows r of group g
 //
 // One CTA per SM walks a static list of uniform-cost work items (expert, N-tile,
-// M-tile), ordered expert by expert and, inside an expert, N-tile by N-tile with the
+// M-tile[, K-slice]), ordered expert by expert and, inside an expert, N-tile by N-tile with the
 // expert's M-tiles adjacent: the CTAs running at the same time share each weight tile
 // through L2, and an expert's activation rows stay L2-resident while its N-tiles run.
 // Because all items cost the same, a skewed expert load does not leave a tail.
@@ -62,7 +62,17 @@ struct GemmParams {
   int masked_cap;              // > 0: masked layout.  offsets is then only the schedule (the
                                // compact 128-padded prefix of counts); group g's rows sit at
                                // g * masked_cap in A and out
+  int k_splits;                // > 1 (EPI_F32 only): the K loop of every tile is cut into
+                               // k_splits slices, slice s adding K-blocks
+                               // [s*KB/k_splits, (s+1)*KB/k_splits) into its own output
+  long long split_stride;      // elements between the outputs of consecutive slices
 };
+
+// K-blocks [kb0, kb1) of slice `split` out of `splits` over KB K-blocks.
+MOE_DEVINL void k_slice(int split, int splits, int KB, int& kb0, int& kb1) {
+  kb0 = static_cast<int>(static_cast<long long>(split) * KB / splits);
+  kb1 = static_cast<int>(static_cast<long long>(split + 1) * KB / splits);
+}
 
 MOE_DEVINL void red_add_v4(float* addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d, float w) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(w * __uint_as_float(a)),
@@ -151,11 +161,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   const uint32_t pad = (1024u - (smem_u32(dsmem) & 1023u)) & 1023u;
   uint8_t* smem = dsmem + pad;
 
-  const int num_m_tiles = p.offsets ? (__ldg(p.offsets + p.G) >> 7) : (p.dense_rows + BM - 1) / BM;
   const int NT = (p.N + Cfg::OUT_COLS - 1) / Cfg::OUT_COLS;
-  const int total = num_m_tiles * NT;
   const int KB = p.K / BK;
-  if ((int)blockIdx.x >= total) return;  // uniform across the CTA: nothing allocated yet
+  const int S = p.k_splits > 1 ? p.k_splits : 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -183,6 +191,11 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = tmem_base_sh;
+  // the offsets (and A) come from the kernels before this one
+  pdl_launch_dependents();
+  pdl_wait();
+  const int num_m_tiles = p.offsets ? (__ldg(p.offsets + p.G) >> 7) : (p.dense_rows + BM - 1) / BM;
+  const int total = num_m_tiles * NT * S;  // CTAs past it run no item
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
@@ -192,10 +205,12 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       long long issued = 0;
       bool ok = true;
       for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
-        const TileCoord t = decode_item(item, NT, p, num_m_tiles, BN);
+        const TileCoord t = decode_item(item / S, NT, p, num_m_tiles, BN);
+        int kb0, kb1;
+        k_slice(item % S, S, KB, kb0, kb1);
         const int a_row = t.row0;
         const int b_row = t.group * p.b_rows_per_group + t.n_tile * Cfg::OUT_COLS;
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, &abort_flag)) { ok = false; break; }
           uint8_t* sa = smem + s * Cfg::STAGE_BYTES;
           uint8_t* sb = sa + Cfg::A_BYTES;
@@ -231,7 +246,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         if (!mbar_wait_bounded(&tempty_bar[acc], acc_ph ^ 1u, &abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * Cfg::ACC_COLS;
-        for (int kb = 0; kb < KB; ++kb) {
+        int kb0, kb1;
+        k_slice(item % S, S, KB, kb0, kb1);
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait_bounded(&full_bar[s], ph, &abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a0 = smem_u32(smem + s * Cfg::STAGE_BYTES);
@@ -239,7 +256,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
             umma_f16(d_tmem, smem_desc_sw128(a0 + k * 32), smem_desc_sw128(b0 + k * 32), IDESC,
-                     (kb | k) != 0);
+                     (kb != kb0) || (k != 0));
           }
           umma_commit(&empty_bar[s]);  // frees the stage once these MMAs have read it
           if (++s == STAGES) { s = 0; ph ^= 1u; }
@@ -260,7 +277,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     int acc = 0;
     uint32_t acc_ph = 0;
     for (int item = blockIdx.x; item < total; item += gridDim.x) {
-      const TileCoord t = decode_item(item, NT, p, num_m_tiles, BN);
+      const TileCoord t = decode_item(item / S, NT, p, num_m_tiles, BN);
       // every lane polls, then the warp agrees (tcgen05.ld below is warp-collective)
       const bool ready = __all_sync(0xffffffffu, mbar_wait_bounded(&tfull_bar[acc], acc_ph, &abort_flag));
       if (!ready) break;
@@ -336,7 +353,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           }
         }
       } else if constexpr (BN % 32 == 0) {
-        float* out = static_cast<float*>(p.out) + row * p.ldo + col0;
+        float* out = static_cast<float*>(p.out) + (item % S) * p.split_stride + row * p.ldo + col0;
         const bool v8 = ((reinterpret_cast<uintptr_t>(p.out) | (static_cast<uintptr_t>(p.ldo) * 4)) & 31) == 0;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
@@ -355,7 +372,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           }
         }
       } else {
-        float* out = static_cast<float*>(p.out) + row * p.ldo + col0;
+        float* out = static_cast<float*>(p.out) + (item % S) * p.split_stride + row * p.ldo + col0;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 16) {
           uint32_t r[16];

@@ -213,13 +213,10 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   const uint32_t pad = (1024u - (smem_u32(dsmem) & 1023u)) & 1023u;
   uint8_t* smem = dsmem + pad;
 
-  const int num_pairs = __ldg(p.offsets + p.G) >> 8;
   const int NT = (p.N + Cfg::OUT_COLS - 1) / Cfg::OUT_COLS;
-  const int total = num_pairs * NT;
   const int KB = p.K / BK;
   const int KB4 = (KB + 3) / 4;  // FP8 scale atoms along K (four K steps each)
   const int cluster_id = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
-  if (cluster_id >= total) return;  // same decision in both CTAs of the cluster
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -248,6 +245,12 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   cluster_sync();  // both CTAs: barriers initialised, TMEM allocated
   tc_fence_after();
   const uint32_t tmem_base = tmem_base_sh;
+  // the offsets and A come from the kernels before this one; a cluster past the last
+  // item runs none (the same decision in both of its CTAs)
+  pdl_launch_dependents();
+  pdl_wait();
+  const int num_pairs = __ldg(p.offsets + p.G) >> 8;
+  const int total = num_pairs * NT;
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer (both)

@@ -183,12 +183,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   const uint32_t pad = (1024u - (smem_u32(dsmem) & 1023u)) & 1023u;
   uint8_t* smem = dsmem + pad;
 
-  const int num_m_tiles = __ldg(p.offsets + p.G) >> 7;
   const int NT = (p.N + Cfg::OUT_COLS - 1) / Cfg::OUT_COLS;
-  const int total = num_m_tiles * NT;
   const int KB = p.K / BK;
   const int KB4 = (KB + 3) / 4;  // scale atoms along K (four K steps each)
-  if ((int)blockIdx.x >= total) return;
 
   // the item decoder of the bf16 kernel works on these fields only
   GemmParams gp{};
@@ -223,6 +220,11 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = tmem_base_sh;
+  // the offsets, A and its scale atoms come from the kernels before this one
+  pdl_launch_dependents();
+  pdl_wait();
+  const int num_m_tiles = __ldg(p.offsets + p.G) >> 7;
+  const int total = num_m_tiles * NT;  // CTAs past it run no item
 
   if (warp == 0) {
     // ---------------------------------------------------------------- producer

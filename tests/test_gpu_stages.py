@@ -30,6 +30,11 @@ ROUTE_CASES = {
                                     renormalize=False, routed_scale=1.5),
     "e_1000": W.Workload("e1000", T=50, H=256, I=128, E=1000, K=32, n_group=8, topk_group=5,
                          group_topn=3, has_bias=True),
+    # few output tiles: the router GEMM splits the H reduction into K-slices (28 here)
+    "dsv3_decode_full": W.DSV3_DECODE,
+    # 5 K-slices over 22 K-blocks of 64: slices of 4 and 5 blocks
+    "split_uneven": W.Workload("split5", T=300, H=1408, I=128, E=96, K=4, score_fn=W.SCORE_SIGMOID,
+                               has_bias=True),
 }
 
 
