@@ -14,13 +14,10 @@
 // each word, chosen by the sf-id fields of the instruction descriptor.  Because the
 // layer's scales cover 128 K-elements (four MX sub-blocks of 32), byte b of a word holds
 // the scale of the b-th of four consecutive 128-wide K steps: one atom serves four
-// pipeline stages.  The MMA thread copies atoms to TMEM with tcgen05.cp.32x128b.warpx4
-// (32 lanes x 4 columns, replicated into the four lane quadrants).  Such a copy drains the
-// tensor pipe (measured: ~600-750 cycles when MMAs are in flight), so the atoms of
-// SF_BURST consecutive K steps travel together: the producer brings them in one set of
-// bulk copies into a scale buffer of their own, the MMA thread copies them all to TMEM
-// columns of their own at the first step of the burst, and each MMA addresses the columns
-// of its step; all MMAs of K step kb select byte kb % 4 of the A atom.
+// pipeline stages.  Every fourth stage the producer brings the A atom and one B atom per
+// 128 rows of B next to the A/B tiles (1D bulk copies on the same mbarrier); the MMA
+// thread copies them to TMEM with tcgen05.cp.32x128b.warpx4 (32 lanes x 4 columns,
+// replicated into the four lane quadrants) and all MMAs of K step kb select byte kb % 4.
 //
 // Epilogues:
 //   EPI8_SWIGLU_Q  B = [128 gate rows; 128 up rows]; h = SiLU(gate) * up in fp32, then
@@ -133,24 +130,19 @@ struct Fp8Cfg {
   static constexpr int B_BYTES = BN * BK;                 // smem bytes of the B tile
   static constexpr int B_TX_BYTES = W4 ? B_BYTES / 2 : B_BYTES;  // bytes the TMA counts: packed e2m1
   static constexpr int SFB_ATOMS = BN / 128;
-  static constexpr int SF_BURST = 16;                     // K steps whose atoms travel together
-  static constexpr int A_ATOMS = SF_BURST / 4;             // four-step A atoms per burst
-  static constexpr int B_STEPS = W4 ? SF_BURST : SF_BURST / 4;  // B atoms per burst and 128 B rows
-  static constexpr int SF_BUF_BYTES = 512 * (A_ATOMS + B_STEPS * SFB_ATOMS);
-  static constexpr int STAGE_BYTES = (A_BYTES + B_BYTES + 1023) / 1024 * 1024;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + SF_BUF_BYTES + 1024;
+  static constexpr int SF_BYTES = 512 * (1 + SFB_ATOMS);
+  static constexpr int STAGE_BYTES = (A_BYTES + B_BYTES + SF_BYTES + 1023) / 1024 * 1024;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
   static constexpr int OUT_COLS = EPI == EPI8_SWIGLU_Q ? BN / 2 : BN;
   // TMEM holds 512 columns: two 256-column accumulators would leave none for the scales,
   // so 256-column tiles keep one and their epilogue hands it back as soon as it is read.
   static constexpr int ACC_STAGES = BN == 256 ? 1 : 2;
   static constexpr int ACC_COLS = BN;
-  static constexpr int SF_COL = ACC_STAGES * ACC_COLS;      // A atoms of a burst (4 columns each)
-  static constexpr int SFB_COL = SF_COL + 4 * A_ATOMS;      // then B: step (or group) j, block a
-                                                            // at 4 * (j * SFB_ATOMS + a)
+  static constexpr int SF_COL = ACC_STAGES * ACC_COLS;      // A scales; B scales at +4
   static constexpr int TMEM_COLS = 512;
   static constexpr int THREADS = 192;
   static_assert(BN % 128 == 0 && BN <= 256, "B tile rows in whole 128-row scale atoms");
-  static_assert(SFB_COL + 4 * B_STEPS * SFB_ATOMS <= TMEM_COLS, "TMEM columns");
+  static_assert(SF_COL + 4 + 4 * SFB_ATOMS <= TMEM_COLS, "TMEM columns");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
   static_assert(EPI != EPI8_SWIGLU_Q || BN == 256, "SwiGLU tile = 128 gate + 128 up rows");
 };
@@ -182,7 +174,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 
   extern __shared__ uint8_t dsmem[];
   __shared__ uint64_t full_bar[STAGES], empty_bar[STAGES];
-  __shared__ uint64_t tfull_bar[2], tempty_bar[2], drain_bar, sf_full_bar, sf_empty_bar;
+  __shared__ uint64_t tfull_bar[2], tempty_bar[2], drain_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
   __shared__ int no_abort_sh[2];
@@ -190,7 +182,6 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
   const int warp = warp_id(), lane = lane_id();
   const uint32_t pad = (1024u - (smem_u32(dsmem) & 1023u)) & 1023u;
   uint8_t* smem = dsmem + pad;
-  uint8_t* sf_buf = smem + STAGES * Cfg::STAGE_BYTES;  // the scale atoms of one burst
 
   const int NT = (p.N + Cfg::OUT_COLS - 1) / Cfg::OUT_COLS;
   const int KB = p.K / BK;
@@ -212,8 +203,6 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       mbar_init(&tempty_bar[a], 128);
     }
     mbar_init(&drain_bar, 1);
-    mbar_init(&sf_full_bar, 1);
-    mbar_init(&sf_empty_bar, 1);
     abort_flag = 0;
     no_abort_sh[0] = no_abort_sh[1] = 0;
     fence_mbar_init();
@@ -241,50 +230,46 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
       int s = 0;
-      uint32_t ph = 0, sf_ph = 0;
-      long long issued = 0, sf_issued = 0;
+      uint32_t ph = 0;
+      long long issued = 0;
       bool ok = true;
       const int nblk = p.N / 128;  // 128-row weight blocks per group
-      const int wsteps = Cfg::W4 ? KB : KB4;  // weight atoms per 128-row block along K
       for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
         const TileCoord t = decode_item(item, NT, gp, num_m_tiles, BN);
         const int a_row = t.row0;
         const int b_row = t.group * p.N + t.n_tile * Cfg::OUT_COLS;
         const int wblk = t.group * nblk + (t.n_tile * Cfg::OUT_COLS) / 128;
         for (int kb = 0; kb < KB; ++kb) {
-          if (kb % Cfg::SF_BURST == 0) {
-            // the atoms of K steps [kb, kb + n): ng four-step A atoms, then per 128-row block
-            // of B its m atoms (one per step for e2m1, per four steps for e4m3)
-            const int n = KB - kb < Cfg::SF_BURST ? KB - kb : Cfg::SF_BURST;
-            const int ng = (n + 3) >> 2;
-            const int m = Cfg::W4 ? n : ng;
-            const int first = Cfg::W4 ? kb : kb >> 2;
-            if (!mbar_wait_bounded(&sf_empty_bar, sf_ph ^ 1u, &abort_flag)) { ok = false; break; }
-            mbar_arrive_expect_tx(&sf_full_bar, 512u * (ng + m * Cfg::SFB_ATOMS));
-            bulk_load(sf_buf, p.sfa + (static_cast<size_t>(t.row0 / BM) * KB4 + (kb >> 2)) * 512, 512u * ng,
-                      &sf_full_bar);
-#pragma unroll
-            for (int a = 0; a < Cfg::SFB_ATOMS; ++a) {
-              // weight atoms [128-row block][K step (e2m1) or four K steps (e4m3)][512 B];
-              // SwiGLU's second block is the up projection's own atom array
-              const uint8_t* src = Cfg::EPI == EPI8_SWIGLU_Q
-                                       ? (a == 0 ? p.sfb0 : p.sfb1) + (static_cast<size_t>(wblk) * wsteps + first) * 512
-                                       : p.sfb0 + (static_cast<size_t>(wblk + a) * wsteps + first) * 512;
-              bulk_load(sf_buf + 512 * (ng + a * m), src, 512u * m, &sf_full_bar);
-            }
-            ++sf_issued;
-            sf_ph ^= 1u;
-          }
           if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, &abort_flag)) { ok = false; break; }
           uint8_t* sa = smem + s * Cfg::STAGE_BYTES;
           uint8_t* sb = sa + Cfg::A_BYTES;
-          mbar_arrive_expect_tx(&full_bar[s], Cfg::A_BYTES + Cfg::B_TX_BYTES);
+          uint8_t* ssf = sb + Cfg::B_BYTES;
+          const bool new_sf = (kb & 3) == 0;            // A atoms: one per four K steps
+          const bool new_sfb = Cfg::W4 || new_sf;        // B atoms: every step for e2m1
+          mbar_arrive_expect_tx(&full_bar[s], Cfg::A_BYTES + Cfg::B_TX_BYTES + (new_sf ? 512 : 0) +
+                                                  (new_sfb ? 512 * Cfg::SFB_ATOMS : 0));
           tma_load_2d(sa, &tmA, kb * BK, a_row, &full_bar[s]);
           if (Cfg::EPI == EPI8_SWIGLU_Q) {
             tma_load_2d(sb, &tmB0, kb * BK, b_row, &full_bar[s]);
             tma_load_2d(sb + 128 * BK, &tmB1, kb * BK, b_row, &full_bar[s]);
           } else {
             tma_load_2d(sb, &tmB0, kb * BK, b_row, &full_bar[s]);
+          }
+          if (new_sf)
+            bulk_load(ssf, p.sfa + (static_cast<size_t>(t.row0 / BM) * KB4 + (kb >> 2)) * 512, 512, &full_bar[s]);
+          if (new_sfb) {
+            // weight atoms [128-row block][K step (e2m1) or four K steps (e4m3)][512 B]
+            const int steps = Cfg::W4 ? KB : KB4;
+            const size_t wsf = (static_cast<size_t>(wblk) * steps + (Cfg::W4 ? kb : kb >> 2)) * 512;
+            if (Cfg::EPI == EPI8_SWIGLU_Q) {
+              bulk_load(ssf + 512, p.sfb0 + wsf, 512, &full_bar[s]);
+              bulk_load(ssf + 1024, p.sfb1 + wsf, 512, &full_bar[s]);
+            } else {
+#pragma unroll
+              for (int a = 0; a < Cfg::SFB_ATOMS; ++a)
+                bulk_load(ssf + 512 * (1 + a), p.sfb0 + wsf + static_cast<size_t>(a) * steps * 512, 512,
+                          &full_bar[s]);
+            }
           }
           ++issued;
           if (++s == STAGES) { s = 0; ph ^= 1u; }
@@ -296,55 +281,41 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         if (s == 0) { s = STAGES - 1; ph ^= 1u; } else { --s; }
         mbar_wait_bounded(&full_bar[s], ph, no_abort);
       }
-      // the last burst of atoms has landed too (it has, unless the pipeline was aborted)
-      if (sf_issued > 0) mbar_wait_bounded(&sf_full_bar, sf_ph ^ 1u, no_abort);
       if (!ok || *no_abort) abort_flag = 1;
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       int s = 0, acc = 0;
-      uint32_t ph = 0, acc_ph = 0, sf_ph = 0;
+      uint32_t ph = 0, acc_ph = 0;
       bool ok = true;
       const uint32_t sfa_t = tmem_base + Cfg::SF_COL;
-      const uint32_t sfb_t = tmem_base + Cfg::SFB_COL;
-      const uint32_t sf0 = smem_u32(sf_buf);
+      const uint32_t sfb_t = sfa_t + 4;
       for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
         if (!mbar_wait_bounded(&tempty_bar[acc], acc_ph ^ 1u, &abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * Cfg::ACC_COLS;
         for (int kb = 0; kb < KB; ++kb) {
-          if (kb % Cfg::SF_BURST == 0) {
-            // the burst's atoms into TMEM in one go (tcgen05.cp and tcgen05.mma of one thread
-            // run in issue order, so the MMAs of the previous burst still read the old
-            // columns); the commit frees the scale buffer once the copies are done
-            if (!mbar_wait_bounded(&sf_full_bar, sf_ph, &abort_flag)) { ok = false; break; }
-            tc_fence_after();
-            const int n = KB - kb < Cfg::SF_BURST ? KB - kb : Cfg::SF_BURST;
-            const int ng = (n + 3) >> 2;
-            const int m = Cfg::W4 ? n : ng;
-            for (int g = 0; g < ng; ++g) tmem_cp_32x128b_warpx4(sfa_t + 4 * g, smem_desc_rows16(sf0 + 512 * g));
-            for (int a = 0; a < Cfg::SFB_ATOMS; ++a)
-              for (int j = 0; j < m; ++j)
-                tmem_cp_32x128b_warpx4(sfb_t + 4 * (j * Cfg::SFB_ATOMS + a),
-                                       smem_desc_rows16(sf0 + 512 * (ng + a * m + j)));
-            umma_commit(&sf_empty_bar);
-            sf_ph ^= 1u;
-          }
           if (!mbar_wait_bounded(&full_bar[s], ph, &abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a0 = smem_u32(smem + s * Cfg::STAGE_BYTES);
           const uint32_t b0 = a0 + Cfg::A_BYTES;
-          const int l = kb % Cfg::SF_BURST;  // step inside the burst
-          const uint32_t sfa_k = sfa_t + 4 * (l >> 2);
-          const uint32_t sfb_k = sfb_t + 4 * Cfg::SFB_ATOMS * (Cfg::W4 ? l : l >> 2);
+          const uint32_t sf0 = b0 + Cfg::B_BYTES;
+          // new scale atoms into TMEM (tcgen05.cp and tcgen05.mma of one thread run in
+          // issue order, so the MMAs of earlier steps still read the old columns)
+          if ((kb & 3) == 0) tmem_cp_32x128b_warpx4(sfa_t, smem_desc_rows16(sf0));
+          if (Cfg::W4 || (kb & 3) == 0) {
+#pragma unroll
+            for (int a = 0; a < Cfg::SFB_ATOMS; ++a)
+              tmem_cp_32x128b_warpx4(sfb_t + 4 * a, smem_desc_rows16(sf0 + 512 * (1 + a)));
+          }
 #pragma unroll
           for (int kk = 0; kk < BK / 32; ++kk) {
             // A: byte kb%4 (one scale per 128 K); B: byte kk of this step's atom (e2m1,
             // one scale per 32 K) or byte kb%4 (e4m3)
             const uint32_t idesc = Cfg::W4 ? idesc_mxf8_e4m3(BM, BN, kb & 3, kk, kFmtE2M1)
                                            : idesc_mxf8_e4m3(BM, BN, kb & 3, kb & 3);
-            umma_mxf8(d_tmem, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32), idesc, sfa_k, sfb_k,
+            umma_mxf8(d_tmem, smem_desc_sw128(a0 + kk * 32), smem_desc_sw128(b0 + kk * 32), idesc, sfa_t, sfb_t,
                       (kb | kk) != 0);
           }
           umma_commit(&empty_bar[s]);
