@@ -220,7 +220,9 @@ def summarize_clock_rows(lines, window=None):
     names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
     reasons = sorted({names[i] for r in use for i in range(4) if r[6 + i] == "Active"})
     loaded = [v for v in sm if smax and v > 0.5 * max(smax)] or sm
+    pw = [float(r[4]) for r in use if _is_num(r[4])]
     return {"sm_mhz": statistics.median(loaded) if loaded else None,
+            "power_w_median": statistics.median(pw) if pw else None,
             "sm_mhz_min": min(loaded) if loaded else None,
             "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
             "sw_power_cap_samples": sum(1 for r in use if r[9] == "Active"),

@@ -124,6 +124,7 @@ cudaError_t gemm_gateup_swiglu(const void* A, int64_t a_rows, const int32_t* off
   gp.ldo = N;
   gp.status = status;
   gp.masked_cap = masked_cap;
+  gp.half_tiles = 1;
   const long long items = ceil_div(a_rows, 128) * ceil_div(N, Cfg::OUT_COLS);
   return launch<Cfg>(ta, tg, tu, gp, items, kid, st);
 }
@@ -148,6 +149,7 @@ cudaError_t gemm_down(const void* A, int64_t a_rows, const int32_t* offsets,
   gp.ldo = N;
   gp.status = status;
   gp.masked_cap = masked_cap;
+  gp.half_tiles = 1;
   if (wide) {
     using Cfg = GemmCfg<256, EPI_F32, 4>;
     return launch<Cfg>(ta, tb, tb, gp, ceil_div(a_rows, 128) * ceil_div(N, 256), kid, st);
@@ -180,6 +182,7 @@ cudaError_t gemm_down_combine(const void* A, int64_t a_rows, const int32_t* offs
   gp.pair_weight = pair_weight;
   gp.topk = topk;
   gp.masked_cap = masked_cap;
+  gp.half_tiles = 1;
   if (wide) {
     using Cfg = GemmCfg<256, EPI_COMBINE, 4>;
     return launch<Cfg>(ta, tb, tb, gp, ceil_div(a_rows, 128) * ceil_div(N, 256), MOE_K_DOWN, st);

@@ -66,6 +66,8 @@ struct GemmParams {
                                // k_splits slices, slice s adding K-blocks
                                // [s*KB/k_splits, (s+1)*KB/k_splits) into its own output
   long long split_stride;      // elements between the outputs of consecutive slices
+  int half_tiles;              // 1 (grouped, with counts): an M-tile holding at most 64 real
+                               // rows runs M=64 MMAs over its first 64 rows
 };
 
 // K-blocks [kb0, kb1) of slice `split` out of `splits` over KB K-blocks.
@@ -138,6 +140,14 @@ MOE_DEVINL TileCoord decode_item(int item, int NT, const GemmParams& p, int num_
   t.local0 = (t.m_tile - mt0) * 128;
   t.row0 = p.masked_cap > 0 ? g * p.masked_cap + t.local0 : t.m_tile * 128;
   return t;
+}
+
+// Whether tile t runs M=64 MMAs: its group has at most 64 real rows from the tile's first
+// row on.  The M=64 accumulator of a one-SM MMA holds tile row 16i + j in TMEM lane
+// 32i + j (j < 16): lanes 0-15 of each 32-lane quadrant.
+MOE_DEVINL bool half_tile(const TileCoord& t, const GemmParams& p) {
+  return p.half_tiles && p.offsets != nullptr && p.counts != nullptr &&
+         __ldg(p.counts + t.group) - t.local0 <= 64;
 }
 
 MOE_DEVINL float silu_mul(float g, float u) {
@@ -248,6 +258,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         const uint32_t d_tmem = tmem_base + acc * Cfg::ACC_COLS;
         int kb0, kb1;
         k_slice(item % S, S, KB, kb0, kb1);
+        const uint32_t idesc = half_tile(decode_item(item / S, NT, p, num_m_tiles, BN), p)
+                                   ? idesc_bf16_f32(64, BN) : IDESC;
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait_bounded(&full_bar[s], ph, &abort_flag)) { ok = false; break; }
           tc_fence_after();
@@ -255,7 +267,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
           const uint32_t b0 = a0 + Cfg::A_BYTES;
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
-            umma_f16(d_tmem, smem_desc_sw128(a0 + k * 32), smem_desc_sw128(b0 + k * 32), IDESC,
+            umma_f16(d_tmem, smem_desc_sw128(a0 + k * 32), smem_desc_sw128(b0 + k * 32), idesc,
                      (kb != kb0) || (k != 0));
           }
           umma_commit(&empty_bar[s]);  // frees the stage once these MMAs have read it
@@ -283,11 +295,13 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
       if (!ready) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * Cfg::ACC_COLS;
-      const long long row = static_cast<long long>(t.row0) + q * 32 + lane;
+      const bool half = half_tile(t, p);
+      const int trow = half ? q * 16 + lane : q * 32 + lane;  // tile row held by this lane
+      const long long row = static_cast<long long>(t.row0) + trow;
       bool row_ok;
       if (p.offsets == nullptr) row_ok = row < p.dense_rows;
       else if (p.counts == nullptr) row_ok = true;
-      else row_ok = t.local0 + q * 32 + lane < __ldg(p.counts + t.group);
+      else row_ok = (!half || lane < 16) && t.local0 + trow < __ldg(p.counts + t.group);
       const int col0 = t.n_tile * Cfg::OUT_COLS;
 
       if constexpr (Cfg::EPI == EPI_SWIGLU) {
