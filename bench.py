@@ -66,25 +66,41 @@ def sources_sha256(files):
     return h.hexdigest()
 
 
-def _profiled_traffic(workload, sources=GEMM_SOURCES):
-    """DRAM bytes per launch of the gate/up kernel from the committed ncu summary of this
-    workload, or None if there is none, it covers another kernel than `sources` (the
-    files of the kernel that runs now), or those sources changed since it was taken.  The
-    summary names the sources it covers (kernel_sources:, default the bf16 GEMM)."""
+def _profiled_traffic(workload, sources=GEMM_SOURCES, algorithmic_bytes=None):
+    """(DRAM bytes per launch of the gate/up kernel, where the figure comes from), from the
+    committed ncu summary of this workload; (None, reason) if there is none, it covers
+    another kernel than `sources` (the files of the kernel that runs now), or those
+    sources changed since it was taken.  A summary gives either the bytes of a full-size
+    capture (traffic_bytes_per_launch:) or, for a workload too large to capture, the
+    ratio of DRAM bytes to algorithmic bytes measured on a smaller case of the same
+    kernel (traffic_per_algorithmic_byte:, scaled_from:), which is applied to this run's
+    algorithmic bytes.  The summary names the sources it covers (kernel_sources:,
+    default the bf16 GEMM)."""
     import re
     path = os.path.join(ROOT, "profiles", f"gateup_swiglu_{workload}.md")
     if not os.path.exists(path):
-        return None
+        return None, "no ncu summary for this workload"
     txt = open(path, encoding="utf-8").read()
     m_t = re.search(r"^traffic_bytes_per_launch:\s*(\d+)", txt, re.M)
+    m_r = re.search(r"^traffic_per_algorithmic_byte:\s*([0-9.]+)", txt, re.M)
+    m_f = re.search(r"^scaled_from:\s*(.+)$", txt, re.M)
     m_h = re.search(r"^kernel_source_sha256:\s*([0-9a-f]+)", txt, re.M)
     m_s = re.search(r"^kernel_sources:\s*(.+)$", txt, re.M)
-    if not (m_t and m_h):
-        return None
+    if not ((m_t or m_r) and m_h):
+        return None, "ncu summary without a traffic figure"
     files = [f.strip() for f in m_s.group(1).split(",")] if m_s else list(GEMM_SOURCES)
     if files != list(sources):
-        return None
-    return int(m_t.group(1)) if sources_sha256(files) == m_h.group(1) else None
+        return None, "ncu summary covers another kernel"
+    if sources_sha256(files) != m_h.group(1):
+        return None, "kernel sources changed since the ncu capture"
+    if m_t:
+        return int(m_t.group(1)), f"ncu capture of {workload} (profiles/gateup_swiglu_{workload}.md)"
+    if algorithmic_bytes is None:
+        return None, "scaled figure needs the algorithmic bytes"
+    ratio = float(m_r.group(1))
+    return int(ratio * algorithmic_bytes), (f"DRAM/algorithmic bytes {ratio:.4f} measured on "
+                                            f"{m_f.group(1).strip() if m_f else 'a smaller case'}, "
+                                            f"times this launch's algorithmic bytes")
 
 
 def _peaks():
@@ -539,8 +555,9 @@ def measure(wl, steps, warmup, world=1, rank=0, local=0, cpu=True, adapt_steps=F
     dt_name = "e4m3 x e2m1" if w4 else ("e4m3" if fp8 else "bf16")
     dom_ms = [ms for k, ms in traced if k == dominant]
     roofline = roofline_record(flops["gateup_swiglu"], bytes_gateup, dom_ms, clk, fp8, _peaks())
+    traffic, traffic_src = _profiled_traffic(wl.name, gateup_sources(wl), bytes_gateup)
     roofline.update({"kernel": f"gateup_swiglu (grouped GEMM, fused SwiGLU, {dt_name})",
-                     "traffic": _profiled_traffic(wl.name, gateup_sources(wl))})
+                     "traffic": traffic, "traffic_source": traffic_src})
     peak_t = _gemm_peak(wl)
     hbm_peak = _peaks()[2]
     gemm_ms = sum(kernel_ms.get(k, 0.0) for k in flops)

@@ -66,11 +66,16 @@ def test_profiled_traffic_only_for_the_kernel_it_covers(tmp_path, monkeypatch):
     sha = bench.sources_sha256(["csrc/a.cuh", "csrc/b.cu"])
     (tmp_path / "profiles" / "gateup_swiglu_w.md").write_text(
         f"traffic_bytes_per_launch: 1234\nkernel_sources: csrc/a.cuh, csrc/b.cu\nkernel_source_sha256: {sha}\n")
-    assert bench._profiled_traffic("w", ("csrc/a.cuh", "csrc/b.cu")) == 1234
-    assert bench._profiled_traffic("w", ("csrc/a.cuh",)) is None          # another kernel runs now
+    (tmp_path / "profiles" / "gateup_swiglu_big.md").write_text(
+        f"traffic_per_algorithmic_byte: 1.25\nscaled_from: small case\n"
+        f"kernel_sources: csrc/a.cuh, csrc/b.cu\nkernel_source_sha256: {sha}\n")
+    assert bench._profiled_traffic("w", ("csrc/a.cuh", "csrc/b.cu"))[0] == 1234
+    t, src = bench._profiled_traffic("big", ("csrc/a.cuh", "csrc/b.cu"), 1000)
+    assert t == 1250 and "small case" in src
+    assert bench._profiled_traffic("w", ("csrc/a.cuh",))[0] is None          # another kernel runs now
     (pkg / "b.cu").write_text("// changed\n")
-    assert bench._profiled_traffic("w", ("csrc/a.cuh", "csrc/b.cu")) is None  # sources changed
-    assert bench._profiled_traffic("none", ("csrc/a.cuh",)) is None
+    assert bench._profiled_traffic("w", ("csrc/a.cuh", "csrc/b.cu"))[0] is None  # sources changed
+    assert bench._profiled_traffic("none", ("csrc/a.cuh",))[0] is None
 
 
 def _smi_line(ts, sm, reason_cap="Not Active", smax=1965):
