@@ -60,7 +60,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 5
+#define MOE_ABI_VERSION 6
 
 typedef enum moe_status {
   MOE_OK = 0,
@@ -119,8 +119,9 @@ typedef struct moe_params {
  * this much).  0 if the parameters are invalid. */
 size_t moe_workspace_size(const moe_params_t* p);
 
-/* Bytes of workspace moe_layer_forward_host() needs: moe_workspace_size() plus device
- * staging for the copied activations and output.  0 if the parameters are invalid. */
+/* Bytes of workspace moe_layer_forward_host() and moe_layer_forward_host_batches() need:
+ * moe_workspace_size() plus two device staging slots for the copied activations and
+ * outputs.  0 if the parameters are invalid. */
 size_t moe_workspace_size_host(const moe_params_t* p);
 
 /* Bucket alignment the calls use for these parameters (128 or 256); -1 if invalid. */
@@ -265,6 +266,26 @@ moe_status_t moe_layer_forward_host(const moe_params_t* p, const void* x_host,
                                     const void* ws_gate, const void* ws_up,
                                     const void* ws_down, void* out_host, void* ws,
                                     size_t ws_bytes, void* stream);
+
+/* The same layer over n_batches independent batches of T tokens, each from and to host
+ * memory: batch b's x_host[b] (and x_scale_host[b] for FP8) is copied in, the layer
+ * runs, and its output is copied to out_host[b].  The copies run on two copy streams of
+ * the library's own and overlap the device work of the neighbouring batches (two device
+ * staging slots in ws, so batch b+1 is copied in and batch b-1 copied out while batch b
+ * runs); the layer itself runs on `stream`.  The call enqueues everything and returns;
+ * `stream` passes the call once every output copy has finished, and the first copy in
+ * starts after the work already on `stream`.  Arrays x_host, x_scale_host (FP8 only,
+ * else NULL) and out_host hold n_batches host pointers each; the same pointer may
+ * repeat.  Host buffers must be pinned for the copies to overlap and must stay valid
+ * until `stream` has passed the call.  ws must hold moe_workspace_size_host() bytes.
+ * Calls on one device share the copy streams.  n_batches = 0 does nothing. */
+moe_status_t moe_layer_forward_host_batches(const moe_params_t* p, int32_t n_batches,
+                                            const void* const* x_host, const float* const* x_scale_host,
+                                            const void* w_r, const float* bias, const void* w_gate,
+                                            const void* w_up, const void* w_down, const void* w_gate_scale,
+                                            const void* w_up_scale, const void* w_down_scale,
+                                            const void* ws_gate, const void* ws_up, const void* ws_down,
+                                            void* const* out_host, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------- */
 /* e2m1 weight scales ("DeepGEMM质变…" §5.3 FP8 x FP4 GEMM; §一 1.3 lays the UE8M0 scale */

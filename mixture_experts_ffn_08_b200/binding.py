@@ -72,6 +72,7 @@ _SIGS = {
     "moe_combine": (ctypes.c_int, [_PP, _P, _P, _P, _P, _P, _P]),
     "moe_layer_forward": (ctypes.c_int, [_PP] + [_P] * 18 + [ctypes.c_size_t, _P]),
     "moe_layer_forward_host": (ctypes.c_int, [_PP] + [_P] * 15 + [ctypes.c_size_t, _P]),
+    "moe_layer_forward_host_batches": (ctypes.c_int, [_PP, ctypes.c_int32] + [_P] * 15 + [ctypes.c_size_t, _P]),
     "moe_get_device_status": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_int32)]),
     "moe_clear_device_status": (ctypes.c_int, [_P, _P]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -220,6 +221,30 @@ def moe_layer_forward_host(p, x_host, x_scale_host, w_r, bias, w_gate, w_up, w_d
         _ptr(w_up), _ptr(w_down), _ptr(w_gate_scale), _ptr(w_up_scale), _ptr(w_down_scale),
         _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), _ptr(out_host), _ptr(ws), ws_bytes,
         _stream(stream))
+
+
+def _ptr_array(items):
+    """ctypes array of void* from tensors / addresses / None (NULL), or NULL if items is None."""
+    if items is None:
+        return None
+    arr = (ctypes.c_void_p * len(items))(*[_ptr(t) for t in items])
+    return ctypes.cast(arr, ctypes.c_void_p).value, arr
+
+
+def moe_layer_forward_host_batches(p, x_host, x_scale_host, w_r, bias, w_gate, w_up, w_down, w_gate_scale,
+                                   w_up_scale, w_down_scale, ws_gate, ws_up, ws_down, out_host, ws,
+                                   ws_bytes, stream=None) -> int:
+    """x_host, x_scale_host (or None) and out_host are lists of host tensors, one per batch."""
+    n = len(x_host)
+    if len(out_host) != n or (x_scale_host is not None and len(x_scale_host) != n):
+        raise ValueError("one x, x_scale and out buffer per batch")
+    xs = _ptr_array(x_host)
+    ss = _ptr_array(x_scale_host)
+    os_ = _ptr_array(out_host)
+    return lib().moe_layer_forward_host_batches(
+        ctypes.byref(p), n, xs[0], ss[0] if ss else None, _ptr(w_r), _ptr(bias), _ptr(w_gate), _ptr(w_up),
+        _ptr(w_down), _ptr(w_gate_scale), _ptr(w_up_scale), _ptr(w_down_scale), _ptr(ws_gate), _ptr(ws_up),
+        _ptr(ws_down), os_[0], _ptr(ws), ws_bytes, _stream(stream))
 
 
 # ------------------------------------------------------------------ status, tracing

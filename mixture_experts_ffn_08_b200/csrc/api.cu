@@ -90,6 +90,46 @@ const Side* side_for_current_device() {
 }
 }  // namespace
 
+// ------------------------------------------------------------------ copy streams
+// moe_layer_forward_host_batches copies activations in on one stream and outputs out on
+// another, both the library's own (non-blocking, made on first use per device and kept
+// until exit), ordered against the layer's kernels on the caller's stream by events: per
+// staging slot, `in` (activations landed), `done` (the layer has read them and written its
+// output) and `out` (the output has left the slot).
+namespace {
+struct Copies {
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t fork = nullptr;
+  cudaEvent_t landed[2] = {nullptr, nullptr}, done[2] = {nullptr, nullptr}, left[2] = {nullptr, nullptr};
+};
+std::mutex g_copy_mu;  // held while a call enqueues, so calls' event records do not interleave
+Copies g_copies[64];
+
+const Copies* copies_for_current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  Copies& c = g_copies[dev];
+  if (c.in != nullptr) return &c;
+  Copies n;
+  bool ok = cudaStreamCreateWithFlags(&n.in, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaStreamCreateWithFlags(&n.out, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaEventCreateWithFlags(&n.fork, cudaEventDisableTiming) == cudaSuccess;
+  for (int s = 0; s < 2 && ok; ++s)
+    ok = cudaEventCreateWithFlags(&n.landed[s], cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&n.done[s], cudaEventDisableTiming) == cudaSuccess &&
+         cudaEventCreateWithFlags(&n.left[s], cudaEventDisableTiming) == cudaSuccess;
+  if (!ok) {
+    if (n.in) cudaStreamDestroy(n.in);
+    if (n.out) cudaStreamDestroy(n.out);
+    for (cudaEvent_t e : {n.fork, n.landed[0], n.landed[1], n.done[0], n.done[1], n.left[0], n.left[1]})
+      if (e) cudaEventDestroy(e);
+    return nullptr;
+  }
+  c = n;
+  return &c;
+}
+}  // namespace
+
 // ------------------------------------------------------------------ tracing
 namespace {
 struct Trace {
@@ -131,7 +171,7 @@ struct Layout {
   size_t status, logits, xb, ids, w, counts, offsets, sched, row_of_pair, pair_of_row, chunk_counts;
   size_t x_perm, x_perm_scale, h, y_perm, h_sh, y_sh, total;
   size_t x_atoms, h_atoms, wg_atoms, wu_atoms, wd_atoms;
-  size_t x_stage, x_scale_stage, out_stage, total_host;
+  size_t x_stage[2], x_scale_stage[2], out_stage[2], total_host;
   long long max_rows;
 };
 
@@ -185,9 +225,11 @@ Layout layout(const moe_params_t* p) {
   L.wu_atoms = take(w8 ? E * (I / 128) * hk4 * 512 : 0);
   L.wd_atoms = take(w8 ? E * (H / 128) * ik4 * 512 : 0);
   L.total = o;
-  L.x_stage = take(T * H * xelem);
-  L.x_scale_stage = take(is_fp8(p) ? T * (H / 128) * 4 : 0);
-  L.out_stage = take(T * H * 2);
+  for (int slot = 0; slot < 2; ++slot) {  // host entry points: two device staging slots
+    L.x_stage[slot] = take(T * H * xelem);
+    L.x_scale_stage[slot] = take(is_fp8(p) ? T * (H / 128) * 4 : 0);
+    L.out_stage[slot] = take(T * H * 2);
+  }
   L.total_host = o;
   return L;
 }
@@ -624,9 +666,9 @@ moe_status_t moe_layer_forward_host(const moe_params_t* p, const void* x_host, c
   if (is_fp8(p) && !x_scale_host) return MOE_ERR_INVALID_ARG;
   if (!weight_scales_ok(p, w_gate_scale, w_up_scale, w_down_scale)) return MOE_ERR_INVALID_ARG;
   const Layout L = layout(p);
-  void* x_dev = at<void>(ws, L.x_stage);
-  float* xs_dev = is_fp8(p) ? at<float>(ws, L.x_scale_stage) : nullptr;
-  void* out_dev = at<void>(ws, L.out_stage);
+  void* x_dev = at<void>(ws, L.x_stage[0]);
+  float* xs_dev = is_fp8(p) ? at<float>(ws, L.x_scale_stage[0]) : nullptr;
+  void* out_dev = at<void>(ws, L.out_stage[0]);
   MOE_TRY(check_layer_args(p, x_dev, xs_dev, w_r, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, out_dev));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t xbytes = static_cast<size_t>(p->T) * p->H * (is_fp8(p) ? 1 : 2);
@@ -638,6 +680,65 @@ moe_status_t moe_layer_forward_host(const moe_params_t* p, const void* x_host, c
                    ws_gate, ws_up, ws_down, out_dev, nullptr, nullptr, nullptr, ws, st));
   MOE_CUDA(cudaMemcpyAsync(out_host, out_dev, static_cast<size_t>(p->T) * p->H * 2, cudaMemcpyDeviceToHost, st));
   return MOE_OK;
+}
+
+moe_status_t moe_layer_forward_host_batches(const moe_params_t* p, int32_t n_batches, const void* const* x_host,
+                                            const float* const* x_scale_host, const void* w_r, const float* bias,
+                                            const void* w_gate, const void* w_up, const void* w_down,
+                                            const void* w_gate_scale, const void* w_up_scale,
+                                            const void* w_down_scale, const void* ws_gate, const void* ws_up,
+                                            const void* ws_down, void* const* out_host, void* ws, size_t ws_bytes,
+                                            void* stream) {
+  MOE_TRY(validate(p));
+  MOE_TRY(check_ws(p, ws, ws_bytes, true));
+  if (n_batches < 0) return MOE_ERR_INVALID_ARG;
+  if (n_batches == 0 || p->T == 0) return MOE_OK;
+  if (!x_host || !out_host || (is_fp8(p) && !x_scale_host)) return MOE_ERR_INVALID_ARG;
+  for (int32_t b = 0; b < n_batches; ++b)
+    if (!x_host[b] || !out_host[b] || (is_fp8(p) && !x_scale_host[b])) return MOE_ERR_INVALID_ARG;
+  if (!weight_scales_ok(p, w_gate_scale, w_up_scale, w_down_scale)) return MOE_ERR_INVALID_ARG;
+  const Layout L = layout(p);
+  for (int slot = 0; slot < 2; ++slot)
+    MOE_TRY(check_layer_args(p, at<void>(ws, L.x_stage[slot]),
+                             is_fp8(p) ? at<float>(ws, L.x_scale_stage[slot]) : nullptr, w_r, w_gate, w_up, w_down,
+                             ws_gate, ws_up, ws_down, at<void>(ws, L.out_stage[slot])));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lock(g_copy_mu);
+  const Copies* c = copies_for_current_device();
+  if (c == nullptr) return MOE_ERR_CUDA;
+  const size_t xbytes = static_cast<size_t>(p->T) * p->H * (is_fp8(p) ? 1 : 2);
+  const size_t sbytes = static_cast<size_t>(p->T) * (p->H / 128) * sizeof(float);
+  const size_t obytes = static_cast<size_t>(p->T) * p->H * 2;
+  // the first copy in comes after the work already on the caller's stream
+  MOE_CUDA(cudaEventRecord(c->fork, st));
+  MOE_CUDA(cudaStreamWaitEvent(c->in, c->fork, 0));
+  MOE_CUDA(cudaStreamWaitEvent(c->out, c->fork, 0));
+  moe_status_t status = MOE_OK;
+  for (int32_t b = 0; b < n_batches && status == MOE_OK; ++b) {
+    const int slot = b & 1;
+    void* x_dev = at<void>(ws, L.x_stage[slot]);
+    float* xs_dev = is_fp8(p) ? at<float>(ws, L.x_scale_stage[slot]) : nullptr;
+    void* out_dev = at<void>(ws, L.out_stage[slot]);
+    // in: the slot's activations were read by the layer of batch b-2 (done[slot])
+    if (b >= 2) MOE_CUDA(cudaStreamWaitEvent(c->in, c->done[slot], 0));
+    MOE_CUDA(cudaMemcpyAsync(x_dev, x_host[b], xbytes, cudaMemcpyHostToDevice, c->in));
+    if (is_fp8(p)) MOE_CUDA(cudaMemcpyAsync(xs_dev, x_scale_host[b], sbytes, cudaMemcpyHostToDevice, c->in));
+    MOE_CUDA(cudaEventRecord(c->landed[slot], c->in));
+    // the layer: after its activations landed and the slot's previous output left
+    MOE_CUDA(cudaStreamWaitEvent(st, c->landed[slot], 0));
+    if (b >= 2) MOE_CUDA(cudaStreamWaitEvent(st, c->left[slot], 0));
+    status = do_layer(p, x_dev, xs_dev, w_r, bias, w_gate, w_up, w_down, w_gate_scale, w_up_scale, w_down_scale,
+                      ws_gate, ws_up, ws_down, out_dev, nullptr, nullptr, nullptr, ws, st);
+    MOE_CUDA(cudaEventRecord(c->done[slot], st));
+    // out
+    MOE_CUDA(cudaStreamWaitEvent(c->out, c->done[slot], 0));
+    MOE_CUDA(cudaMemcpyAsync(out_host[b], out_dev, obytes, cudaMemcpyDeviceToHost, c->out));
+    MOE_CUDA(cudaEventRecord(c->left[slot], c->out));
+  }
+  // the caller's stream passes the call once every output has left
+  MOE_CUDA(cudaStreamWaitEvent(st, c->left[0], 0));
+  if (n_batches > 1) MOE_CUDA(cudaStreamWaitEvent(st, c->left[1], 0));
+  return status;
 }
 
 moe_status_t moe_get_device_status(const void* ws, void* stream, int32_t* host_status) {

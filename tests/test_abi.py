@@ -38,7 +38,7 @@ def test_exports_every_declared_symbol(lib):
     for name in declared:
         assert hasattr(raw, name), name
     assert declared == set(B.EXPORTED), declared ^ set(B.EXPORTED)
-    assert lib.moe_abi_version() == 5
+    assert lib.moe_abi_version() == 6
 
 
 def test_params_struct_matches_header():
