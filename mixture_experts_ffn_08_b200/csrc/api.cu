@@ -314,12 +314,14 @@ moe_status_t do_route(const moe_params_t* p, const void* x, const float* x_scale
   return MOE_OK;
 }
 
+// fill_pad: zero x_perm's pad rows (moe_permute's contract); the layer skips it (its GEMMs
+// never store a pad row).
 moe_status_t do_permute(const moe_params_t* p, const int32_t* ids, const void* x, const float* x_scale,
                         int32_t* counts, int32_t* offsets, int32_t* rop, int32_t* por, void* x_perm,
-                        float* x_perm_scale, void* ws, cudaStream_t st) {
+                        float* x_perm_scale, void* ws, cudaStream_t st, bool fill_pad = true) {
   const Layout L = layout(p);
   return cuda_status(launch_permute(*p, block_m_of(p), ids, x, x_scale, counts, offsets, rop, por, x_perm, x_perm_scale,
-                                    at<int32_t>(ws, L.chunk_counts), at<int32_t>(ws, L.status), st));
+                                    at<int32_t>(ws, L.chunk_counts), at<int32_t>(ws, L.status), st, fill_pad));
 }
 
 moe_status_t do_expert_ffn_fp8(const moe_params_t* p, const void* x_perm, const float* x_perm_scale,
@@ -464,7 +466,7 @@ moe_status_t do_layer_after_fork(const moe_params_t* p, const void* x, const flo
   int32_t* rop = at<int32_t>(ws, L.row_of_pair);
   float* y_perm = at<float>(ws, L.y_perm);
   MOE_TRY(do_permute(p, ids, x, x_scale, counts, offsets, rop, at<int32_t>(ws, L.pair_of_row),
-                     at<void>(ws, L.x_perm), at<float>(ws, L.x_perm_scale), ws, st));
+                     at<void>(ws, L.x_perm), at<float>(ws, L.x_perm_scale), ws, st, /*fill_pad=*/false));
   if (p->fused_combine) {
     // acc starts as the shared expert's output (or zero); the routed down projection adds
     // w * y of every pair into it; one pass rounds it to bf16

@@ -79,11 +79,14 @@ cudaError_t launch_masked_schedule(const int32_t* counts, int E, int32_t* sched,
 cudaError_t launch_bounded_wait_selftest(int32_t* status, long long limit_ns, cudaStream_t st);
 // offsets[e] = e * cap for e in [0, E] (masked layout row ranges).
 cudaError_t launch_masked_offsets(int E, int cap, int32_t* offsets, cudaStream_t st);
+// fill_pad: contiguous layout only, zero the pad rows of x_perm (scale 1 for FP8).  The
+// layer itself passes false: its GEMMs never store a pad row, and an MMA row depends on
+// its own A row only, so whatever the pad rows hold stays in rows nobody reads.
 cudaError_t launch_permute(const moe_params_t& p, int block_m, const int32_t* ids, const void* x,
                            const float* x_scale, int32_t* counts, int32_t* offsets,
                            int32_t* row_of_pair, int32_t* pair_of_row, void* x_perm,
                            float* x_perm_scale, int32_t* chunk_counts, int32_t* status,
-                           cudaStream_t st);
+                           cudaStream_t st, bool fill_pad = true);
 
 // ---------------------------------------------------------------- combine (kernels.cu)
 // y_perm is fp32 for bf16 workloads and bf16 for FP8 workloads (p.dtype).

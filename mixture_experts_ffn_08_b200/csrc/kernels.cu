@@ -512,7 +512,7 @@ cudaError_t launch_permute(const moe_params_t& p, int block_m, const int32_t* id
                            const float* x_scale, int32_t* counts, int32_t* offsets,
                            int32_t* row_of_pair, int32_t* pair_of_row, void* x_perm,
                            float* x_perm_scale, int32_t* chunk_counts, int32_t* status,
-                           cudaStream_t st) {
+                           cudaStream_t st, bool fill_pad) {
   const int P = p.T * p.K;
   const int nchunks = (P + kPermChunk - 1) / kPermChunk;
   const int bm = block_m;
@@ -538,6 +538,7 @@ cudaError_t launch_permute(const moe_params_t& p, int block_m, const int32_t* id
     if (err != cudaSuccess || (err = cudaGetLastError()) != cudaSuccess) return err;
   }
   const bool masked = p.masked_cap > 0;
+  const bool zero_pad = !masked && fill_pad;
   const long long max_rows = masked ? static_cast<long long>(p.E) * p.masked_cap
                                     : static_cast<long long>(P) + static_cast<long long>(p.E) * (bm - 1);
   const long long blocks = (max_rows + kGatherWarps - 1) / kGatherWarps;
@@ -545,10 +546,10 @@ cudaError_t launch_permute(const moe_params_t& p, int block_m, const int32_t* id
   trace_before(MOE_K_PERM_GATHER, st);
   if (act_e4m3(p))
     err = launch_k(perm_gather_kernel<true>, grid, 32 * kGatherWarps, 0, st, x, x_scale, p.H, p.K, p.E, counts,
-                   offsets, pair_of_row, x_perm, x_perm_scale, !masked);
+                   offsets, pair_of_row, x_perm, x_perm_scale, zero_pad);
   else
     err = launch_k(perm_gather_kernel<false>, grid, 32 * kGatherWarps, 0, st, x, x_scale, p.H, p.K, p.E, counts,
-                   offsets, pair_of_row, x_perm, x_perm_scale, !masked);
+                   offsets, pair_of_row, x_perm, x_perm_scale, zero_pad);
   trace_after(MOE_K_PERM_GATHER, st);
   return err != cudaSuccess ? err : cudaGetLastError();
 }
