@@ -31,6 +31,9 @@ SMALL = {
     "dsv3_small": W.DSV3_PREFILL.with_(name="dsv3_small", T=200, H=512, I=256, E=32, I_shared=256),
     "dsv3_decode_small": W.DSV3_DECODE.with_(name="dsv3_decode_small", T=16, H=512, I=256, E=32,
                                              I_shared=256),
+    # H not a multiple of 256: the shared expert's down projection does not take in the
+    # combine, which then runs as its own kernel
+    "dsv3_small_h384": W.DSV3_PREFILL.with_(name="dsv3_small_h384", T=200, H=384, I=256, E=32, I_shared=256),
     "one_token": W.MIXTRAL_PREFILL.with_(name="one_token", T=1, H=256, I=128, E=4, K=2),
     "dense_like": W.TINY.with_(name="dense_like", T=300, E=1, K=1),
     # buckets aligned to 256 rows: the two-SM (cta_group::2) GEMMs
