@@ -104,6 +104,11 @@ cudaError_t gemm_gateup_swiglu(const void* A, int64_t a_rows, const int32_t* off
                                const int32_t* counts, int G, int dense_rows, const void* w_gate,
                                const void* w_up, int N, int K, void* h, int32_t* status, int kid,
                                cudaStream_t st, int masked_cap = 0);
+// The same gate/up projection with two M-tiles of an expert per work item (grouped, with
+// counts, N multiple of 128); counter is a device int the call zeroes before the launch.
+cudaError_t gemm_gateup_swiglu_dual(const void* A, int64_t a_rows, const int32_t* offsets, const int32_t* counts,
+                                    int G, const void* w_gate, const void* w_up, int N, int K, void* h,
+                                    int32_t* counter, int32_t* status, cudaStream_t st, int masked_cap = 0);
 // y [rows, N] fp32 = A W^T, grouped by offsets (or dense when null); with counts, pad
 // rows of each group are not stored.
 cudaError_t gemm_down(const void* A, int64_t a_rows, const int32_t* offsets,

@@ -36,6 +36,11 @@ SMALL = {
     "dsv3_small_h384": W.DSV3_PREFILL.with_(name="dsv3_small_h384", T=200, H=384, I=256, E=32, I_shared=256),
     "one_token": W.MIXTRAL_PREFILL.with_(name="one_token", T=1, H=256, I=128, E=4, K=2),
     "dense_like": W.TINY.with_(name="dense_like", T=300, E=1, K=1),
+    # T*K >= 256*E: the two-M-tile gate/up kernel (pairs of M-tiles plus one-tile tails)
+    "mixtral_small_dual": W.MIXTRAL_PREFILL.with_(name="mixtral_small_dual", T=1200, H=512, I=384),
+    "dsv3_small_dual": W.DSV3_PREFILL.with_(name="dsv3_small_dual", T=1100, H=512, I=256, E=32, I_shared=256),
+    "mixtral_small_dual_masked": W.MIXTRAL_PREFILL.with_(name="mixtral_small_dual_masked", T=1200, H=512, I=384,
+                                                         masked_cap=640),
     # buckets aligned to 256 rows: the two-SM (cta_group::2) GEMMs
     "mixtral_small_pair": W.MIXTRAL_PREFILL.with_(name="mixtral_small_pair", T=1000, H=512, I=384, block_m=256),
     "dsv3_small_pair": W.DSV3_PREFILL.with_(name="dsv3_small_pair", T=300, H=512, I=256, E=32, I_shared=256,
@@ -48,11 +53,13 @@ SMALL = {
 }
 
 
-# Cases whose max|err| against the exact-h oracle is above 2e-2 * RMS: measured 0.0208
-# (0.0159 against the bf16-h oracle), of which 0.0159 is the floor that rounding the
-# exact output once to bf16 already costs on these 512,000 outputs.  Every other case
+# Cases whose max|err| against the exact-h oracle is above 2e-2 * RMS: the Mixtral-shaped
+# small layers (H=512, I=384), measured at 0.0208 (0.0159 against the bf16-h oracle), of
+# which 0.0159 is the floor that rounding the exact output once to bf16 already costs on
+# these 512,000-614,400 outputs.  Every other case
 # asserts the max bound against the exact-h oracle as well.
-EXACT_MAX_EXCEEDS = {"mixtral_small", "mixtral_small_pair", "mixtral_small_fused"}
+EXACT_MAX_EXCEEDS = {"mixtral_small", "mixtral_small_pair", "mixtral_small_fused", "mixtral_small_dual",
+                     "mixtral_small_dual_masked"}
 
 
 def _both(x, ids, w, d, wl):
