@@ -146,20 +146,51 @@ cudaError_t gemm_gateup_swiglu_dual(const void* A, int64_t a_rows, const int32_t
   dp.K = K;
   dp.N = N;
   dp.masked_cap = masked_cap;
-  dp.out = static_cast<__nv_bfloat16*>(h);
+  dp.out = h;
   dp.ldo = N;
   dp.status = status;
   dp.next_item = counter;
   cudaError_t err = cudaMemsetAsync(counter, 0, sizeof(int32_t), st);
   if (err != cudaSuccess) return err;
-  err = cudaFuncSetAttribute(tc_gemm_dual_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDualSmemBytes);
+  err = cudaFuncSetAttribute(tc_gemm_dual_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDualSmemBytes);
   if (err != cudaSuccess) return err;
   const long long max_items = ceil_div(a_rows, 128) * (N / 128);
   const long long sms = num_sms();
   const int grid = static_cast<int>(max_items < sms ? (max_items > 0 ? max_items : 1) : sms);
   trace_before(MOE_K_GATEUP, st);
-  err = launch_k(tc_gemm_dual_kernel, grid, kDualThreads, kDualSmemBytes, st, ta, tg, tu, dp);
+  err = launch_k(tc_gemm_dual_kernel<true>, grid, kDualThreads, kDualSmemBytes, st, ta, tg, tu, dp);
   trace_after(MOE_K_GATEUP, st);
+  return err != cudaSuccess ? err : cudaGetLastError();
+}
+
+cudaError_t gemm_down_dual(const void* A, int64_t a_rows, const int32_t* offsets, const int32_t* counts, int G,
+                           const void* w, int N, int K, float* y, int32_t* counter, int32_t* status, cudaStream_t st,
+                           int masked_cap) {
+  if (G > kDualMaxGroups || N % 256 != 0 || K % 64 != 0) return cudaErrorInvalidValue;
+  CUtensorMap ta, tb;
+  if (!make_tmap_bf16(&ta, A, a_rows, K, 128) || !make_tmap_bf16(&tb, w, static_cast<uint64_t>(G) * N, K, 256))
+    return cudaErrorInvalidValue;
+  DualParams dp{};
+  dp.offsets = offsets;
+  dp.counts = counts;
+  dp.G = G;
+  dp.K = K;
+  dp.N = N;
+  dp.masked_cap = masked_cap;
+  dp.out = y;
+  dp.ldo = N;
+  dp.status = status;
+  dp.next_item = counter;
+  cudaError_t err = cudaMemsetAsync(counter, 0, sizeof(int32_t), st);
+  if (err != cudaSuccess) return err;
+  err = cudaFuncSetAttribute(tc_gemm_dual_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDualSmemBytes);
+  if (err != cudaSuccess) return err;
+  const long long max_items = ceil_div(a_rows, 128) * (N / 256);
+  const long long sms = num_sms();
+  const int grid = static_cast<int>(max_items < sms ? (max_items > 0 ? max_items : 1) : sms);
+  trace_before(MOE_K_DOWN, st);
+  err = launch_k(tc_gemm_dual_kernel<false>, grid, kDualThreads, kDualSmemBytes, st, ta, tb, tb, dp);
+  trace_after(MOE_K_DOWN, st);
   return err != cudaSuccess ? err : cudaGetLastError();
 }
 

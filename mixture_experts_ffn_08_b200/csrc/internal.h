@@ -109,6 +109,10 @@ cudaError_t gemm_gateup_swiglu(const void* A, int64_t a_rows, const int32_t* off
 cudaError_t gemm_gateup_swiglu_dual(const void* A, int64_t a_rows, const int32_t* offsets, const int32_t* counts,
                                     int G, const void* w_gate, const void* w_up, int N, int K, void* h,
                                     int32_t* counter, int32_t* status, cudaStream_t st, int masked_cap = 0);
+// The down projection with two M-tiles per work item (N multiple of 256); counter as above.
+cudaError_t gemm_down_dual(const void* A, int64_t a_rows, const int32_t* offsets, const int32_t* counts, int G,
+                           const void* w, int N, int K, float* y, int32_t* counter, int32_t* status, cudaStream_t st,
+                           int masked_cap = 0);
 // y [rows, N] fp32 = A W^T, grouped by offsets (or dense when null); with counts, pad
 // rows of each group are not stored.
 cudaError_t gemm_down(const void* A, int64_t a_rows, const int32_t* offsets,

@@ -1,9 +1,11 @@
-// Gate/up projection with fused SwiGLU, two M-tiles per work item.
+// Grouped expert GEMMs with two M-tiles per work item: the gate/up projection with fused
+// SwiGLU (SWIGLU = true) and the down projection (fp32 out).
 //
-// The same grouped GEMM as tc_gemm_kernel<EPI_SWIGLU> (routing primer "MoE 路由入门" §5.2;
-// the "MoE" chapter index's M-grouped contiguous layout), with one change in how a CTA
-// spends its shared memory: a work item is up to two consecutive 128-row M-tiles of one
-// expert against one 256-row weight tile [128 gate rows; 128 up rows].  Each K-step stage
+// The same grouped GEMMs as tc_gemm_kernel<EPI_SWIGLU / EPI_F32> (routing primer "MoE 路由入门"
+// §5.2; the "MoE" chapter index's M-grouped contiguous layout), with one change in how a
+// CTA spends its shared memory: a work item is up to two consecutive 128-row M-tiles of one
+// expert against one 256-row weight tile ([128 gate rows; 128 up rows], or 256 rows of
+// W_down).  Each K-step stage
 // holds both A tiles and the one B tile (64 KB), and the MMA thread issues, per 16-wide K
 // slice, one M=128 N=256 tcgen05.mma per M-tile into its own 256-column TMEM accumulator.
 // Every weight tile staged in shared memory is so used twice, which halves the weight
@@ -21,7 +23,7 @@
 // at most 64 real rows runs M=64 MMAs (accumulator rows in lanes 0-15 of each quadrant).
 //
 // Warp roles (192 threads): warp 0 takes items and issues TMA loads, warp 1 allocates
-// TMEM and issues MMAs, warps 2-5 run the SwiGLU epilogue.  Every wait is bounded; on a
+// TMEM and issues MMAs, warps 2-5 run the epilogue.  Every wait is bounded; on a
 // timeout the CTA sets MOE_DEV_TIMEOUT, drains its copies and MMAs, frees TMEM and exits.
 #pragma once
 
@@ -34,9 +36,9 @@ struct DualParams {
   const int32_t* counts;    // [G] real rows of each group (rows past it are not stored)
   int G;                    // groups (G <= kDualMaxGroups)
   int K;                    // reduction length, multiple of 64
-  int N;                    // output columns (h width); weight rows per group and matrix
+  int N;                    // output columns; weight rows per group (and matrix, for SwiGLU)
   int masked_cap;           // > 0: group g's rows sit at g * masked_cap in A and out
-  __nv_bfloat16* out;       // h [rows, ldo]
+  void* out;                // SwiGLU: h [rows, ldo] bf16; else y [rows, ldo] fp32
   int64_t ldo;
   int32_t* status;
   int32_t* next_item;       // work counter, zero at launch
@@ -61,11 +63,13 @@ struct DualItem {
   int mt0;       // first M-tile of the group
 };
 
-// Item -> (group, weight tile, M-tiles).  pref[g] = sum over e < g of NT * pairs(e), with
+// Item -> (group, weight tile, M-tiles); weight tiles of 128 output columns for SwiGLU
+// (128 gate + 128 up rows), of 256 for the plain projection.  pref[g] = sum over e < g of NT * pairs(e), with
 // pairs(e) = ceil(tiles(e) / 2).  Inside a group, weight tiles are outer (every pair of
 // M-tiles in flight shares each weight tile) unless the group's activation rows outnumber
 // its weight rows (NT * 256), as for a very hot expert, where pairs are outer.
 MOE_DEVINL DualItem dual_decode(int item, int NT, const DualParams& p, const int* pref) {
+  // (NT * 256 is the group's weight rows in both forms: SwiGLU tiles hold 256 rows too)
   int lo = 0, hi = p.G - 1;  // group with pref[g] <= item < pref[g+1]
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -87,9 +91,14 @@ MOE_DEVINL DualItem dual_decode(int item, int NT, const DualParams& p, const int
   return d;
 }
 
+// SWIGLU: tmG / tmU are the gate and up weights (boxes of 128 rows) and h = SiLU(g) * u is
+// stored in bf16; otherwise tmG is the one weight matrix (boxes of 256 rows) and the fp32
+// product is stored.
+template <bool SWIGLU>
 __global__ void __launch_bounds__(kDualThreads, 1)
     tc_gemm_dual_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmG,
                         const __grid_constant__ CUtensorMap tmU, const DualParams p) {
+  constexpr int OUT_COLS = SWIGLU ? 128 : 256;
   constexpr int BK = kDualBK, STAGES = kDualStages, R = kDualRing;
   constexpr uint32_t IDESC = idesc_bf16_f32(128, 256);
   constexpr uint32_t IDESC_HALF = idesc_bf16_f32(64, 256);
@@ -106,7 +115,7 @@ __global__ void __launch_bounds__(kDualThreads, 1)
   const int warp = warp_id(), lane = lane_id();
   const uint32_t pad = (1024u - (smem_u32(dsmem) & 1023u)) & 1023u;
   uint8_t* smem = dsmem + pad;
-  const int NT = (p.N + 127) / 128;
+  const int NT = (p.N + OUT_COLS - 1) / OUT_COLS;
   const int KB = p.K / BK;
 
   if (threadIdx.x == 0) {
@@ -129,7 +138,7 @@ __global__ void __launch_bounds__(kDualThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmG);
-    prefetch_tmap(&tmU);
+    if (SWIGLU) prefetch_tmap(&tmU);
   }
   if (warp == 1) {
     tmem_alloc(&tmem_base_sh, 512);
@@ -184,7 +193,7 @@ __global__ void __launch_bounds__(kDualThreads, 1)
         mbar_arrive(&item_full[rs]);
         if (it >= total) break;
         const DualItem d = dual_decode(it, NT, p, pref);
-        const int b_row = d.group * p.N + d.n_tile * 128;
+        const int b_row = d.group * p.N + d.n_tile * OUT_COLS;
         int a_row[2];
         for (int u = 0; u < 2; ++u) {
           const int local0 = (d.tile0 + u - d.mt0) * 128;
@@ -198,7 +207,7 @@ __global__ void __launch_bounds__(kDualThreads, 1)
           tma_load_2d(st, &tmA, kb * BK, a_row[0], &full_bar[s]);
           if (d.ntiles == 2) tma_load_2d(st + kDualABytes, &tmA, kb * BK, a_row[1], &full_bar[s]);
           tma_load_2d(st + 2 * kDualABytes, &tmG, kb * BK, b_row, &full_bar[s]);
-          tma_load_2d(st + 2 * kDualABytes + kDualBBytes / 2, &tmU, kb * BK, b_row, &full_bar[s]);
+          if (SWIGLU) tma_load_2d(st + 2 * kDualABytes + kDualBBytes / 2, &tmU, kb * BK, b_row, &full_bar[s]);
           ++issued;
           if (++s == STAGES) { s = 0; ph ^= 1u; }
         }
@@ -271,7 +280,7 @@ __global__ void __launch_bounds__(kDualThreads, 1)
     const int q = warp & 3;
     int nxt = 0;
     uint32_t uses[2] = {0u, 0u};
-    const bool v8 = ((reinterpret_cast<uintptr_t>(p.out) | (static_cast<uintptr_t>(p.ldo) * 2)) & 31) == 0;
+    const bool v8 = ((reinterpret_cast<uintptr_t>(p.out) | (static_cast<uintptr_t>(p.ldo) * (SWIGLU ? 2 : 4))) & 31) == 0;
     bool ok = true;
     for (int i = 0; ok; ++i) {
       const int rs = i % R;
@@ -286,7 +295,7 @@ __global__ void __launch_bounds__(kDualThreads, 1)
       const int slot0 = nxt, slot1 = nxt ^ 1;
       if (d.ntiles == 1) nxt ^= 1;
       const int count = __ldg(p.counts + d.group);
-      const int col0 = d.n_tile * 128;
+      const int col0 = d.n_tile * OUT_COLS;
       for (int u = 0; u < d.ntiles && ok; ++u) {
         const int slot = u == 0 ? slot0 : slot1;
         ok = __all_sync(0xffffffffu, mbar_wait_bounded(&tfull_bar[slot], uses[slot] & 1u, &abort_flag));
@@ -298,28 +307,49 @@ __global__ void __launch_bounds__(kDualThreads, 1)
         const int trow = half ? q * 16 + lane : q * 32 + lane;
         const bool row_ok = (!half || lane < 16) && local0 + trow < count;
         const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + slot * 256;
-        __nv_bfloat16* out = p.out + (static_cast<long long>(row0) + trow) * p.ldo + col0;
+        const long long orow = static_cast<long long>(row0) + trow;
+        if constexpr (SWIGLU) {
+          __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + orow * p.ldo + col0;
 #pragma unroll 1
-        for (int c = 0; c < 128; c += 32) {
-          uint32_t rg[32], ru[32];
-          tmem_ld_32x32b_x32(tbase + c, rg);
-          tmem_ld_32x32b_x32(tbase + 128 + c, ru);
-          tmem_ld_wait(rg);
-          reg_fence(ru);
-          uint32_t packed[16];
+          for (int c = 0; c < 128; c += 32) {
+            uint32_t rg[32], ru[32];
+            tmem_ld_32x32b_x32(tbase + c, rg);
+            tmem_ld_32x32b_x32(tbase + 128 + c, ru);
+            tmem_ld_wait(rg);
+            reg_fence(ru);
+            uint32_t packed[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            packed[e] = pack_bf16x2(silu_mul(__uint_as_float(rg[2 * e]), __uint_as_float(ru[2 * e])),
-                                    silu_mul(__uint_as_float(rg[2 * e + 1]), __uint_as_float(ru[2 * e + 1])));
-          if (row_ok && col0 + c < p.N) {
-            if (v8) {
-              st_global_v8(out + c, packed);
-              st_global_v8(out + c + 16, packed + 8);
-            } else {
-              uint4* dst = reinterpret_cast<uint4*>(out + c);
+            for (int e = 0; e < 16; ++e)
+              packed[e] = pack_bf16x2(silu_mul(__uint_as_float(rg[2 * e]), __uint_as_float(ru[2 * e])),
+                                      silu_mul(__uint_as_float(rg[2 * e + 1]), __uint_as_float(ru[2 * e + 1])));
+            if (row_ok && col0 + c < p.N) {
+              if (v8) {
+                st_global_v8(out + c, packed);
+                st_global_v8(out + c + 16, packed + 8);
+              } else {
+                uint4* dst = reinterpret_cast<uint4*>(out + c);
 #pragma unroll
-              for (int v = 0; v < 4; ++v)
-                dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+                for (int v = 0; v < 4; ++v)
+                  dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+              }
+            }
+          }
+        } else {
+          float* out = static_cast<float*>(p.out) + orow * p.ldo + col0;
+#pragma unroll 1
+          for (int c = 0; c < 256; c += 32) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(tbase + c, r);
+            tmem_ld_wait(r);
+            if (row_ok && col0 + c < p.N) {
+              if (v8 && col0 + c + 32 <= p.N) {
+#pragma unroll
+                for (int v = 0; v < 4; ++v) st_global_v8(out + c + 8 * v, r + 8 * v);
+              } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                  if (col0 + c + e < p.N) out[c + e] = __uint_as_float(r[e]);
+              }
             }
           }
         }

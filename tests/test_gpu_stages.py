@@ -191,7 +191,7 @@ def test_permute_bad_ids_are_reported_and_skipped():
 # ------------------------------------------------------------------ expert FFN
 @pytest.mark.parametrize("E,K,T,H,I,bm", [(1, 1, 300, 256, 128, 0), (6, 2, 700, 384, 256, 0),
                                           (16, 4, 64, 512, 384, 0), (3, 3, 129, 1024, 640, 0),
-                                          (4, 2, 1200, 384, 256, 0),  # two-M-tile gate/up kernel
+                                          (4, 2, 1200, 512, 256, 0),  # two-M-tile gate/up and down kernels
                                           (1, 1, 300, 256, 128, 256), (6, 2, 700, 512, 256, 256),
                                           (3, 3, 700, 384, 640, 256)])
 def test_expert_ffn_grouped_gemm(E, K, T, H, I, bm):
