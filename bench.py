@@ -48,13 +48,17 @@ FLUSH_BYTES = 512 << 20
 
 
 GEMM_SOURCES = ("csrc/tc_gemm.cuh", "csrc/common.cuh", "csrc/gemm.cu")
+DUAL_GEMM_SOURCES = ("csrc/tc_gemm_dual.cuh", "csrc/tc_gemm.cuh", "csrc/common.cuh", "csrc/gemm.cu")
 FP8_GEMM_SOURCES = ("csrc/tc_gemm_fp8.cuh", "csrc/tc_gemm.cuh", "csrc/common.cuh", "csrc/gemm_fp8.cu")
 
 
 def gateup_sources(wl):
     """Source files of the gate/up kernel the library runs for this workload: the
-    block-scaled GEMM for e4m3 activations, the bf16 GEMM otherwise."""
-    return FP8_GEMM_SOURCES if wl.dtype in (W.DTYPE_FP8, W.DTYPE_FP8_FP4) else GEMM_SOURCES
+    block-scaled GEMM for e4m3 activations; for bf16, the two-M-tile GEMM when the
+    average expert holds two 128-row M-tiles (T*K >= 256*E), else the one-tile GEMM."""
+    if wl.dtype in (W.DTYPE_FP8, W.DTYPE_FP8_FP4):
+        return FP8_GEMM_SOURCES
+    return DUAL_GEMM_SOURCES if wl.T * wl.K >= 256 * wl.E else GEMM_SOURCES
 
 
 def sources_sha256(files):

@@ -80,4 +80,5 @@ PROFILE = {w.name: w for w in (
     DSV3_PREFILL.with_(name="dsv3_prefill_e32", T=1024, E=32),
     SKEWED_FP8.with_(name="skewed_fp8_e32", T=4096, E=32),
     DSV3_DECODE.with_(name="dsv3_decode_fp4_e64", T=32, E=64, dtype=DTYPE_FP8_FP4, I_shared=0),
+    DSV3_DECODE.with_(name="dsv3_decode_e32", T=16, E=32),
 )}

@@ -50,7 +50,9 @@ def test_no_launches_gives_no_fraction():
 
 def test_gate_up_kernel_sources_follow_the_library_rule():
     from mixture_experts_ffn_08_b200 import workloads as W
-    assert bench.gateup_sources(W.MIXTRAL_PREFILL) == bench.GEMM_SOURCES
+    assert bench.gateup_sources(W.MIXTRAL_PREFILL) == bench.DUAL_GEMM_SOURCES
+    assert bench.gateup_sources(W.DSV3_PREFILL) == bench.DUAL_GEMM_SOURCES
+    assert bench.gateup_sources(W.DSV3_DECODE) == bench.GEMM_SOURCES
     assert bench.gateup_sources(W.SKEWED_FP8) == bench.FP8_GEMM_SOURCES
     assert bench.gateup_sources(W.FP4["dsv3_prefill_fp4"]) == bench.FP8_GEMM_SOURCES
     assert bench.gateup_sources(W.FP4["dsv3_decode_fp4"]) == bench.FP8_GEMM_SOURCES
