@@ -854,7 +854,8 @@ int32_t moe_layer_launch_count(const moe_params_t* p) {
   int n = 2;                                 // router GEMM, top-k
   if (is_fp8(p)) n += is_fp4(p) ? 2 : 5;     // dequantise x for the router; scale atoms of x
                                              // (and of the three e4m3 weights)
-  n += (p->T * p->K > 0) ? 4 : 2;            // count, scan, rank, gather
+  const long long P = static_cast<long long>(p->T) * p->K;
+  n += P <= kSmallPairs ? 2 : 4;             // count, scan, rank (one kernel for few pairs), gather
   n += 2;                                    // gate/up, down
   if (p->I_shared > 0) n += 2;               // shared gate/up, down
   n += 1;                                    // combine

@@ -14,6 +14,7 @@ constexpr int kBlockM2 = 256;   // bucket alignment for the two-SM (cta_group::2
 constexpr int kMaxExperts = 1024;
 constexpr int kMaxTopK = 32;
 constexpr int kPermChunk = 256;  // pairs per chunk of the stable bucket ranking
+constexpr int kSmallPairs = 2048;  // up to this many pairs one block counts, scans and ranks
 
 // Programmatic dependent launch of the layer's kernels (api.cu): on unless the
 // environment sets MOE_DISABLE_PDL to a non-empty value other than "0".

@@ -457,6 +457,83 @@ __global__ void __launch_bounds__(32 * kRankWarps) perm_rank_kernel(
   }
 }
 
+// 1-3 in one block, for at most kSmallPairs pairs (decode-sized batches): expert counts
+// in shared memory, the padded scan, then one warp walks the pairs in order, 32 at a
+// time, for the stable ranks.  Same outputs as the three kernels above.
+__global__ void __launch_bounds__(1024) perm_small_kernel(
+    const int32_t* __restrict__ ids, int P, int E, int block_m, int cap, int32_t* __restrict__ counts,
+    int32_t* __restrict__ offsets, int32_t* __restrict__ row_of_pair, int32_t* __restrict__ pair_of_row,
+    int32_t* status) {
+  pdl_launch_dependents();
+  pdl_wait();
+  __shared__ int cnt[kMaxExperts];
+  __shared__ int next_row[kMaxExperts];
+  __shared__ int warp_tot[32];
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  for (int e = tid; e < E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  for (int p = tid; p < P; p += blockDim.x) {
+    const int e = __ldg(ids + p);
+    if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
+    else set_status(status, MOE_DEV_BAD_EXPERT_ID);
+  }
+  __syncthreads();
+  // padded exclusive scan over the experts (E <= blockDim.x)
+  const int e = tid;
+  const int total = e < E ? cnt[e] : 0;
+  const int padded = e >= E ? 0 : cap > 0 ? cap : (total + block_m - 1) / block_m * block_m;
+  int v = padded;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(kFull, v, o);
+    if (lane >= o) v += n;
+  }
+  if (lane == 31) warp_tot[w] = v;
+  __syncthreads();
+  if (w == 0) {
+    int t = warp_tot[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(kFull, t, o);
+      if (lane >= o) t += n;
+    }
+    warp_tot[lane] = t;
+  }
+  __syncthreads();
+  const int incl = v + (w > 0 ? warp_tot[w - 1] : 0);
+  const int excl = incl - padded;
+  if (e < E) {
+    if (cap > 0 && total > cap) set_status(status, MOE_DEV_CAPACITY);
+    counts[e] = cap > 0 && total > cap ? cap : total;
+    offsets[e] = excl;
+    next_row[e] = excl;
+  }
+  if (e == E - 1) offsets[E] = incl;
+  __syncthreads();
+  if (w == 0) {
+    for (int base = 0; base < P; base += 32) {
+      const int p = base + lane;
+      const int ex = p < P ? __ldg(ids + p) : -1;
+      const bool ok = p < P && ex >= 0 && ex < E;
+      const int key = ok ? ex : -1 - lane;  // invalid lanes match nobody
+      const unsigned peers = __match_any_sync(kFull, key);
+      const int rank = __popc(peers & ((1u << lane) - 1u));
+      const int r0 = ok ? next_row[ex] : 0;
+      __syncwarp();
+      if (ok) {
+        const int row = r0 + rank;
+        const bool kept = cap <= 0 || row < (ex + 1) * cap;
+        row_of_pair[p] = kept ? row : -1;
+        if (kept) pair_of_row[row] = p;
+        if (rank == 0) next_row[ex] = r0 + __popc(peers);
+      } else if (p < P) {
+        row_of_pair[p] = -1;
+      }
+      __syncwarp();
+    }
+  }
+}
+
 // 4) row gather: x_perm[r] = x[pair_of_row[r] / K]; pad rows -> pair -1 and, unless
 //    zero_pad is false (masked layout: unused rows are left as they are), zero.
 //    One warp per row; each lane keeps up to 8 16-byte loads in flight, so the copy runs
@@ -517,6 +594,13 @@ cudaError_t launch_permute(const moe_params_t& p, int block_m, const int32_t* id
   const int nchunks = (P + kPermChunk - 1) / kPermChunk;
   const int bm = block_m;
   cudaError_t err;
+  if (P > 0 && P <= kSmallPairs) {
+    trace_before(MOE_K_PERM_SCAN, st);
+    err = launch_k(perm_small_kernel, 1, 1024, 0, st, ids, P, p.E, bm, p.masked_cap, counts, offsets, row_of_pair,
+                   pair_of_row, status);
+    trace_after(MOE_K_PERM_SCAN, st);
+    if (err != cudaSuccess || (err = cudaGetLastError()) != cudaSuccess) return err;
+  } else {
   if (nchunks > 0) {
     trace_before(MOE_K_PERM_COUNT, st);
     err = launch_k(perm_count_kernel, nchunks, kPermChunk, p.E * sizeof(int), st, ids, P, p.E, chunk_counts,
@@ -536,6 +620,7 @@ cudaError_t launch_permute(const moe_params_t& p, int block_m, const int32_t* id
                    p.masked_cap, chunk_counts, row_of_pair, pair_of_row);
     trace_after(MOE_K_PERM_RANK, st);
     if (err != cudaSuccess || (err = cudaGetLastError()) != cudaSuccess) return err;
+  }
   }
   const bool masked = p.masked_cap > 0;
   const bool zero_pad = !masked && fill_pad;

@@ -115,6 +115,36 @@ def test_permute_random(seed, block_m):
     assert B.moe_get_device_status(r["ws"]) == 0
 
 
+@pytest.mark.parametrize("E,K,T,cap", [(1000, 2, 1000, 0), (1024, 4, 512, 0), (16, 8, 256, 128)])
+def test_permute_one_block_path_many_experts(E, K, T, cap):
+    """At most 2048 pairs: one block counts, scans and ranks; up to 1024 experts, and the
+    masked layout's capacity."""
+    wl = W.Workload("perm1", T=T, H=128, I=128, E=E, K=K, masked_cap=cap)
+    rng = np.random.default_rng(E + K)
+    ids = np.stack([rng.choice(E, K, replace=False) for _ in range(T)]).astype(np.int32)
+    if cap:
+        p = B.params(wl)
+        ws = _ws(wl)
+        rows = B.moe_max_padded_rows(p)
+        d_ids = torch.as_tensor(ids, device="cuda")
+        x = torch.randn((T, wl.H), device="cuda").to(torch.bfloat16)
+        counts = torch.empty(E, dtype=torch.int32, device="cuda")
+        offs = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+        rop = torch.empty(T * K, dtype=torch.int32, device="cuda")
+        por = torch.empty(rows, dtype=torch.int32, device="cuda")
+        xp = torch.empty((rows, wl.H), dtype=torch.bfloat16, device="cuda")
+        B.check(B.moe_permute(p, d_ids, x, None, counts, offs, rop, por, xp, None, ws, ws.numel()))
+        torch.cuda.synchronize()
+        o_counts, o_offs, o_rop, o_por, _ = o.permute_masked(ids, E, cap)   # some experts overflow cap
+        np.testing.assert_array_equal(offs.cpu().numpy(), o_offs)
+        np.testing.assert_array_equal(counts.cpu().numpy(), o_counts)
+        np.testing.assert_array_equal(rop.cpu().numpy(), o_rop)
+        np.testing.assert_array_equal(por.cpu().numpy(), o_por)
+        return
+    r = _permute(wl, ids)
+    _check_perm(wl, ids, r)
+
+
 def test_permute_bucket_edge_sizes():
     # experts with 0, 1, BM-1, BM, BM+1, 2*BM+5 rows (K = 1 so counts are set directly)
     sizes = [0, 1, BM - 1, BM, BM + 1, 2 * BM + 5, 0, 3]
