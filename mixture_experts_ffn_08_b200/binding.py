@@ -23,6 +23,7 @@ MOE_OK = 0
 MOE_DEV_BAD_EXPERT_ID = 0x1
 MOE_DEV_TIMEOUT = 0x2
 MOE_DEV_CAPACITY = 0x4
+MOE_DEV_RANGE = 0x8
 BLOCK_M = 128
 
 # Kernel ids for tracing (include/moe.h).

@@ -164,8 +164,8 @@ cudaError_t gemm_gateup_swiglu_dual(const void* A, int64_t a_rows, const int32_t
 }
 
 cudaError_t gemm_down_dual(const void* A, int64_t a_rows, const int32_t* offsets, const int32_t* counts, int G,
-                           const void* w, int N, int K, float* y, int32_t* counter, int32_t* status, cudaStream_t st,
-                           int masked_cap) {
+                           const void* w, int N, int K, void* y, int32_t* counter, int32_t* status, cudaStream_t st,
+                           int masked_cap, bool y_f16) {
   if (G > kDualMaxGroups || N % 256 != 0 || K % 64 != 0) return cudaErrorInvalidValue;
   CUtensorMap ta, tb;
   if (!make_tmap_bf16(&ta, A, a_rows, K, 128) || !make_tmap_bf16(&tb, w, static_cast<uint64_t>(G) * N, K, 256))
@@ -181,6 +181,7 @@ cudaError_t gemm_down_dual(const void* A, int64_t a_rows, const int32_t* offsets
   dp.ldo = N;
   dp.status = status;
   dp.next_item = counter;
+  dp.out_f16 = y_f16 ? 1 : 0;
   cudaError_t err = cudaMemsetAsync(counter, 0, sizeof(int32_t), st);
   if (err != cudaSuccess) return err;
   err = cudaFuncSetAttribute(tc_gemm_dual_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDualSmemBytes);

@@ -703,7 +703,18 @@ MOE_DEVINL void load8(const __nv_bfloat16* row, int v, float (&f)[8]) {
   }
 }
 
-// out[t] = sum_k w[t,k] y_perm[row_of_pair[t*K+k]] (+ y_sh[t]); YT = float or bf16.
+MOE_DEVINL void load8(const __half* row, int v, float (&f)[8]) {
+  const uint4 q = __ldg(reinterpret_cast<const uint4*>(row) + v);
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 t = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+
+// out[t] = sum_k w[t,k] y_perm[row_of_pair[t*K+k]] (+ y_sh[t]); YT = float, bf16 or fp16.
 template <class YT>
 __global__ void __launch_bounds__(128) combine_kernel(
     const YT* __restrict__ y_perm, const int32_t* __restrict__ row_of_pair,
@@ -768,12 +779,15 @@ cudaError_t launch_f32_to_bf16(const float* acc, long long n, void* out, cudaStr
 }
 
 cudaError_t launch_combine(const moe_params_t& p, const void* y_perm, const int32_t* row_of_pair,
-                           const float* w, const float* y_shared, void* out, cudaStream_t st) {
+                           const float* w, const float* y_shared, void* out, cudaStream_t st, bool y_f16) {
   if (p.T == 0) return cudaSuccess;
   const int grid = p.T < num_sms() * 16 ? p.T : num_sms() * 16;
   trace_before(MOE_K_COMBINE, st);
   cudaError_t err;
-  if (act_e4m3(p))
+  if (y_f16)
+    err = launch_k(combine_kernel<__half>, grid, 128, 0, st, static_cast<const __half*>(y_perm), row_of_pair, w,
+                   y_shared, static_cast<__nv_bfloat16*>(out), p.T, p.H, p.K);
+  else if (act_e4m3(p))
     err = launch_k(combine_kernel<__nv_bfloat16>, grid, 128, 0, st, static_cast<const __nv_bfloat16*>(y_perm),
                    row_of_pair, w, y_shared, static_cast<__nv_bfloat16*>(out), p.T, p.H, p.K);
   else

@@ -42,6 +42,7 @@ struct DualParams {
   int64_t ldo;
   int32_t* status;
   int32_t* next_item;       // work counter, zero at launch
+  int out_f16;              // plain projection: store y as fp16 (|y| > 65504 sets MOE_DEV_RANGE)
 };
 
 constexpr int kDualMaxGroups = 1024;
@@ -334,6 +335,28 @@ __global__ void __launch_bounds__(kDualThreads, 1)
               }
             }
           }
+        } else if (p.out_f16) {
+          __half* out = static_cast<__half*>(p.out) + orow * p.ldo + col0;
+          bool range_ok = true;
+#pragma unroll 1
+          for (int c = 0; c < 256; c += 32) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(tbase + c, r);
+            tmem_ld_wait(r);
+            if (row_ok && col0 + c < p.N) {
+              uint32_t packed[16];
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                const float a = __uint_as_float(r[2 * e]), b = __uint_as_float(r[2 * e + 1]);
+                range_ok = range_ok && fabsf(a) <= 65504.f && fabsf(b) <= 65504.f;
+                __half2 hv = __floats2half2_rn(a, b);
+                packed[e] = *reinterpret_cast<uint32_t*>(&hv);
+              }
+              st_global_v8(out + c, packed);
+              st_global_v8(out + c + 16, packed + 8);
+            }
+          }
+          if (!range_ok) set_status(p.status, MOE_DEV_RANGE);
         } else {
           float* out = static_cast<float*>(p.out) + orow * p.ldo + col0;
 #pragma unroll 1

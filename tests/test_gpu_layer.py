@@ -54,12 +54,11 @@ SMALL = {
 
 
 # Cases whose max|err| against the exact-h oracle is above 2e-2 * RMS: the Mixtral-shaped
-# small layers (H=512, I=384), measured at 0.0208 (0.0159 against the bf16-h oracle), of
-# which 0.0159 is the floor that rounding the exact output once to bf16 already costs on
-# these 512,000-614,400 outputs.  Every other case
+# small layer (T=1000, H=512, I=384) in its three forms, measured at 0.0208 (0.0159 against
+# the bf16-h oracle), of which 0.0159 is the floor that rounding the exact output once to
+# bf16 already costs on these 512,000 outputs.  Every other case
 # asserts the max bound against the exact-h oracle as well.
-EXACT_MAX_EXCEEDS = {"mixtral_small", "mixtral_small_pair", "mixtral_small_fused", "mixtral_small_dual",
-                     "mixtral_small_dual_masked"}
+EXACT_MAX_EXCEEDS = {"mixtral_small", "mixtral_small_pair", "mixtral_small_fused"}
 
 
 def _both(x, ids, w, d, wl):
@@ -146,3 +145,18 @@ def test_host_entry_point_matches_device_entry_point():
                                      a["ws_down"], out_host, ws, ws.numel()))
     torch.cuda.synchronize()
     assert torch.equal(out_host, r["out"].cpu())
+
+
+def test_expert_output_beyond_fp16_range_is_reported():
+    """At prefill sizes the layer keeps routed expert outputs in fp16: one beyond 65504
+    must set MOE_DEV_RANGE (and nothing else) in the status word."""
+    wl = SMALL["mixtral_small_dual"]
+    d = inputs.make_inputs(wl, seed=0, device="cuda")
+    orig = d["w_down"]
+    # y has an RMS of ~0.04 here; scaled by 1e6 its largest values pass 65504
+    d["w_down"] = (orig.float() * 1.0e6).to(torch.bfloat16)
+    r = P.run_layer(wl, d)
+    assert B.moe_get_device_status(r["ws"]) == B.MOE_DEV_RANGE
+    d["w_down"] = orig
+    r = P.run_layer(wl, d)
+    assert B.moe_get_device_status(r["ws"]) == 0
