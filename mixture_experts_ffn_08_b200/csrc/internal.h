@@ -80,9 +80,11 @@ cudaError_t launch_masked_schedule(const int32_t* counts, int E, int32_t* sched,
 cudaError_t launch_bounded_wait_selftest(int32_t* status, long long limit_ns, cudaStream_t st);
 // offsets[e] = e * cap for e in [0, E] (masked layout row ranges).
 cudaError_t launch_masked_offsets(int E, int cap, int32_t* offsets, cudaStream_t st);
-// fill_pad: contiguous layout only, zero the pad rows of x_perm (scale 1 for FP8).  The
-// layer itself passes false: its GEMMs never store a pad row, and an MMA row depends on
-// its own A row only, so whatever the pad rows hold stays in rows nobody reads.
+// fill_pad: the moe_permute contract: contiguous layout, zero the pad rows of x_perm (scale 1
+// for FP8); both layouts, pair_of_row = -1 on rows without a pair.  The layer itself passes
+// false: its GEMMs never store a pad row and an MMA row depends on its own A row only, so
+// whatever the pad rows hold stays in rows nobody reads; x is then copied token by token
+// (each x row read once) instead of row by row.
 cudaError_t launch_permute(const moe_params_t& p, int block_m, const int32_t* ids, const void* x,
                            const float* x_scale, int32_t* counts, int32_t* offsets,
                            int32_t* row_of_pair, int32_t* pair_of_row, void* x_perm,

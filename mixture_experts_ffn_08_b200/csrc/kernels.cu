@@ -585,6 +585,53 @@ __global__ void __launch_bounds__(32 * kGatherWarps) perm_gather_kernel(
   }
 }
 
+// 4') token scatter, for the layer itself (no pad rows written, pair_of_row of pad rows not
+//     needed): one warp per token reads x[t] once and stores it to the bucket rows of its
+//     K pairs, so x crosses HBM once where the row gather re-reads each token K times.
+constexpr int kScatterWarps = 8;
+template <bool FP8>
+__global__ void __launch_bounds__(32 * kScatterWarps) perm_scatter_kernel(
+    const void* __restrict__ x, const float* __restrict__ x_scale, int T, int H, int K,
+    const int32_t* __restrict__ row_of_pair, void* __restrict__ x_perm, float* __restrict__ x_perm_scale) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int row_bytes = FP8 ? H : 2 * H;
+  const int nvec = row_bytes / 16;
+  const int nsc = H / 128;
+  const int warps = gridDim.x * kScatterWarps;
+  for (int t = blockIdx.x * kScatterWarps + (threadIdx.x >> 5); t < T; t += warps) {
+    const int my_row = lane < K ? __ldg(row_of_pair + static_cast<long long>(t) * K + lane) : -1;
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(x) + static_cast<long long>(t) * row_bytes);
+    for (int v0 = 0; v0 < nvec; v0 += 32 * 8) {
+      uint4 buf[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int v = v0 + 32 * u + lane;
+        buf[u] = v < nvec ? __ldg(src + v) : make_uint4(0, 0, 0, 0);
+      }
+      for (int k = 0; k < K; ++k) {
+        const int r = __shfl_sync(kFull, my_row, k);
+        if (r < 0) continue;  // a pair left out (masked layout) or with a bad expert id
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(x_perm) + static_cast<long long>(r) * row_bytes);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int v = v0 + 32 * u + lane;
+          if (v < nvec) dst[v] = buf[u];
+        }
+      }
+    }
+    if (FP8) {
+      for (int k = 0; k < K; ++k) {
+        const int r = __shfl_sync(kFull, my_row, k);
+        if (r < 0) continue;
+        for (int j = lane; j < nsc; j += 32)
+          x_perm_scale[static_cast<long long>(r) * nsc + j] = __ldg(x_scale + static_cast<long long>(t) * nsc + j);
+      }
+    }
+  }
+}
+
 cudaError_t launch_permute(const moe_params_t& p, int block_m, const int32_t* ids, const void* x,
                            const float* x_scale, int32_t* counts, int32_t* offsets,
                            int32_t* row_of_pair, int32_t* pair_of_row, void* x_perm,
@@ -624,6 +671,19 @@ cudaError_t launch_permute(const moe_params_t& p, int block_m, const int32_t* id
   }
   const bool masked = p.masked_cap > 0;
   const bool zero_pad = !masked && fill_pad;
+  if (!fill_pad && p.T > 0) {
+    const long long want = (static_cast<long long>(p.T) + kScatterWarps - 1) / kScatterWarps;
+    const int grid = static_cast<int>(want < num_sms() * 8LL ? want : num_sms() * 8LL);
+    trace_before(MOE_K_PERM_GATHER, st);
+    if (act_e4m3(p))
+      err = launch_k(perm_scatter_kernel<true>, grid, 32 * kScatterWarps, 0, st, x, x_scale, p.T, p.H, p.K,
+                     row_of_pair, x_perm, x_perm_scale);
+    else
+      err = launch_k(perm_scatter_kernel<false>, grid, 32 * kScatterWarps, 0, st, x, x_scale, p.T, p.H, p.K,
+                     row_of_pair, x_perm, x_perm_scale);
+    trace_after(MOE_K_PERM_GATHER, st);
+    return err != cudaSuccess ? err : cudaGetLastError();
+  }
   const long long max_rows = masked ? static_cast<long long>(p.E) * p.masked_cap
                                     : static_cast<long long>(P) + static_cast<long long>(p.E) * (bm - 1);
   const long long blocks = (max_rows + kGatherWarps - 1) / kGatherWarps;
