@@ -408,6 +408,12 @@ bool layer_y16(const moe_params_t* p, const int32_t* counts) {
   return two_tile_items(p, counts) && p->H % 256 == 0 && !is_fp8(p);
 }
 
+// The shared expert of a bf16 layer on one stream (prefill sizes: its T rows hold at least
+// two M-tiles) runs through the two-tile kernels as one dense group, y_sh in fp16.
+bool shared_two_tile(const moe_params_t* p) {
+  return !is_fp8(p) && p->T >= 256 && p->H % 256 == 0 && p->I_shared % 128 == 0;
+}
+
 moe_status_t do_expert_ffn(const moe_params_t* p, const void* x_perm, const int32_t* offsets,
                            const int32_t* counts, const void* w_gate, const void* w_up,
                            const void* w_down, float* y_perm, void* ws, cudaStream_t st, bool y16 = false) {
@@ -533,10 +539,24 @@ moe_status_t do_layer_after_fork(const moe_params_t* p, const void* x, const flo
   else
     MOE_TRY(do_expert_ffn(p, at<void>(ws, L.x_perm), offsets, counts, w_gate, w_up, w_down, y_perm, ws, st,
                           layer_y16(p, counts)));
-  if (side != nullptr) MOE_CUDA(cudaStreamWaitEvent(st, side->join, 0));
-  else if (p->I_shared > 0) MOE_TRY(do_shared(p, x, wsg, wsu, wsd, y_sh, ws, st));
+  bool ysh16 = false;
+  if (side != nullptr) {
+    MOE_CUDA(cudaStreamWaitEvent(st, side->join, 0));
+  } else if (p->I_shared > 0 && shared_two_tile(p)) {
+    // the dense shared expert at prefill sizes through the two-tile kernels, y_sh in fp16
+    const Layout Ls = layout(p);
+    int32_t* status = at<int32_t>(ws, Ls.status);
+    int32_t* ctr = at<int32_t>(ws, Ls.counter);
+    MOE_CUDA(gemm_gateup_swiglu_dual(x, p->T, nullptr, nullptr, 1, wsg, wsu, p->I_shared, p->H,
+                                     at<void>(ws, Ls.h_sh), ctr, status, st, 0, MOE_K_SHARED_GATEUP));
+    MOE_CUDA(gemm_down_dual(at<void>(ws, Ls.h_sh), p->T, nullptr, nullptr, 1, wsd, p->H, p->I_shared, y_sh,
+                            ctr + 1, status, st, 0, /*y_f16=*/true, MOE_K_SHARED_DOWN));
+    ysh16 = true;
+  } else if (p->I_shared > 0) {
+    MOE_TRY(do_shared(p, x, wsg, wsu, wsd, y_sh, ws, st));
+  }
   return cuda_status(launch_combine(*p, y_perm, rop, w, p->I_shared > 0 ? y_sh : nullptr, out, st,
-                                    layer_y16(p, counts)));
+                                    layer_y16(p, counts), ysh16));
 }
 
 moe_status_t check_layer_args(const moe_params_t* p, const void* x, const float* x_scale, const void* w_r,

@@ -132,7 +132,7 @@ cudaError_t gemm_gateup_swiglu(const void* A, int64_t a_rows, const int32_t* off
 
 cudaError_t gemm_gateup_swiglu_dual(const void* A, int64_t a_rows, const int32_t* offsets, const int32_t* counts,
                                     int G, const void* w_gate, const void* w_up, int N, int K, void* h,
-                                    int32_t* counter, int32_t* status, cudaStream_t st, int masked_cap) {
+                                    int32_t* counter, int32_t* status, cudaStream_t st, int masked_cap, int kid) {
   if (G > kDualMaxGroups || N % 128 != 0 || K % 64 != 0) return cudaErrorInvalidValue;
   CUtensorMap ta, tg, tu;
   if (!make_tmap_bf16(&ta, A, a_rows, K, 128) ||
@@ -142,7 +142,8 @@ cudaError_t gemm_gateup_swiglu_dual(const void* A, int64_t a_rows, const int32_t
   DualParams dp{};
   dp.offsets = offsets;
   dp.counts = counts;
-  dp.G = G;
+  dp.dense_rows = static_cast<int>(a_rows);  // used when offsets is null (one dense group)
+  dp.G = offsets != nullptr ? G : 1;
   dp.K = K;
   dp.N = N;
   dp.masked_cap = masked_cap;
@@ -157,15 +158,15 @@ cudaError_t gemm_gateup_swiglu_dual(const void* A, int64_t a_rows, const int32_t
   const long long max_items = ceil_div(a_rows, 128) * (N / 128);
   const long long sms = num_sms();
   const int grid = static_cast<int>(max_items < sms ? (max_items > 0 ? max_items : 1) : sms);
-  trace_before(MOE_K_GATEUP, st);
+  trace_before(kid, st);
   err = launch_k(tc_gemm_dual_kernel<true>, grid, kDualThreads, kDualSmemBytes, st, ta, tg, tu, dp);
-  trace_after(MOE_K_GATEUP, st);
+  trace_after(kid, st);
   return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 cudaError_t gemm_down_dual(const void* A, int64_t a_rows, const int32_t* offsets, const int32_t* counts, int G,
                            const void* w, int N, int K, void* y, int32_t* counter, int32_t* status, cudaStream_t st,
-                           int masked_cap, bool y_f16) {
+                           int masked_cap, bool y_f16, int kid) {
   if (G > kDualMaxGroups || N % 256 != 0 || K % 64 != 0) return cudaErrorInvalidValue;
   CUtensorMap ta, tb;
   if (!make_tmap_bf16(&ta, A, a_rows, K, 128) || !make_tmap_bf16(&tb, w, static_cast<uint64_t>(G) * N, K, 256))
@@ -173,7 +174,8 @@ cudaError_t gemm_down_dual(const void* A, int64_t a_rows, const int32_t* offsets
   DualParams dp{};
   dp.offsets = offsets;
   dp.counts = counts;
-  dp.G = G;
+  dp.dense_rows = static_cast<int>(a_rows);  // used when offsets is null (one dense group)
+  dp.G = offsets != nullptr ? G : 1;
   dp.K = K;
   dp.N = N;
   dp.masked_cap = masked_cap;
@@ -189,9 +191,9 @@ cudaError_t gemm_down_dual(const void* A, int64_t a_rows, const int32_t* offsets
   const long long max_items = ceil_div(a_rows, 128) * (N / 256);
   const long long sms = num_sms();
   const int grid = static_cast<int>(max_items < sms ? (max_items > 0 ? max_items : 1) : sms);
-  trace_before(MOE_K_DOWN, st);
+  trace_before(kid, st);
   err = launch_k(tc_gemm_dual_kernel<false>, grid, kDualThreads, kDualSmemBytes, st, ta, tb, tb, dp);
-  trace_after(MOE_K_DOWN, st);
+  trace_after(kid, st);
   return err != cudaSuccess ? err : cudaGetLastError();
 }
 

@@ -93,8 +93,10 @@ cudaError_t launch_permute(const moe_params_t& p, int block_m, const int32_t* id
 
 // ---------------------------------------------------------------- combine (kernels.cu)
 // y_perm is fp32 for bf16 workloads and bf16 for FP8 workloads (p.dtype).
+// y_shared: [T,H] fp32, or fp16 when ysh_f16.
 cudaError_t launch_combine(const moe_params_t& p, const void* y_perm, const int32_t* row_of_pair,
-                           const float* w, const float* y_shared, void* out, cudaStream_t st, bool y_f16 = false);
+                           const float* w, const void* y_shared, void* out, cudaStream_t st, bool y_f16 = false,
+                           bool ysh_f16 = false);
 
 // ---------------------------------------------------------------- GEMMs (gemm.cu)
 // Router logits x [T,H] bf16 @ W_r[E,H]^T as router_k_splits(T, H, E) fp32 partial
@@ -109,13 +111,15 @@ cudaError_t gemm_gateup_swiglu(const void* A, int64_t a_rows, const int32_t* off
                                cudaStream_t st, int masked_cap = 0);
 // The same gate/up projection with two M-tiles of an expert per work item (grouped, with
 // counts, N multiple of 128); counter is a device int the call zeroes before the launch.
+// offsets == nullptr: one dense group of a_rows rows (counts unused).
 cudaError_t gemm_gateup_swiglu_dual(const void* A, int64_t a_rows, const int32_t* offsets, const int32_t* counts,
                                     int G, const void* w_gate, const void* w_up, int N, int K, void* h,
-                                    int32_t* counter, int32_t* status, cudaStream_t st, int masked_cap = 0);
+                                    int32_t* counter, int32_t* status, cudaStream_t st, int masked_cap = 0,
+                                    int kid = MOE_K_GATEUP);
 // The down projection with two M-tiles per work item (N multiple of 256); counter as above.
 cudaError_t gemm_down_dual(const void* A, int64_t a_rows, const int32_t* offsets, const int32_t* counts, int G,
                            const void* w, int N, int K, void* y, int32_t* counter, int32_t* status, cudaStream_t st,
-                           int masked_cap = 0, bool y_f16 = false);
+                           int masked_cap = 0, bool y_f16 = false, int kid = MOE_K_DOWN);
 // y [rows, N] fp32 = A W^T, grouped by offsets (or dense when null); with counts, pad
 // rows of each group are not stored.
 cudaError_t gemm_down(const void* A, int64_t a_rows, const int32_t* offsets,

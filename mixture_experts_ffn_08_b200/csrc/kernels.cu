@@ -774,11 +774,11 @@ MOE_DEVINL void load8(const __half* row, int v, float (&f)[8]) {
   }
 }
 
-// out[t] = sum_k w[t,k] y_perm[row_of_pair[t*K+k]] (+ y_sh[t]); YT = float, bf16 or fp16.
-template <class YT>
+// out[t] = sum_k w[t,k] y_perm[row_of_pair[t*K+k]] (+ y_sh[t]); YT, ST = float, bf16 or fp16.
+template <class YT, class ST>
 __global__ void __launch_bounds__(128) combine_kernel(
     const YT* __restrict__ y_perm, const int32_t* __restrict__ row_of_pair,
-    const float* __restrict__ w, const float* __restrict__ y_sh,
+    const float* __restrict__ w, const ST* __restrict__ y_sh,
     __nv_bfloat16* __restrict__ out, int T, int H, int K) {
   pdl_launch_dependents();
   pdl_wait();
@@ -839,20 +839,30 @@ cudaError_t launch_f32_to_bf16(const float* acc, long long n, void* out, cudaStr
 }
 
 cudaError_t launch_combine(const moe_params_t& p, const void* y_perm, const int32_t* row_of_pair,
-                           const float* w, const float* y_shared, void* out, cudaStream_t st, bool y_f16) {
+                           const float* w, const void* y_shared, void* out, cudaStream_t st, bool y_f16,
+                           bool ysh_f16) {
   if (p.T == 0) return cudaSuccess;
   const int grid = p.T < num_sms() * 16 ? p.T : num_sms() * 16;
   trace_before(MOE_K_COMBINE, st);
   cudaError_t err;
-  if (y_f16)
-    err = launch_k(combine_kernel<__half>, grid, 128, 0, st, static_cast<const __half*>(y_perm), row_of_pair, w,
-                   y_shared, static_cast<__nv_bfloat16*>(out), p.T, p.H, p.K);
+  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
+  const float* ys32 = static_cast<const float*>(y_shared);
+  const __half* ys16 = static_cast<const __half*>(y_shared);
+  if (y_f16 && ysh_f16)
+    err = launch_k(combine_kernel<__half, __half>, grid, 128, 0, st, static_cast<const __half*>(y_perm), row_of_pair,
+                   w, ys16, o, p.T, p.H, p.K);
+  else if (y_f16)
+    err = launch_k(combine_kernel<__half, float>, grid, 128, 0, st, static_cast<const __half*>(y_perm), row_of_pair,
+                   w, ys32, o, p.T, p.H, p.K);
+  else if (ysh_f16)
+    err = launch_k(combine_kernel<float, __half>, grid, 128, 0, st, static_cast<const float*>(y_perm), row_of_pair,
+                   w, ys16, o, p.T, p.H, p.K);
   else if (act_e4m3(p))
-    err = launch_k(combine_kernel<__nv_bfloat16>, grid, 128, 0, st, static_cast<const __nv_bfloat16*>(y_perm),
-                   row_of_pair, w, y_shared, static_cast<__nv_bfloat16*>(out), p.T, p.H, p.K);
+    err = launch_k(combine_kernel<__nv_bfloat16, float>, grid, 128, 0, st,
+                   static_cast<const __nv_bfloat16*>(y_perm), row_of_pair, w, ys32, o, p.T, p.H, p.K);
   else
-    err = launch_k(combine_kernel<float>, grid, 128, 0, st, static_cast<const float*>(y_perm), row_of_pair, w,
-                   y_shared, static_cast<__nv_bfloat16*>(out), p.T, p.H, p.K);
+    err = launch_k(combine_kernel<float, float>, grid, 128, 0, st, static_cast<const float*>(y_perm), row_of_pair,
+                   w, ys32, o, p.T, p.H, p.K);
   trace_after(MOE_K_COMBINE, st);
   return err != cudaSuccess ? err : cudaGetLastError();
 }

@@ -32,8 +32,10 @@
 namespace moe {
 
 struct DualParams {
-  const int32_t* offsets;   // [G+1] schedule: first row of each group, multiples of 128
+  const int32_t* offsets;   // [G+1] schedule: first row of each group, multiples of 128;
+                            // nullptr: one dense group of dense_rows rows (G = 1)
   const int32_t* counts;    // [G] real rows of each group (rows past it are not stored)
+  int dense_rows;
   int G;                    // groups (G <= kDualMaxGroups)
   int K;                    // reduction length, multiple of 64
   int N;                    // output columns; weight rows per group (and matrix, for SwiGLU)
@@ -69,6 +71,14 @@ struct DualItem {
 // pairs(e) = ceil(tiles(e) / 2).  Inside a group, weight tiles are outer (every pair of
 // M-tiles in flight shares each weight tile) unless the group's activation rows outnumber
 // its weight rows (NT * 256), as for a very hot expert, where pairs are outer.
+// First row of group g in the schedule (g = G: the end), and its real rows.
+MOE_DEVINL int group_row(const DualParams& p, int g) {
+  return p.offsets != nullptr ? __ldg(p.offsets + g) : (g == 0 ? 0 : (p.dense_rows + 127) / 128 * 128);
+}
+MOE_DEVINL int group_count(const DualParams& p, int g) {
+  return p.offsets != nullptr ? __ldg(p.counts + g) : p.dense_rows;
+}
+
 MOE_DEVINL DualItem dual_decode(int item, int NT, const DualParams& p, const int* pref) {
   // (NT * 256 is the group's weight rows in both forms: SwiGLU tiles hold 256 rows too)
   int lo = 0, hi = p.G - 1;  // group with pref[g] <= item < pref[g+1]
@@ -77,8 +87,8 @@ MOE_DEVINL DualItem dual_decode(int item, int NT, const DualParams& p, const int
     if (pref[mid] <= item) lo = mid; else hi = mid - 1;
   }
   const int g = lo;
-  const int mt0 = __ldg(p.offsets + g) >> 7;
-  const int tiles = (__ldg(p.offsets + g + 1) >> 7) - mt0;
+  const int mt0 = group_row(p, g) >> 7;
+  const int tiles = (group_row(p, g + 1) >> 7) - mt0;
   const int pairs = (tiles + 1) >> 1;
   const int local = item - pref[g];
   const bool pairs_outer = tiles * 128 > NT * 256;
@@ -158,7 +168,7 @@ __global__ void __launch_bounds__(kDualThreads, 1)
     const int g0 = lane * per;
     int run = 0;
     for (int g = g0; g < g0 + per && g < p.G; ++g) {
-      const int tiles = (__ldg(p.offsets + g + 1) - __ldg(p.offsets + g)) >> 7;
+      const int tiles = (group_row(p, g + 1) - group_row(p, g)) >> 7;
       run += NT * ((tiles + 1) >> 1);
     }
     int incl = run;
@@ -170,7 +180,7 @@ __global__ void __launch_bounds__(kDualThreads, 1)
     int acc = incl - run;
     for (int g = g0; g < g0 + per && g < p.G; ++g) {
       pref[g] = acc;
-      const int tiles = (__ldg(p.offsets + g + 1) - __ldg(p.offsets + g)) >> 7;
+      const int tiles = (group_row(p, g + 1) - group_row(p, g)) >> 7;
       acc += NT * ((tiles + 1) >> 1);
     }
     if (lane == 31) pref[p.G] = incl;
@@ -242,7 +252,7 @@ __global__ void __launch_bounds__(kDualThreads, 1)
         for (int u = 0; u < d.ntiles; ++u) {
           const int slot = u == 0 ? slot0 : slot1;
           if (!mbar_wait_bounded(&tempty_bar[slot], (uses[slot] & 1u) ^ 1u, &abort_flag)) { ok = false; break; }
-          const int rows = __ldg(p.counts + d.group) - (d.tile0 + u - d.mt0) * 128;
+          const int rows = group_count(p, d.group) - (d.tile0 + u - d.mt0) * 128;
           idesc[u] = rows <= 64 ? IDESC_HALF : IDESC;
         }
         if (!ok) break;
@@ -295,7 +305,7 @@ __global__ void __launch_bounds__(kDualThreads, 1)
       const DualItem d = dual_decode(it, NT, p, pref);
       const int slot0 = nxt, slot1 = nxt ^ 1;
       if (d.ntiles == 1) nxt ^= 1;
-      const int count = __ldg(p.counts + d.group);
+      const int count = group_count(p, d.group);
       const int col0 = d.n_tile * OUT_COLS;
       for (int u = 0; u < d.ntiles && ok; ++u) {
         const int slot = u == 0 ? slot0 : slot1;

@@ -41,6 +41,13 @@ SMALL = {
     "dsv3_small_dual": W.DSV3_PREFILL.with_(name="dsv3_small_dual", T=1100, H=512, I=256, E=32, I_shared=256),
     "mixtral_small_dual_masked": W.MIXTRAL_PREFILL.with_(name="mixtral_small_dual_masked", T=1200, H=512, I=384,
                                                          masked_cap=640),
+    # more than 16384 pairs: the shared expert runs on the caller's stream through the
+    # two-tile kernels as one dense group with an fp16 output, beside fp32 routed outputs
+    # (T*K < 256*E) or fp16 ones (T*K >= 256*E)
+    "dsv3_small_shared_dense": W.DSV3_PREFILL.with_(name="dsv3_small_shared_dense", T=2100, H=512, I=256,
+                                                    E=128, I_shared=256),
+    "dsv3_small_shared_dense_y16": W.DSV3_PREFILL.with_(name="dsv3_small_shared_dense_y16", T=2100, H=512,
+                                                        I=256, E=64, I_shared=256),
     # buckets aligned to 256 rows: the two-SM (cta_group::2) GEMMs
     "mixtral_small_pair": W.MIXTRAL_PREFILL.with_(name="mixtral_small_pair", T=1000, H=512, I=384, block_m=256),
     "dsv3_small_pair": W.DSV3_PREFILL.with_(name="dsv3_small_pair", T=300, H=512, I=256, E=32, I_shared=256,
