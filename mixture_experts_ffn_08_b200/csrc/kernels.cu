@@ -115,7 +115,25 @@ __global__ void __launch_bounds__(128) topk_kernel(
     const int e = j * 32 + lane;
     s[j] = e < E ? __ldg(z + e) : -CUDART_INF_F;
   }
-  for (int part = 1; part < n_part; ++part) {
+  // (U slices' loads in flight at once, then added in slice order: the same sum)
+  constexpr int U = EPL <= 8 ? 4 : 1;
+  int part = 1;
+  for (; part + U <= n_part; part += U) {
+    float a[U][EPL];
+#pragma unroll
+    for (int q = 0; q < U; ++q)
+#pragma unroll
+      for (int j = 0; j < EPL; ++j) {
+        const int e = j * 32 + lane;
+        a[q][j] = e < E ? __ldg(z + (part + q) * part_stride + e) : 0.f;
+      }
+#pragma unroll
+    for (int q = 0; q < U; ++q)
+#pragma unroll
+      for (int j = 0; j < EPL; ++j)
+        if (j * 32 + lane < E) s[j] += a[q][j];
+  }
+  for (; part < n_part; ++part) {
 #pragma unroll
     for (int j = 0; j < EPL; ++j) {
       const int e = j * 32 + lane;
@@ -586,8 +604,10 @@ __global__ void __launch_bounds__(32 * kGatherWarps) perm_gather_kernel(
 }
 
 // 4') token scatter, for the layer itself (no pad rows written, pair_of_row of pad rows not
-//     needed): one warp per token reads x[t] once and stores it to the bucket rows of its
-//     K pairs, so x crosses HBM once where the row gather re-reads each token K times.
+//     needed): a warp reads a 256-vector (4 or 8 KB) piece of x[t] once and stores it to the
+//     bucket rows of its K pairs, so x crosses HBM once where the row gather re-reads each
+//     token K times.  Work units are (token, piece), so a decode-sized batch still spreads
+//     over the SMs.
 constexpr int kScatterWarps = 8;
 template <bool FP8>
 __global__ void __launch_bounds__(32 * kScatterWarps) perm_scatter_kernel(
@@ -599,11 +619,16 @@ __global__ void __launch_bounds__(32 * kScatterWarps) perm_scatter_kernel(
   const int row_bytes = FP8 ? H : 2 * H;
   const int nvec = row_bytes / 16;
   const int nsc = H / 128;
+  const int nchunk = (nvec + 255) / 256;
+  const long long units = static_cast<long long>(T) * nchunk;
   const int warps = gridDim.x * kScatterWarps;
-  for (int t = blockIdx.x * kScatterWarps + (threadIdx.x >> 5); t < T; t += warps) {
+  for (long long u = blockIdx.x * kScatterWarps + (threadIdx.x >> 5); u < units; u += warps) {
+    const int t = static_cast<int>(u / nchunk);
+    const int chunk = static_cast<int>(u % nchunk);
     const int my_row = lane < K ? __ldg(row_of_pair + static_cast<long long>(t) * K + lane) : -1;
     const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(x) + static_cast<long long>(t) * row_bytes);
-    for (int v0 = 0; v0 < nvec; v0 += 32 * 8) {
+    {
+      const int v0 = chunk * 256;
       uint4 buf[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
@@ -621,7 +646,7 @@ __global__ void __launch_bounds__(32 * kScatterWarps) perm_scatter_kernel(
         }
       }
     }
-    if (FP8) {
+    if (FP8 && chunk == 0) {
       for (int k = 0; k < K; ++k) {
         const int r = __shfl_sync(kFull, my_row, k);
         if (r < 0) continue;
@@ -672,7 +697,9 @@ cudaError_t launch_permute(const moe_params_t& p, int block_m, const int32_t* id
   const bool masked = p.masked_cap > 0;
   const bool zero_pad = !masked && fill_pad;
   if (!fill_pad && p.T > 0) {
-    const long long want = (static_cast<long long>(p.T) + kScatterWarps - 1) / kScatterWarps;
+    const long long row_vecs = (act_e4m3(p) ? p.H : 2LL * p.H) / 16;
+    const long long units = static_cast<long long>(p.T) * ((row_vecs + 255) / 256);
+    const long long want = (units + kScatterWarps - 1) / kScatterWarps;
     const int grid = static_cast<int>(want < num_sms() * 8LL ? want : num_sms() * 8LL);
     trace_before(MOE_K_PERM_GATHER, st);
     if (act_e4m3(p))
@@ -775,6 +802,8 @@ MOE_DEVINL void load8(const __half* row, int v, float (&f)[8]) {
 }
 
 // out[t] = sum_k w[t,k] y_perm[row_of_pair[t*K+k]] (+ y_sh[t]); YT, ST = float, bf16 or fp16.
+// One block per token; 32 registers, so 16 blocks share an SM and keep enough loads in
+// flight for large batches.
 template <class YT, class ST>
 __global__ void __launch_bounds__(128) combine_kernel(
     const YT* __restrict__ y_perm, const int32_t* __restrict__ row_of_pair,
@@ -816,6 +845,63 @@ __global__ void __launch_bounds__(128) combine_kernel(
   }
 }
 
+// The same sum for decode-sized batches (T < 8 * SMs): a block takes one of `pieces` pieces
+// of a token's H/8 output vectors, so the batch still spreads over the SMs, and each thread
+// loads the rows of four pairs before it adds them, in k order (the same sum as one row at
+// a time, with four loads in flight instead of one).
+template <class YT, class ST>
+__global__ void __launch_bounds__(128) combine_pieces_kernel(
+    const YT* __restrict__ y_perm, const int32_t* __restrict__ row_of_pair,
+    const float* __restrict__ w, const ST* __restrict__ y_sh,
+    __nv_bfloat16* __restrict__ out, int T, int H, int K, int pieces) {
+  pdl_launch_dependents();
+  pdl_wait();
+  __shared__ int rows[kMaxTopK];
+  __shared__ float wk[kMaxTopK];
+  const int nvec = H / 8;
+  const int span = (nvec + pieces - 1) / pieces;
+  const int units = T * pieces;
+  for (int u = blockIdx.x; u < units; u += gridDim.x) {
+    const int t = u / pieces;
+    const int v0 = (u - t * pieces) * span;
+    const int v1 = v0 + span < nvec ? v0 + span : nvec;
+    __syncthreads();
+    if (threadIdx.x < K) {
+      rows[threadIdx.x] = __ldg(row_of_pair + static_cast<long long>(t) * K + threadIdx.x);
+      wk[threadIdx.x] = __ldg(w + static_cast<long long>(t) * K + threadIdx.x);
+    }
+    __syncthreads();
+    for (int v = v0 + threadIdx.x; v < v1; v += blockDim.x) {
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      for (int k0 = 0; k0 < K; k0 += 4) {
+        int r[4];
+        float f[4][8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          r[j] = k0 + j < K ? rows[k0 + j] : -1;
+          if (r[j] >= 0) load8(y_perm + static_cast<long long>(r[j]) * H, v, f[j]);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (r[j] < 0) continue;
+          const float wv = wk[k0 + j];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[i] = fmaf(wv, f[j][i], acc[i]);
+        }
+      }
+      if (y_sh) {
+        float f[8];
+        load8(y_sh + static_cast<long long>(t) * H, v, f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] += f[i];
+      }
+      reinterpret_cast<uint4*>(out + static_cast<long long>(t) * H)[v] =
+          make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                     pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+    }
+  }
+}
+
 __global__ void f32_to_bf16_kernel(const float* __restrict__ acc, long long n8, __nv_bfloat16* __restrict__ out) {
   pdl_launch_dependents();
   pdl_wait();
@@ -838,31 +924,42 @@ cudaError_t launch_f32_to_bf16(const float* acc, long long n, void* out, cudaStr
   return err != cudaSuccess ? err : cudaGetLastError();
 }
 
+// Launches combine_kernel (pieces == 0) or combine_pieces_kernel for the output types.
+template <class YT, class ST>
+cudaError_t launch_combine_t(const moe_params_t& p, const void* y_perm, const int32_t* row_of_pair, const float* w,
+                             const void* y_shared, void* out, cudaStream_t st, int grid, int pieces) {
+  const YT* y = static_cast<const YT*>(y_perm);
+  const ST* ys = static_cast<const ST*>(y_shared);
+  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
+  if (pieces == 0) return launch_k(combine_kernel<YT, ST>, grid, 128, 0, st, y, row_of_pair, w, ys, o, p.T, p.H, p.K);
+  return launch_k(combine_pieces_kernel<YT, ST>, grid, 128, 0, st, y, row_of_pair, w, ys, o, p.T, p.H, p.K, pieces);
+}
+
 cudaError_t launch_combine(const moe_params_t& p, const void* y_perm, const int32_t* row_of_pair,
                            const float* w, const void* y_shared, void* out, cudaStream_t st, bool y_f16,
                            bool ysh_f16) {
   if (p.T == 0) return cudaSuccess;
-  const int grid = p.T < num_sms() * 16 ? p.T : num_sms() * 16;
+  int grid = p.T < num_sms() * 16 ? p.T : num_sms() * 16;
+  int pieces = 0;
+  if (p.T < num_sms() * 8) {
+    // pieces per token: about eight blocks per SM, at most one piece per 128 vectors
+    const int max_pieces = (p.H / 8 + 127) / 128;
+    const int want = (num_sms() * 8 + p.T - 1) / p.T;
+    pieces = want > max_pieces ? max_pieces : want;
+    grid = p.T * pieces;
+  }
   trace_before(MOE_K_COMBINE, st);
   cudaError_t err;
-  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
-  const float* ys32 = static_cast<const float*>(y_shared);
-  const __half* ys16 = static_cast<const __half*>(y_shared);
   if (y_f16 && ysh_f16)
-    err = launch_k(combine_kernel<__half, __half>, grid, 128, 0, st, static_cast<const __half*>(y_perm), row_of_pair,
-                   w, ys16, o, p.T, p.H, p.K);
+    err = launch_combine_t<__half, __half>(p, y_perm, row_of_pair, w, y_shared, out, st, grid, pieces);
   else if (y_f16)
-    err = launch_k(combine_kernel<__half, float>, grid, 128, 0, st, static_cast<const __half*>(y_perm), row_of_pair,
-                   w, ys32, o, p.T, p.H, p.K);
+    err = launch_combine_t<__half, float>(p, y_perm, row_of_pair, w, y_shared, out, st, grid, pieces);
   else if (ysh_f16)
-    err = launch_k(combine_kernel<float, __half>, grid, 128, 0, st, static_cast<const float*>(y_perm), row_of_pair,
-                   w, ys16, o, p.T, p.H, p.K);
+    err = launch_combine_t<float, __half>(p, y_perm, row_of_pair, w, y_shared, out, st, grid, pieces);
   else if (act_e4m3(p))
-    err = launch_k(combine_kernel<__nv_bfloat16, float>, grid, 128, 0, st,
-                   static_cast<const __nv_bfloat16*>(y_perm), row_of_pair, w, ys32, o, p.T, p.H, p.K);
+    err = launch_combine_t<__nv_bfloat16, float>(p, y_perm, row_of_pair, w, y_shared, out, st, grid, pieces);
   else
-    err = launch_k(combine_kernel<float, float>, grid, 128, 0, st, static_cast<const float*>(y_perm), row_of_pair,
-                   w, ys32, o, p.T, p.H, p.K);
+    err = launch_combine_t<float, float>(p, y_perm, row_of_pair, w, y_shared, out, st, grid, pieces);
   trace_after(MOE_K_COMBINE, st);
   return err != cudaSuccess ? err : cudaGetLastError();
 }

@@ -205,18 +205,17 @@ __global__ void __launch_bounds__(kDualThreads, 1)
         if (it >= total) break;
         const DualItem d = dual_decode(it, NT, p, pref);
         const int b_row = d.group * p.N + d.n_tile * OUT_COLS;
-        int a_row[2];
-        for (int u = 0; u < 2; ++u) {
-          const int local0 = (d.tile0 + u - d.mt0) * 128;
-          a_row[u] = p.masked_cap > 0 ? d.group * p.masked_cap + local0 : (d.tile0 + u) * 128;
-        }
+        // (scalars, not arrays: an array indexed at run time lives in local memory)
+        const int local0 = (d.tile0 - d.mt0) * 128;
+        const int a_row0 = p.masked_cap > 0 ? d.group * p.masked_cap + local0 : d.tile0 * 128;
+        const int a_row1 = a_row0 + 128;
         const uint32_t tx = static_cast<uint32_t>(d.ntiles * kDualABytes + kDualBBytes);
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, &abort_flag)) { ok = false; break; }
           uint8_t* st = smem + s * kDualStageBytes;
           mbar_arrive_expect_tx(&full_bar[s], tx);
-          tma_load_2d(st, &tmA, kb * BK, a_row[0], &full_bar[s]);
-          if (d.ntiles == 2) tma_load_2d(st + kDualABytes, &tmA, kb * BK, a_row[1], &full_bar[s]);
+          tma_load_2d(st, &tmA, kb * BK, a_row0, &full_bar[s]);
+          if (d.ntiles == 2) tma_load_2d(st + kDualABytes, &tmA, kb * BK, a_row1, &full_bar[s]);
           tma_load_2d(st + 2 * kDualABytes, &tmG, kb * BK, b_row, &full_bar[s]);
           if (SWIGLU) tma_load_2d(st + 2 * kDualABytes + kDualBBytes / 2, &tmU, kb * BK, b_row, &full_bar[s]);
           ++issued;
@@ -236,7 +235,7 @@ __global__ void __launch_bounds__(kDualThreads, 1)
     if (lane == 0) {
       int s = 0, nxt = 0;
       uint32_t ph = 0;
-      uint32_t uses[2] = {0u, 0u};
+      uint32_t uses = 0u;  // bit a: phase of slot a's accumulator
       bool ok = true;
       for (int i = 0; ok; ++i) {
         const int rs = i % R;
@@ -248,14 +247,12 @@ __global__ void __launch_bounds__(kDualThreads, 1)
         const DualItem d = dual_decode(it, NT, p, pref);
         const int slot0 = nxt, slot1 = nxt ^ 1;
         if (d.ntiles == 1) nxt ^= 1;
-        uint32_t idesc[2];
-        for (int u = 0; u < d.ntiles; ++u) {
-          const int slot = u == 0 ? slot0 : slot1;
-          if (!mbar_wait_bounded(&tempty_bar[slot], (uses[slot] & 1u) ^ 1u, &abort_flag)) { ok = false; break; }
-          const int rows = group_count(p, d.group) - (d.tile0 + u - d.mt0) * 128;
-          idesc[u] = rows <= 64 ? IDESC_HALF : IDESC;
-        }
-        if (!ok) break;
+        const int rows0 = group_count(p, d.group) - (d.tile0 - d.mt0) * 128;
+        const uint32_t idesc0 = rows0 <= 64 ? IDESC_HALF : IDESC;
+        const uint32_t idesc1 = rows0 - 128 <= 64 ? IDESC_HALF : IDESC;
+        if (!mbar_wait_bounded(&tempty_bar[slot0], ((uses >> slot0) & 1u) ^ 1u, &abort_flag)) { ok = false; break; }
+        if (d.ntiles == 2 &&
+            !mbar_wait_bounded(&tempty_bar[slot1], ((uses >> slot1) & 1u) ^ 1u, &abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d0 = tmem_base + slot0 * 256, d1 = tmem_base + slot1 * 256;
         for (int kb = 0; kb < KB; ++kb) {
@@ -267,18 +264,18 @@ __global__ void __launch_bounds__(kDualThreads, 1)
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
             const uint32_t acc = (kb | k) != 0;
-            umma_f16(d0, smem_desc_sw128(a0 + k * 32), smem_desc_sw128(b0 + k * 32), idesc[0], acc);
-            if (d.ntiles == 2) umma_f16(d1, smem_desc_sw128(a1 + k * 32), smem_desc_sw128(b0 + k * 32), idesc[1], acc);
+            umma_f16(d0, smem_desc_sw128(a0 + k * 32), smem_desc_sw128(b0 + k * 32), idesc0, acc);
+            if (d.ntiles == 2) umma_f16(d1, smem_desc_sw128(a1 + k * 32), smem_desc_sw128(b0 + k * 32), idesc1, acc);
           }
           umma_commit(&empty_bar[s]);
           if (++s == STAGES) { s = 0; ph ^= 1u; }
         }
         if (!ok) break;
         umma_commit(&tfull_bar[slot0]);
-        ++uses[slot0];
+        uses ^= 1u << slot0;
         if (d.ntiles == 2) {
           umma_commit(&tfull_bar[slot1]);
-          ++uses[slot1];
+          uses ^= 1u << slot1;
         }
       }
       umma_commit(&drain_bar);
@@ -290,7 +287,7 @@ __global__ void __launch_bounds__(kDualThreads, 1)
     // ---------------------------------------------------------------- SwiGLU epilogue
     const int q = warp & 3;
     int nxt = 0;
-    uint32_t uses[2] = {0u, 0u};
+    uint32_t uses = 0u;  // bit a: phase of slot a's accumulator
     const bool v8 = ((reinterpret_cast<uintptr_t>(p.out) | (static_cast<uintptr_t>(p.ldo) * (SWIGLU ? 2 : 4))) & 31) == 0;
     bool ok = true;
     for (int i = 0; ok; ++i) {
@@ -309,7 +306,7 @@ __global__ void __launch_bounds__(kDualThreads, 1)
       const int col0 = d.n_tile * OUT_COLS;
       for (int u = 0; u < d.ntiles && ok; ++u) {
         const int slot = u == 0 ? slot0 : slot1;
-        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&tfull_bar[slot], uses[slot] & 1u, &abort_flag));
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&tfull_bar[slot], (uses >> slot) & 1u, &abort_flag));
         if (!ok) break;
         tc_fence_after();
         const int local0 = (d.tile0 + u - d.mt0) * 128;
@@ -388,7 +385,7 @@ __global__ void __launch_bounds__(kDualThreads, 1)
         }
         tc_fence_before();
         mbar_arrive(&tempty_bar[slot]);
-        ++uses[slot];
+        uses ^= 1u << slot;
       }
     }
   }
