@@ -387,6 +387,8 @@ __global__ void __launch_bounds__(kPermChunk) perm_count_kernel(
 // 2) one block: expert totals, padded exclusive scan -> offsets, and per-chunk bases
 //    (chunk_counts is overwritten with the first row of each (chunk, expert) run).
 //    cap > 0 (masked layout): every expert spans cap rows, counts are capped at cap.
+//    Thread (part, e) handles expert e over one of 1024 / E contiguous ranges of chunks,
+//    so all 1024 threads walk the chunk table, not only E of them.
 __global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t* __restrict__ chunk_counts,
                                                          int nchunks, int E, int block_m, int cap,
                                                          int32_t* __restrict__ counts,
@@ -395,10 +397,29 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t* __restrict__ c
   pdl_launch_dependents();
   pdl_wait();
   __shared__ int warp_tot[32];
-  const int e = threadIdx.x, lane = e & 31, w = e >> 5;
+  __shared__ int part_run[1024];        // [part][E]: pairs of expert e in the part's chunks, then
+                                        // the pairs of e in the parts before it
+  __shared__ int first_row[kMaxExperts];
+  const int tid = threadIdx.x;
+  const int parts = E <= 1024 ? 1024 / E : 1;
+  const int per = (nchunks + parts - 1) / parts;
+  const int my_part = tid / E, my_e = tid - my_part * E;
+  const bool walker = my_part < parts;
+  const int c0 = my_part * per, c1 = c0 + per < nchunks ? c0 + per : nchunks;
+  if (walker) {
+    int sum = 0;
+    for (int c = c0; c < c1; ++c) sum += chunk_counts[static_cast<long long>(c) * E + my_e];
+    part_run[tid] = sum;
+  }
+  __syncthreads();
+  const int e = tid, lane = e & 31, w = e >> 5;
   int total = 0;
   if (e < E)
-    for (int c = 0; c < nchunks; ++c) total += chunk_counts[static_cast<long long>(c) * E + e];
+    for (int q = 0; q < parts; ++q) {
+      const int n = part_run[q * E + e];
+      part_run[q * E + e] = total;
+      total += n;
+    }
   const int padded = e >= E ? 0 : cap > 0 ? cap : (total + block_m - 1) / block_m * block_m;
   // inclusive scan of `padded` across the block
   int v = padded;
@@ -425,15 +446,19 @@ __global__ void __launch_bounds__(1024) perm_scan_kernel(int32_t* __restrict__ c
     if (cap > 0 && total > cap) set_status(status, MOE_DEV_CAPACITY);
     counts[e] = cap > 0 && total > cap ? cap : total;
     offsets[e] = excl;
-    int run = excl;
-    for (int c = 0; c < nchunks; ++c) {
-      const long long idx = static_cast<long long>(c) * E + e;
+    first_row[e] = excl;
+  }
+  if (e == E - 1) offsets[E] = incl;
+  __syncthreads();
+  if (walker) {
+    int run = first_row[my_e] + part_run[tid];
+    for (int c = c0; c < c1; ++c) {
+      const long long idx = static_cast<long long>(c) * E + my_e;
       const int n = chunk_counts[idx];
       chunk_counts[idx] = run;
       run += n;
     }
   }
-  if (e == E - 1) offsets[E] = incl;
 }
 
 // 3) stable rank inside each chunk: one warp per chunk walks its pairs in order,
