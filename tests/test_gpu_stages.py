@@ -145,6 +145,19 @@ def test_permute_one_block_path_many_experts(E, K, T, cap):
     _check_perm(wl, ids, r)
 
 
+@pytest.mark.parametrize("E,K,T", [(1, 1, 5000), (3, 2, 4000), (96, 8, 9000), (1000, 4, 3000), (1024, 8, 4096)])
+def test_permute_chunked_scan(E, K, T):
+    """More than 2048 pairs: count per 256-pair chunk, scan, rank.  The scan spreads each
+    expert's chunks over 1024 // E threads: 1024 of them for one expert, 341 for three (more
+    threads than chunks), 10 for 96 (ranges of 29 chunks), one for 1000 and 1024 experts."""
+    wl = W.Workload("perm_chunked", T=T, H=128, I=128, E=E, K=K)
+    rng = np.random.default_rng(E * 7 + K)
+    ids = np.stack([rng.choice(E, K, replace=False) for _ in range(T)]).astype(np.int32)
+    r = _permute(wl, ids)
+    _check_perm(wl, ids, r)
+    assert B.moe_get_device_status(r["ws"]) == 0
+
+
 def test_permute_bucket_edge_sizes():
     # experts with 0, 1, BM-1, BM, BM+1, 2*BM+5 rows (K = 1 so counts are set directly)
     sizes = [0, 1, BM - 1, BM, BM + 1, 2 * BM + 5, 0, 3]
