@@ -75,9 +75,10 @@ typedef enum moe_status {
 #define MOE_DEV_BAD_EXPERT_ID 0x1   /* a topk id outside [0,E): the pair was skipped      */
 #define MOE_DEV_TIMEOUT 0x2         /* a GEMM pipeline wait exceeded its limit and exited */
 #define MOE_DEV_CAPACITY 0x4        /* masked layout: an expert had more than masked_cap    */
-#define MOE_DEV_RANGE 0x8           /* moe_layer_forward at prefill sizes keeps the routed    */
-                                    /* expert outputs in fp16; one exceeded |y| = 65504       */
                                     /* pairs; the pairs past it got no row (left out)       */
+#define MOE_DEV_RANGE 0x8           /* moe_layer_forward at prefill sizes keeps the routed  */
+                                    /* (and shared) expert outputs in fp16; one exceeded    */
+                                    /* |y| = 65504                                          */
 
 enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 };
 enum { MOE_DTYPE_BF16 = 0, MOE_DTYPE_FP8_E4M3 = 1, MOE_DTYPE_FP8_FP4 = 2 };
@@ -247,7 +248,9 @@ moe_status_t moe_combine(const moe_params_t* p, const void* y_perm, const int32_
 /* routing decision (NULL: kept in ws only).  ws_gate/ws_up/ws_down are the shared      */
 /* expert's weights (required iff I_shared > 0).  For bf16 layers with T*K >= 256*E and */
 /* H a multiple of 256, the routed experts' outputs pass to the combine in fp16 (2^-11  */
-/* relative rounding); an output beyond +-65504 sets MOE_DEV_RANGE in the status word.  */
+/* relative rounding), and so does the shared expert's output of a bf16 layer with      */
+/* T >= 256 and more than 16384 pairs; an output beyond +-65504 sets MOE_DEV_RANGE in   */
+/* the status word.                                                                     */
 /* ---------------------------------------------------------------------------------- */
 moe_status_t moe_layer_forward(const moe_params_t* p, const void* x, const float* x_scale,
                                const void* w_r, const float* bias, const void* w_gate,

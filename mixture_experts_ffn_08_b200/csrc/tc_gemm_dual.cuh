@@ -1,5 +1,6 @@
 // Grouped expert GEMMs with two M-tiles per work item: the gate/up projection with fused
-// SwiGLU (SWIGLU = true) and the down projection (fp32 out).
+// SwiGLU (SWIGLU = true) and the down projection (fp32 or fp16 out).  With no schedule
+// (offsets == nullptr) the A rows form one dense group, as for the shared expert.
 //
 // The same grouped GEMMs as tc_gemm_kernel<EPI_SWIGLU / EPI_F32> (routing primer "MoE 路由入门"
 // §5.2; the "MoE" chapter index's M-grouped contiguous layout), with one change in how a
@@ -40,7 +41,7 @@ struct DualParams {
   int K;                    // reduction length, multiple of 64
   int N;                    // output columns; weight rows per group (and matrix, for SwiGLU)
   int masked_cap;           // > 0: group g's rows sit at g * masked_cap in A and out
-  void* out;                // SwiGLU: h [rows, ldo] bf16; else y [rows, ldo] fp32
+  void* out;                // SwiGLU: h [rows, ldo] bf16; else y [rows, ldo] fp32 (fp16: out_f16)
   int64_t ldo;
   int32_t* status;
   int32_t* next_item;       // work counter, zero at launch
@@ -103,8 +104,8 @@ MOE_DEVINL DualItem dual_decode(int item, int NT, const DualParams& p, const int
 }
 
 // SWIGLU: tmG / tmU are the gate and up weights (boxes of 128 rows) and h = SiLU(g) * u is
-// stored in bf16; otherwise tmG is the one weight matrix (boxes of 256 rows) and the fp32
-// product is stored.
+// stored in bf16; otherwise tmG is the one weight matrix (boxes of 256 rows) and the
+// product is stored in fp32, or in fp16 with out_f16.
 template <bool SWIGLU>
 __global__ void __launch_bounds__(kDualThreads, 1)
     tc_gemm_dual_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmG,
