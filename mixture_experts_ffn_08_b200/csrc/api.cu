@@ -316,20 +316,23 @@ moe_status_t do_route(const moe_params_t* p, const void* x, const float* x_scale
 }
 
 // fill_pad: zero x_perm's pad rows (moe_permute's contract); the layer skips it (its GEMMs
-// never store a pad row).
+// never store a pad row).  x_atoms (FP8 layers, only with fill_pad false): the copy writes
+// x's scales straight into the GEMM's scale atoms instead of x_perm_scale.
 moe_status_t do_permute(const moe_params_t* p, const int32_t* ids, const void* x, const float* x_scale,
                         int32_t* counts, int32_t* offsets, int32_t* rop, int32_t* por, void* x_perm,
-                        float* x_perm_scale, void* ws, cudaStream_t st, bool fill_pad = true) {
+                        float* x_perm_scale, void* ws, cudaStream_t st, bool fill_pad = true,
+                        uint8_t* x_atoms = nullptr) {
   const Layout L = layout(p);
   return cuda_status(launch_permute(*p, block_m_of(p), ids, x, x_scale, counts, offsets, rop, por, x_perm, x_perm_scale,
-                                    at<int32_t>(ws, L.chunk_counts), at<int32_t>(ws, L.status), st, fill_pad));
+                                    at<int32_t>(ws, L.chunk_counts), at<int32_t>(ws, L.status), st, fill_pad,
+                                    x_atoms));
 }
 
 moe_status_t do_expert_ffn_fp8(const moe_params_t* p, const void* x_perm, const float* x_perm_scale,
                                const int32_t* offsets, const int32_t* counts, const void* w_gate,
                                const void* w_up, const void* w_down, const void* wgs,
                                const void* wus, const void* wds, void* y_perm, void* ws,
-                               cudaStream_t st) {
+                               cudaStream_t st, bool x_atoms_ready = false) {
   const Layout L = layout(p);
   int32_t* status = at<int32_t>(ws, L.status);
   // masked layout: the GEMMs walk a compact schedule and address expert e's rows at e*cap
@@ -358,8 +361,9 @@ moe_status_t do_expert_ffn_fp8(const moe_params_t* p, const void* x_perm, const 
     wu_atoms = at<uint8_t>(ws, L.wu_atoms);
     wd_atoms = at<uint8_t>(ws, L.wd_atoms);
   }
-  MOE_CUDA(launch_sf_rows_to_atoms(x_perm_scale, p->H / 128, offsets, p->E, L.max_rows,
-                                   at<uint8_t>(ws, L.x_atoms), st));
+  if (!x_atoms_ready)
+    MOE_CUDA(launch_sf_rows_to_atoms(x_perm_scale, p->H / 128, offsets, p->E, L.max_rows,
+                                     at<uint8_t>(ws, L.x_atoms), st));
   void* h = at<void>(ws, L.h);
   if (block_m_of(p) == kBlockM2) {
     MOE_CUDA(gemm_pair_gateup_swiglu_fp8(x_perm, at<uint8_t>(ws, L.x_atoms), L.max_rows, offsets, counts, p->E,
@@ -510,7 +514,8 @@ moe_status_t do_layer_after_fork(const moe_params_t* p, const void* x, const flo
   int32_t* rop = at<int32_t>(ws, L.row_of_pair);
   float* y_perm = at<float>(ws, L.y_perm);
   MOE_TRY(do_permute(p, ids, x, x_scale, counts, offsets, rop, at<int32_t>(ws, L.pair_of_row),
-                     at<void>(ws, L.x_perm), at<float>(ws, L.x_perm_scale), ws, st, /*fill_pad=*/false));
+                     at<void>(ws, L.x_perm), at<float>(ws, L.x_perm_scale), ws, st, /*fill_pad=*/false,
+                     is_fp8(p) ? at<uint8_t>(ws, L.x_atoms) : nullptr));
   if (p->fused_combine) {
     // acc starts as the shared expert's output (or zero); the routed down projection adds
     // w * y of every pair into it; one pass rounds it to bf16
@@ -535,7 +540,7 @@ moe_status_t do_layer_after_fork(const moe_params_t* p, const void* x, const flo
   }
   if (is_fp8(p))
     MOE_TRY(do_expert_ffn_fp8(p, at<void>(ws, L.x_perm), at<float>(ws, L.x_perm_scale), offsets, counts,
-                              w_gate, w_up, w_down, wgs, wus, wds, y_perm, ws, st));
+                              w_gate, w_up, w_down, wgs, wus, wds, y_perm, ws, st, /*x_atoms_ready=*/true));
   else
     MOE_TRY(do_expert_ffn(p, at<void>(ws, L.x_perm), offsets, counts, w_gate, w_up, w_down, y_perm, ws, st,
                           layer_y16(p, counts)));
@@ -884,8 +889,8 @@ int32_t moe_layer_launch_count(const moe_params_t* p) {
   if (validate(p) != MOE_OK) return -1;
   if (p->T == 0) return 0;
   int n = 2;                                 // router GEMM, top-k
-  if (is_fp8(p)) n += is_fp4(p) ? 2 : 5;     // dequantise x for the router; scale atoms of x
-                                             // (and of the three e4m3 weights)
+  if (is_fp8(p)) n += is_fp4(p) ? 1 : 4;     // dequantise x for the router (and the scale atoms
+                                             // of the three e4m3 weights; x's come with the copy)
   const long long P = static_cast<long long>(p->T) * p->K;
   n += P <= kSmallPairs ? 2 : 4;             // count, scan, rank (one kernel for few pairs), gather
   n += 2;                                    // gate/up, down

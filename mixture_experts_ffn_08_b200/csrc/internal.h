@@ -89,7 +89,7 @@ cudaError_t launch_permute(const moe_params_t& p, int block_m, const int32_t* id
                            const float* x_scale, int32_t* counts, int32_t* offsets,
                            int32_t* row_of_pair, int32_t* pair_of_row, void* x_perm,
                            float* x_perm_scale, int32_t* chunk_counts, int32_t* status,
-                           cudaStream_t st, bool fill_pad = true);
+                           cudaStream_t st, bool fill_pad = true, uint8_t* x_atoms = nullptr);
 
 // ---------------------------------------------------------------- combine (kernels.cu)
 // y_perm is fp32 for bf16 workloads and bf16 for FP8 workloads (p.dtype).

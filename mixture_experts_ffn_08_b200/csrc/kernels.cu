@@ -13,6 +13,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "tc_gemm_fp8.cuh"  // the scale-atom layout (sf_atom_offset)
 
 namespace moe {
 
@@ -637,7 +638,8 @@ constexpr int kScatterWarps = 8;
 template <bool FP8>
 __global__ void __launch_bounds__(32 * kScatterWarps) perm_scatter_kernel(
     const void* __restrict__ x, const float* __restrict__ x_scale, int T, int H, int K,
-    const int32_t* __restrict__ row_of_pair, void* __restrict__ x_perm, float* __restrict__ x_perm_scale) {
+    const int32_t* __restrict__ row_of_pair, void* __restrict__ x_perm, float* __restrict__ x_perm_scale,
+    uint8_t* __restrict__ x_atoms) {
   pdl_launch_dependents();
   pdl_wait();
   const int lane = threadIdx.x & 31;
@@ -672,11 +674,30 @@ __global__ void __launch_bounds__(32 * kScatterWarps) perm_scatter_kernel(
       }
     }
     if (FP8 && chunk == 0) {
+      const int nsc4 = (nsc + 3) / 4;
       for (int k = 0; k < K; ++k) {
         const int r = __shfl_sync(kFull, my_row, k);
         if (r < 0) continue;
-        for (int j = lane; j < nsc; j += 32)
-          x_perm_scale[static_cast<long long>(r) * nsc + j] = __ldg(x_scale + static_cast<long long>(t) * nsc + j);
+        if (x_atoms != nullptr) {
+          // the block-scaled GEMM's scale atoms directly: row r's word in atom (r / 128, q)
+          // holds the UE8M0 exponents of its scales 4q ... 4q + 3 (127 = 1.0 past the end)
+          for (int q = lane; q < nsc4; q += 32) {
+            uint32_t word = 0;
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+              const int j = 4 * q + b;
+              const uint32_t e =
+                  j < nsc ? (__float_as_uint(__ldg(x_scale + static_cast<long long>(t) * nsc + j)) >> 23) & 0xFFu
+                          : 127u;
+              word |= e << (8 * b);
+            }
+            *reinterpret_cast<uint32_t*>(x_atoms + (static_cast<long long>(r >> 7) * nsc4 + q) * 512 +
+                                         sf_atom_offset(r & 127)) = word;
+          }
+        } else {
+          for (int j = lane; j < nsc; j += 32)
+            x_perm_scale[static_cast<long long>(r) * nsc + j] = __ldg(x_scale + static_cast<long long>(t) * nsc + j);
+        }
       }
     }
   }
@@ -686,7 +707,7 @@ cudaError_t launch_permute(const moe_params_t& p, int block_m, const int32_t* id
                            const float* x_scale, int32_t* counts, int32_t* offsets,
                            int32_t* row_of_pair, int32_t* pair_of_row, void* x_perm,
                            float* x_perm_scale, int32_t* chunk_counts, int32_t* status,
-                           cudaStream_t st, bool fill_pad) {
+                           cudaStream_t st, bool fill_pad, uint8_t* x_atoms) {
   const int P = p.T * p.K;
   const int nchunks = (P + kPermChunk - 1) / kPermChunk;
   const int bm = block_m;
@@ -729,10 +750,10 @@ cudaError_t launch_permute(const moe_params_t& p, int block_m, const int32_t* id
     trace_before(MOE_K_PERM_GATHER, st);
     if (act_e4m3(p))
       err = launch_k(perm_scatter_kernel<true>, grid, 32 * kScatterWarps, 0, st, x, x_scale, p.T, p.H, p.K,
-                     row_of_pair, x_perm, x_perm_scale);
+                     row_of_pair, x_perm, x_perm_scale, x_atoms);
     else
       err = launch_k(perm_scatter_kernel<false>, grid, 32 * kScatterWarps, 0, st, x, x_scale, p.T, p.H, p.K,
-                     row_of_pair, x_perm, x_perm_scale);
+                     row_of_pair, x_perm, x_perm_scale, static_cast<uint8_t*>(nullptr));
     trace_after(MOE_K_PERM_GATHER, st);
     return err != cudaSuccess ? err : cudaGetLastError();
   }
