@@ -13,7 +13,9 @@ The headline workload is the DeepSeek-V3-shaped prefill layer (T=8192, H=7168, I
 256 routed experts, top-8, plus a shared expert), the largest of the five workloads.
 On one GPU the line also carries, under "configs", the same record for each of the
 other four workloads (tiny, Mixtral-shaped prefill, DeepSeek-V3-shaped decode, skewed
-FP8), each timed over enough steps to fill a few hundred ms.
+FP8) and for the decode layer with e2m1 expert weights, each timed over enough steps to
+fill a few hundred ms, and under "micro" the GroupedTopK kernel alone (83 tokens, 256
+experts) in us per call.
 
 Each record has `value` (tokens/s), the grouped-GEMM TFLOP/s and each GEMM kernel's
 fraction of the measured bf16 burst peak, an end-to-end number through
@@ -638,6 +640,8 @@ def measure(wl, steps, warmup, world=1, rank=0, local=0, cpu=True, adapt_steps=F
 
 
 SUB_CONFIGS = ("tiny", "mixtral_prefill", "dsv3_decode", "skewed_fp8", "dsv3_prefill")
+# beyond the five workloads: the DeepSeek-V3 decode layer with e2m1 expert weights
+EXTRA_CONFIGS = ("dsv3_decode_fp4",)
 
 
 def run_ours(args):
@@ -663,11 +667,14 @@ def run_ours(args):
     configs = None
     if world == 1 and not args.no_configs:
         configs = {}
-        for name in SUB_CONFIGS:
+        for name in SUB_CONFIGS + EXTRA_CONFIGS:
             if name == wl.name:
                 continue
-            configs[name] = measure(W.ALL[name], args.steps, args.warmup, cpu=not args.no_cpu_baseline,
-                                    adapt_steps=True)
+            # (the e2m1 record carries no CPU baseline: its oracle would first widen ~50 GB of
+            # expert weights to fp64, a minute of the run for a figure the other records give)
+            configs[name] = measure((W.ALL | W.FP4)[name], args.steps, args.warmup,
+                                    cpu=not args.no_cpu_baseline and name not in EXTRA_CONFIGS, adapt_steps=True)
+        micro = {"grouped_topk": micro_grouped_topk_record(1000, args.warmup)}
     if rank != 0:
         return
     line = {
@@ -683,6 +690,7 @@ def run_ours(args):
                                                            "steps", "dtype")})
     if configs is not None:
         line["configs"] = configs
+        line["micro"] = micro
     print(json.dumps(line), flush=True)
 
 
@@ -726,7 +734,7 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
-def run_micro_grouped_topk(args):
+def micro_grouped_topk_record(steps, warmup):
     """GroupedTopK alone at the routing primer's KernelSwift shape (§十): 83 tokens, 256
     experts in 8 groups of 32, keep 4 groups, top-8, softmax, renormalised."""
     wl = W.Workload("grouped_topk_kernelswift", T=83, H=7168, I=128, E=256, K=8, n_group=8,
@@ -736,7 +744,7 @@ def run_micro_grouped_topk(args):
     logits = torch.randn((wl.T, wl.E), generator=g, device="cuda")
     ids = torch.empty((wl.T, wl.K), dtype=torch.int32, device="cuda")
     w = torch.empty((wl.T, wl.K), dtype=torch.float32, device="cuda")
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         B.check(B.moe_grouped_topk(p, logits, None, ids, w))
     # the launches go into a CUDA graph so the host's per-call cost does not set the pace
     per_graph = 50
@@ -749,7 +757,7 @@ def run_micro_grouped_topk(args):
                 B.check(B.moe_grouped_topk(p, logits, None, ids, w))
     torch.cuda.current_stream().wait_stream(side)
     graph.replay()
-    reps = max(args.steps // per_graph, 4)
+    reps = max(steps // per_graph, 4)
     n = reps * per_graph
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
@@ -760,10 +768,14 @@ def run_micro_grouped_topk(args):
     torch.cuda.synchronize()
     us = s.elapsed_time(e) * 1e3 / n
     del graph
-    print(json.dumps({"metric": "GroupedTopK latency (83 tokens, 256 experts, 8x32 groups, keep 4, top-8)",
-                      "value": us, "unit": "us/call", "higher_is_better": False, "steps": n,
-                      "warmup": args.warmup, "n_gpus": 1, "dtype": "f32",
-                      "config": {"workload": wl.name}, "gpu_launches": n}), flush=True)
+    return {"metric": "GroupedTopK latency (83 tokens, 256 experts, 8x32 groups, keep 4, top-8)",
+            "value": us, "unit": "us/call", "higher_is_better": False, "steps": n,
+            "warmup": warmup, "n_gpus": 1, "dtype": "f32",
+            "config": {"workload": wl.name}, "gpu_launches": n}
+
+
+def run_micro_grouped_topk(args):
+    print(json.dumps(micro_grouped_topk_record(args.steps, args.warmup)), flush=True)
 
 
 def main():
