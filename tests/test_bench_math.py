@@ -133,3 +133,35 @@ def test_host_weights_load_time_is_kept_apart_and_cache_is_bounded():
         g, u, dn = hw(e)
         assert g.dtype.name == "float64" and (g == d["w_gate"][e].double().numpy()).all()
     assert len(hw.cache) <= 2 and hw.load_s > 0
+
+
+def test_default_line_carries_every_workload_and_the_micro_record(monkeypatch, capsys):
+    """run_ours on one GPU: the headline record, one record per other workload (the e2m1
+    decode layer without a CPU baseline) and the GroupedTopK micro record, in one line.
+    measure() and the micro benchmark are stubbed, so this runs without a GPU."""
+    import argparse
+    import json
+    calls = []
+
+    def fake_measure(wl, steps, warmup, world=1, rank=0, local=0, cpu=True, adapt_steps=False):
+        calls.append((wl.name, cpu, adapt_steps))
+        return {"workload": wl.name, "value": 1.0, "unit": "tokens/s", "ms_per_step": 1.0, "steps": steps,
+                "dtype": "bf16", "roofline": {}, "cpu_baseline": {"value": 1.0} if cpu else None}
+
+    monkeypatch.setattr(bench, "measure", fake_measure)
+    monkeypatch.setattr(bench, "micro_grouped_topk_record", lambda steps, warmup: {"value": 6.3, "unit": "us/call"})
+    monkeypatch.setattr(bench.torch.cuda, "set_device", lambda d: None)
+    for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    args = argparse.Namespace(workload="dsv3_prefill", steps=5, warmup=3, no_cpu_baseline=False, no_configs=False,
+                              fused_combine=False, block_m=0, masked_cap=0)
+    bench.run_ours(args)
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["config"]["workload"] == "dsv3_prefill"
+    assert set(line["configs"]) == {"tiny", "mixtral_prefill", "dsv3_decode", "skewed_fp8", "dsv3_decode_fp4"}
+    assert line["configs"]["dsv3_decode_fp4"]["cpu_baseline"] is None
+    assert all(line["configs"][n]["cpu_baseline"] is not None for n in ("tiny", "mixtral_prefill", "dsv3_decode",
+                                                                       "skewed_fp8"))
+    assert line["micro"]["grouped_topk"]["unit"] == "us/call"
+    assert calls[0] == ("dsv3_prefill", True, False)
+    assert all(adapt for _, _, adapt in calls[1:])
