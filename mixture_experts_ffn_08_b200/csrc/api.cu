@@ -549,12 +549,11 @@ moe_status_t do_layer_after_fork(const moe_params_t* p, const void* x, const flo
     MOE_CUDA(cudaStreamWaitEvent(st, side->join, 0));
   } else if (p->I_shared > 0 && shared_two_tile(p)) {
     // the dense shared expert at prefill sizes through the two-tile kernels, y_sh in fp16
-    const Layout Ls = layout(p);
-    int32_t* status = at<int32_t>(ws, Ls.status);
-    int32_t* ctr = at<int32_t>(ws, Ls.counter);
+    int32_t* status = at<int32_t>(ws, L.status);
+    int32_t* ctr = at<int32_t>(ws, L.counter);
     MOE_CUDA(gemm_gateup_swiglu_dual(x, p->T, nullptr, nullptr, 1, wsg, wsu, p->I_shared, p->H,
-                                     at<void>(ws, Ls.h_sh), ctr, status, st, 0, MOE_K_SHARED_GATEUP));
-    MOE_CUDA(gemm_down_dual(at<void>(ws, Ls.h_sh), p->T, nullptr, nullptr, 1, wsd, p->H, p->I_shared, y_sh,
+                                     at<void>(ws, L.h_sh), ctr, status, st, 0, MOE_K_SHARED_GATEUP));
+    MOE_CUDA(gemm_down_dual(at<void>(ws, L.h_sh), p->T, nullptr, nullptr, 1, wsd, p->H, p->I_shared, y_sh,
                             ctr + 1, status, st, 0, /*y_f16=*/true, MOE_K_SHARED_DOWN));
     ysh16 = true;
   } else if (p->I_shared > 0) {

@@ -848,8 +848,8 @@ MOE_DEVINL void load8(const __half* row, int v, float (&f)[8]) {
 }
 
 // out[t] = sum_k w[t,k] y_perm[row_of_pair[t*K+k]] (+ y_sh[t]); YT, ST = float, bf16 or fp16.
-// One block per token; 32 registers, so 16 blocks share an SM and keep enough loads in
-// flight for large batches.
+// One block per token, with few registers (32 for the layer's fp16 and bf16 outputs), so up
+// to 16 blocks share an SM and keep enough loads in flight for large batches.
 template <class YT, class ST>
 __global__ void __launch_bounds__(128) combine_kernel(
     const YT* __restrict__ y_perm, const int32_t* __restrict__ row_of_pair,
