@@ -567,6 +567,13 @@ def measure(wl, steps, warmup, world=1, rank=0, local=0, cpu=True, adapt_steps=F
              "shared_gateup": 4.0 * wl.T * wl.H * wl.I_shared, "shared_down": 2.0 * wl.T * wl.H * wl.I_shared}
     gemm_flops = sum(flops.values())
     bytes_gateup = (active * 2 * wl.I * wl.H * wbytes + P * wl.H * abytes + P * wl.I * abytes)
+    # at prefill sizes the shared expert is one more group of the routed two-tile launches
+    # (no launches of its own in the trace): its work then counts toward theirs
+    shared_in_routed = wl.I_shared > 0 and "shared_gateup" not in kernel_ms
+    if shared_in_routed:
+        flops["gateup_swiglu"] += flops.pop("shared_gateup")
+        flops["down"] += flops.pop("shared_down")
+        bytes_gateup += 2 * wl.I_shared * wl.H * 2 + wl.T * wl.H * 2 + wl.T * wl.I_shared * 2
     layer_bytes = (active * 3 * wl.I * wl.H * wbytes + 3 * wl.I_shared * wl.H * 2 + wl.E * wl.H * 2
                    + wl.T * wl.H * (abytes + 2))
     dt_name = "e4m3 x e2m1" if w4 else ("e4m3" if fp8 else "bf16")
@@ -622,6 +629,7 @@ def measure(wl, steps, warmup, world=1, rank=0, local=0, cpu=True, adapt_steps=F
         "layer_hbm_frac": layer_bytes / (ms_step / 1e3) / 1e9 / hbm_peak,
         "layer_algorithmic_bytes": layer_bytes,
         "active_experts": active,
+        "shared_expert_in_routed_launches": shared_in_routed,
         "routed_gemm_rows": {"real": P, "computed": mma_rows,
                              "pad_frac": (mma_rows - P) / mma_rows if mma_rows else 0.0},
         "e2e": {"value": wl.T * world / (e2e_ms / 1e3), "unit": "tokens/s",

@@ -391,13 +391,15 @@ bool two_tile_items(const moe_params_t* p, const int32_t* counts) {
 }
 
 moe_status_t do_gateup(const moe_params_t* p, const void* x_perm, const int32_t* sched, const int32_t* counts,
-                       const void* w_gate, const void* w_up, void* ws, cudaStream_t st) {
+                       const void* w_gate, const void* w_up, void* ws, cudaStream_t st,
+                       const DualExtra* extra = nullptr) {
   const Layout L = layout(p);
   int32_t* status = at<int32_t>(ws, L.status);
   void* h = at<void>(ws, L.h);
   if (two_tile_items(p, counts))
     return cuda_status(gemm_gateup_swiglu_dual(x_perm, L.max_rows, sched, counts, p->E, w_gate, w_up, p->I, p->H,
-                                               h, at<int32_t>(ws, L.counter), status, st, p->masked_cap));
+                                               h, at<int32_t>(ws, L.counter), status, st, p->masked_cap,
+                                               MOE_K_GATEUP, extra));
   return cuda_status(gemm_gateup_swiglu(x_perm, L.max_rows, sched, counts, p->E, 0, w_gate, w_up, p->I, p->H, h,
                                         status, MOE_K_GATEUP, st, p->masked_cap));
 }
@@ -418,9 +420,22 @@ bool shared_two_tile(const moe_params_t* p) {
   return !is_fp8(p) && p->T >= 256 && p->H % 256 == 0 && p->I_shared % 128 == 0;
 }
 
+// ... and when the routed experts run through the two-tile kernels too, it is one more group
+// of their launches (one launch and one tail per projection instead of two).  Decided from
+// the parameters alone (the side stream takes the shared expert for few pairs).
+bool shared_merged(const moe_params_t* p) {
+  const long long P = static_cast<long long>(p->T) * p->K;
+  const bool side = P <= kOverlapMaxPairs && overlap_shared_enabled();
+  return p->I_shared > 0 && !side && !p->fused_combine && shared_two_tile(p) && block_m_of(p) != kBlockM2 &&
+         p->E <= 1024 && P >= 256LL * p->E;
+}
+
+// gu_extra / dn_extra: the shared expert as an extra group of the two-tile launches (only
+// passed when those run, see shared_merged).
 moe_status_t do_expert_ffn(const moe_params_t* p, const void* x_perm, const int32_t* offsets,
                            const int32_t* counts, const void* w_gate, const void* w_up,
-                           const void* w_down, float* y_perm, void* ws, cudaStream_t st, bool y16 = false) {
+                           const void* w_down, float* y_perm, void* ws, cudaStream_t st, bool y16 = false,
+                           const DualExtra* gu_extra = nullptr, const DualExtra* dn_extra = nullptr) {
   const Layout L = layout(p);
   int32_t* status = at<int32_t>(ws, L.status);
   void* h = at<void>(ws, L.h);
@@ -436,13 +451,13 @@ moe_status_t do_expert_ffn(const moe_params_t* p, const void* x_perm, const int3
     MOE_CUDA(launch_masked_schedule(counts, p->E, at<int32_t>(ws, L.sched), st));
     sched = at<int32_t>(ws, L.sched);
   }
-  MOE_TRY(do_gateup(p, x_perm, sched, counts, w_gate, w_up, ws, st));
+  MOE_TRY(do_gateup(p, x_perm, sched, counts, w_gate, w_up, ws, st, gu_extra));
   // the down projection takes two M-tiles per item under the same rule as gate/up
   // (measured: Mixtral prefill down 0.72 against 0.82 ms, DeepSeek-V3 prefill step 7.9
   // against 8.1 ms); its weight tiles are 256 rows, so H must be a multiple of 256
   if (two_tile_items(p, counts) && p->H % 256 == 0)
     MOE_CUDA(gemm_down_dual(h, L.max_rows, sched, counts, p->E, w_down, p->H, p->I, y_perm,
-                            at<int32_t>(ws, L.counter) + 1, status, st, cap, y16));
+                            at<int32_t>(ws, L.counter) + 1, status, st, cap, y16, MOE_K_DOWN, dn_extra));
   else
     MOE_CUDA(gemm_down(h, L.max_rows, sched, counts, p->E, 0, w_down, p->H, p->I, y_perm, status,
                        MOE_K_DOWN, st, cap));
@@ -538,15 +553,25 @@ moe_status_t do_layer_after_fork(const moe_params_t* p, const void* x, const flo
                                at<int32_t>(ws, L.pair_of_row), w, p->K, acc, status, st, cap));
     return cuda_status(launch_f32_to_bf16(acc, static_cast<long long>(p->T) * p->H, out, st));
   }
-  if (is_fp8(p))
+  const bool merged = side == nullptr && shared_merged(p);
+  if (is_fp8(p)) {
     MOE_TRY(do_expert_ffn_fp8(p, at<void>(ws, L.x_perm), at<float>(ws, L.x_perm_scale), offsets, counts,
                               w_gate, w_up, w_down, wgs, wus, wds, y_perm, ws, st, /*x_atoms_ready=*/true));
-  else
+  } else if (merged) {
+    // the shared expert as the extra group of the routed two-tile launches, y_sh in fp16
+    const DualExtra gu{x, p->T, wsg, wsu, p->I_shared, p->H, at<void>(ws, L.h_sh)};
+    const DualExtra dn{at<void>(ws, L.h_sh), p->T, wsd, nullptr, p->H, p->I_shared, y_sh};
+    MOE_TRY(do_expert_ffn(p, at<void>(ws, L.x_perm), offsets, counts, w_gate, w_up, w_down, y_perm, ws, st,
+                          layer_y16(p, counts), &gu, &dn));
+  } else {
     MOE_TRY(do_expert_ffn(p, at<void>(ws, L.x_perm), offsets, counts, w_gate, w_up, w_down, y_perm, ws, st,
                           layer_y16(p, counts)));
-  bool ysh16 = false;
+  }
+  bool ysh16 = merged;
   if (side != nullptr) {
     MOE_CUDA(cudaStreamWaitEvent(st, side->join, 0));
+  } else if (merged) {
+    // done inside the routed launches
   } else if (p->I_shared > 0 && shared_two_tile(p)) {
     // the dense shared expert at prefill sizes through the two-tile kernels, y_sh in fp16
     int32_t* status = at<int32_t>(ws, L.status);
@@ -893,7 +918,7 @@ int32_t moe_layer_launch_count(const moe_params_t* p) {
   const long long P = static_cast<long long>(p->T) * p->K;
   n += P <= kSmallPairs ? 2 : 4;             // count, scan, rank (one kernel for few pairs), gather
   n += 2;                                    // gate/up, down
-  if (p->I_shared > 0) n += 2;               // shared gate/up, down
+  if (p->I_shared > 0 && !shared_merged(p)) n += 2;  // shared gate/up, down (unless in the routed ones)
   n += 1;                                    // combine
   if (p->masked_cap > 0) n += 1;             // compact GEMM schedule of the masked layout
   return n;

@@ -132,14 +132,34 @@ cudaError_t gemm_gateup_swiglu(const void* A, int64_t a_rows, const int32_t* off
 
 cudaError_t gemm_gateup_swiglu_dual(const void* A, int64_t a_rows, const int32_t* offsets, const int32_t* counts,
                                     int G, const void* w_gate, const void* w_up, int N, int K, void* h,
-                                    int32_t* counter, int32_t* status, cudaStream_t st, int masked_cap, int kid) {
+                                    int32_t* counter, int32_t* status, cudaStream_t st, int masked_cap, int kid,
+                                    const DualExtra* extra) {
   if (G > kDualMaxGroups || N % 128 != 0 || K % 64 != 0) return cudaErrorInvalidValue;
-  CUtensorMap ta, tg, tu;
+  const bool has_x = extra != nullptr && extra->rows > 0;
+  if (has_x && (extra->N % 128 != 0 || extra->K % 64 != 0)) return cudaErrorInvalidValue;
+  CUtensorMap ta, tg, tu, ta2, tg2, tu2;
   if (!make_tmap_bf16(&ta, A, a_rows, K, 128) ||
       !make_tmap_bf16(&tg, w_gate, static_cast<uint64_t>(G) * N, K, 128) ||
       !make_tmap_bf16(&tu, w_up, static_cast<uint64_t>(G) * N, K, 128))
     return cudaErrorInvalidValue;
+  if (has_x) {
+    if (!make_tmap_bf16(&ta2, extra->a, extra->rows, extra->K, 128) ||
+        !make_tmap_bf16(&tg2, extra->w0, extra->N, extra->K, 128) ||
+        !make_tmap_bf16(&tu2, extra->w1, extra->N, extra->K, 128))
+      return cudaErrorInvalidValue;
+  } else {
+    ta2 = ta;  // never read without an extra group
+    tg2 = tg;
+    tu2 = tu;
+  }
   DualParams dp{};
+  if (has_x) {
+    dp.x_rows = extra->rows;
+    dp.x_N = extra->N;
+    dp.x_K = extra->K;
+    dp.x_out = extra->out;
+    dp.x_ldo = extra->N;
+  }
   dp.offsets = offsets;
   dp.counts = counts;
   dp.dense_rows = static_cast<int>(a_rows);  // used when offsets is null (one dense group)
@@ -155,23 +175,40 @@ cudaError_t gemm_gateup_swiglu_dual(const void* A, int64_t a_rows, const int32_t
   if (err != cudaSuccess) return err;
   err = cudaFuncSetAttribute(tc_gemm_dual_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDualSmemBytes);
   if (err != cudaSuccess) return err;
-  const long long max_items = ceil_div(a_rows, 128) * (N / 128);
+  const long long max_items = ceil_div(a_rows, 128) * (N / 128) + (has_x ? ceil_div(extra->rows, 128) * (extra->N / 128) : 0);
   const long long sms = num_sms();
   const int grid = static_cast<int>(max_items < sms ? (max_items > 0 ? max_items : 1) : sms);
   trace_before(kid, st);
-  err = launch_k(tc_gemm_dual_kernel<true>, grid, kDualThreads, kDualSmemBytes, st, ta, tg, tu, dp);
+  err = launch_k(tc_gemm_dual_kernel<true>, grid, kDualThreads, kDualSmemBytes, st, ta, tg, tu, ta2, tg2, tu2, dp);
   trace_after(kid, st);
   return err != cudaSuccess ? err : cudaGetLastError();
 }
 
 cudaError_t gemm_down_dual(const void* A, int64_t a_rows, const int32_t* offsets, const int32_t* counts, int G,
                            const void* w, int N, int K, void* y, int32_t* counter, int32_t* status, cudaStream_t st,
-                           int masked_cap, bool y_f16, int kid) {
+                           int masked_cap, bool y_f16, int kid, const DualExtra* extra) {
   if (G > kDualMaxGroups || N % 256 != 0 || K % 64 != 0) return cudaErrorInvalidValue;
-  CUtensorMap ta, tb;
+  const bool has_x = extra != nullptr && extra->rows > 0;
+  if (has_x && (extra->N % 256 != 0 || extra->K % 64 != 0)) return cudaErrorInvalidValue;
+  CUtensorMap ta, tb, ta2, tb2;
   if (!make_tmap_bf16(&ta, A, a_rows, K, 128) || !make_tmap_bf16(&tb, w, static_cast<uint64_t>(G) * N, K, 256))
     return cudaErrorInvalidValue;
+  if (has_x) {
+    if (!make_tmap_bf16(&ta2, extra->a, extra->rows, extra->K, 128) ||
+        !make_tmap_bf16(&tb2, extra->w0, extra->N, extra->K, 256))
+      return cudaErrorInvalidValue;
+  } else {
+    ta2 = ta;  // never read without an extra group
+    tb2 = tb;
+  }
   DualParams dp{};
+  if (has_x) {
+    dp.x_rows = extra->rows;
+    dp.x_N = extra->N;
+    dp.x_K = extra->K;
+    dp.x_out = extra->out;
+    dp.x_ldo = extra->N;
+  }
   dp.offsets = offsets;
   dp.counts = counts;
   dp.dense_rows = static_cast<int>(a_rows);  // used when offsets is null (one dense group)
@@ -188,11 +225,11 @@ cudaError_t gemm_down_dual(const void* A, int64_t a_rows, const int32_t* offsets
   if (err != cudaSuccess) return err;
   err = cudaFuncSetAttribute(tc_gemm_dual_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kDualSmemBytes);
   if (err != cudaSuccess) return err;
-  const long long max_items = ceil_div(a_rows, 128) * (N / 256);
+  const long long max_items = ceil_div(a_rows, 128) * (N / 256) + (has_x ? ceil_div(extra->rows, 128) * (extra->N / 256) : 0);
   const long long sms = num_sms();
   const int grid = static_cast<int>(max_items < sms ? (max_items > 0 ? max_items : 1) : sms);
   trace_before(kid, st);
-  err = launch_k(tc_gemm_dual_kernel<false>, grid, kDualThreads, kDualSmemBytes, st, ta, tb, tb, dp);
+  err = launch_k(tc_gemm_dual_kernel<false>, grid, kDualThreads, kDualSmemBytes, st, ta, tb, tb, ta2, tb2, tb2, dp);
   trace_after(kid, st);
   return err != cudaSuccess ? err : cudaGetLastError();
 }

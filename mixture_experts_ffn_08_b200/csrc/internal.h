@@ -112,14 +112,27 @@ cudaError_t gemm_gateup_swiglu(const void* A, int64_t a_rows, const int32_t* off
 // The same gate/up projection with two M-tiles of an expert per work item (grouped, with
 // counts, N multiple of 128); counter is a device int the call zeroes before the launch.
 // offsets == nullptr: one dense group of a_rows rows (counts unused).
+// An extra dense group for the two-tile launches (the shared expert): A [rows, K] bf16,
+// weights [N, K] bf16 (w1: the up projection's, for gate/up), output [rows, N] stored like
+// the launch's own (h bf16; y fp16 or fp32 as the launch's y_f16 says).
+struct DualExtra {
+  const void* a;
+  int rows;
+  const void* w0;
+  const void* w1;
+  int N;
+  int K;
+  void* out;
+};
 cudaError_t gemm_gateup_swiglu_dual(const void* A, int64_t a_rows, const int32_t* offsets, const int32_t* counts,
                                     int G, const void* w_gate, const void* w_up, int N, int K, void* h,
                                     int32_t* counter, int32_t* status, cudaStream_t st, int masked_cap = 0,
-                                    int kid = MOE_K_GATEUP);
+                                    int kid = MOE_K_GATEUP, const DualExtra* extra = nullptr);
 // The down projection with two M-tiles per work item (N multiple of 256); counter as above.
 cudaError_t gemm_down_dual(const void* A, int64_t a_rows, const int32_t* offsets, const int32_t* counts, int G,
                            const void* w, int N, int K, void* y, int32_t* counter, int32_t* status, cudaStream_t st,
-                           int masked_cap = 0, bool y_f16 = false, int kid = MOE_K_DOWN);
+                           int masked_cap = 0, bool y_f16 = false, int kid = MOE_K_DOWN,
+                           const DualExtra* extra = nullptr);
 // y [rows, N] fp32 = A W^T, grouped by offsets (or dense when null); with counts, pad
 // rows of each group are not stored.
 cudaError_t gemm_down(const void* A, int64_t a_rows, const int32_t* offsets,

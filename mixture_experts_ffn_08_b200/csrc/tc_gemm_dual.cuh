@@ -1,6 +1,9 @@
 // Grouped expert GEMMs with two M-tiles per work item: the gate/up projection with fused
 // SwiGLU (SWIGLU = true) and the down projection (fp32 or fp16 out).  With no schedule
-// (offsets == nullptr) the A rows form one dense group, as for the shared expert.
+// (offsets == nullptr) the A rows form one dense group, as for the shared expert.  With
+// x_rows > 0 a dense extra group follows the G groups in the same launch, with A, weights
+// and output of its own (tmA2 / tmG2 / tmU2, x_out): the shared expert of a layer whose
+// routed experts also take two M-tiles per item, so the two share one launch and one tail.
 //
 // The same grouped GEMMs as tc_gemm_kernel<EPI_SWIGLU / EPI_F32> (routing primer "MoE 路由入门"
 // §5.2; the "MoE" chapter index's M-grouped contiguous layout), with one change in how a
@@ -46,6 +49,11 @@ struct DualParams {
   int32_t* status;
   int32_t* next_item;       // work counter, zero at launch
   int out_f16;              // plain projection: store y as fp16 (|y| > 65504 sets MOE_DEV_RANGE)
+  // the extra dense group (0 rows: none): its rows, output columns, reduction length
+  // (multiple of 64) and output, stored like the others (out_f16 applies to it as well)
+  int x_rows, x_N, x_K;
+  void* x_out;
+  int64_t x_ldo;
 };
 
 constexpr int kDualMaxGroups = 1024;
@@ -57,7 +65,7 @@ constexpr int kDualStageBytes = 2 * kDualABytes + kDualBBytes;  // 64 KB
 constexpr int kDualSmemBytes = kDualStages * kDualStageBytes + 1024;
 constexpr int kDualRing = 4;                                   // items between producer and consumers
 constexpr int kDualThreads = 192;
-static_assert(kDualSmemBytes + (kDualMaxGroups + 1) * 4 + 1024 <= 227 * 1024, "shared memory");
+static_assert(kDualSmemBytes + (kDualMaxGroups + 2) * 4 + 1024 <= 227 * 1024, "shared memory");
 
 struct DualItem {
   int group;
@@ -80,8 +88,22 @@ MOE_DEVINL int group_count(const DualParams& p, int g) {
   return p.offsets != nullptr ? __ldg(p.counts + g) : p.dense_rows;
 }
 
-MOE_DEVINL DualItem dual_decode(int item, int NT, const DualParams& p, const int* pref) {
+MOE_DEVINL DualItem dual_decode(int item, int NT, int NT2, const DualParams& p, const int* pref) {
   // (NT * 256 is the group's weight rows in both forms: SwiGLU tiles hold 256 rows too)
+  if (item >= pref[p.G]) {  // the extra dense group (group index G)
+    const int tiles = (p.x_rows + 127) >> 7;
+    const int pairs = (tiles + 1) >> 1;
+    const int local = item - pref[p.G];
+    const bool pairs_outer = tiles * 128 > NT2 * 256;
+    const int j = pairs_outer ? local / NT2 : local % pairs;
+    DualItem d;
+    d.group = p.G;
+    d.n_tile = pairs_outer ? local % NT2 : local / pairs;
+    d.tile0 = 2 * j;
+    d.ntiles = (2 * j + 1 < tiles) ? 2 : 1;
+    d.mt0 = 0;
+    return d;
+  }
   int lo = 0, hi = p.G - 1;  // group with pref[g] <= item < pref[g+1]
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -109,7 +131,9 @@ MOE_DEVINL DualItem dual_decode(int item, int NT, const DualParams& p, const int
 template <bool SWIGLU>
 __global__ void __launch_bounds__(kDualThreads, 1)
     tc_gemm_dual_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmG,
-                        const __grid_constant__ CUtensorMap tmU, const DualParams p) {
+                        const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmA2,
+                        const __grid_constant__ CUtensorMap tmG2, const __grid_constant__ CUtensorMap tmU2,
+                        const DualParams p) {
   constexpr int OUT_COLS = SWIGLU ? 128 : 256;
   constexpr int BK = kDualBK, STAGES = kDualStages, R = kDualRing;
   constexpr uint32_t IDESC = idesc_bf16_f32(128, 256);
@@ -120,7 +144,7 @@ __global__ void __launch_bounds__(kDualThreads, 1)
   __shared__ uint64_t tfull_bar[2], tempty_bar[2], drain_bar;
   __shared__ uint64_t item_full[R], item_empty[R];
   __shared__ int item_ring[R];
-  __shared__ int pref[kDualMaxGroups + 1];
+  __shared__ int pref[kDualMaxGroups + 2];
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
 
@@ -128,7 +152,7 @@ __global__ void __launch_bounds__(kDualThreads, 1)
   const uint32_t pad = (1024u - (smem_u32(dsmem) & 1023u)) & 1023u;
   uint8_t* smem = dsmem + pad;
   const int NT = (p.N + OUT_COLS - 1) / OUT_COLS;
-  const int KB = p.K / BK;
+  const int NT2 = (p.x_N + OUT_COLS - 1) / OUT_COLS;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -151,6 +175,11 @@ __global__ void __launch_bounds__(kDualThreads, 1)
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmG);
     if (SWIGLU) prefetch_tmap(&tmU);
+    if (p.x_rows > 0) {
+      prefetch_tmap(&tmA2);
+      prefetch_tmap(&tmG2);
+      if (SWIGLU) prefetch_tmap(&tmU2);
+    }
   }
   if (warp == 1) {
     tmem_alloc(&tmem_base_sh, 512);
@@ -184,10 +213,14 @@ __global__ void __launch_bounds__(kDualThreads, 1)
       const int tiles = (group_row(p, g + 1) - group_row(p, g)) >> 7;
       acc += NT * ((tiles + 1) >> 1);
     }
-    if (lane == 31) pref[p.G] = incl;
+    if (lane == 31) {
+      pref[p.G] = incl;
+      const int x_tiles = (p.x_rows + 127) >> 7;
+      pref[p.G + 1] = incl + (p.x_rows > 0 ? NT2 * ((x_tiles + 1) >> 1) : 0);
+    }
   }
   __syncthreads();
-  const int total = pref[p.G];
+  const int total = pref[p.G + 1];
 
   if (warp == 0) {
     // ---------------------------------------------------------------- scheduler + TMA
@@ -204,21 +237,26 @@ __global__ void __launch_bounds__(kDualThreads, 1)
         item_ring[rs] = it;
         mbar_arrive(&item_full[rs]);
         if (it >= total) break;
-        const DualItem d = dual_decode(it, NT, p, pref);
-        const int b_row = d.group * p.N + d.n_tile * OUT_COLS;
+        const DualItem d = dual_decode(it, NT, NT2, p, pref);
+        const bool ex = d.group == p.G;  // the extra dense group
+        const CUtensorMap* mA = ex ? &tmA2 : &tmA;
+        const CUtensorMap* mG = ex ? &tmG2 : &tmG;
+        const CUtensorMap* mU = ex ? &tmU2 : &tmU;
+        const int b_row = (ex ? 0 : d.group * p.N) + d.n_tile * OUT_COLS;
         // (scalars, not arrays: an array indexed at run time lives in local memory)
         const int local0 = (d.tile0 - d.mt0) * 128;
-        const int a_row0 = p.masked_cap > 0 ? d.group * p.masked_cap + local0 : d.tile0 * 128;
+        const int a_row0 = (p.masked_cap > 0 && !ex) ? d.group * p.masked_cap + local0 : d.tile0 * 128;
         const int a_row1 = a_row0 + 128;
+        const int KB = (ex ? p.x_K : p.K) / BK;
         const uint32_t tx = static_cast<uint32_t>(d.ntiles * kDualABytes + kDualBBytes);
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, &abort_flag)) { ok = false; break; }
           uint8_t* st = smem + s * kDualStageBytes;
           mbar_arrive_expect_tx(&full_bar[s], tx);
-          tma_load_2d(st, &tmA, kb * BK, a_row0, &full_bar[s]);
-          if (d.ntiles == 2) tma_load_2d(st + kDualABytes, &tmA, kb * BK, a_row1, &full_bar[s]);
-          tma_load_2d(st + 2 * kDualABytes, &tmG, kb * BK, b_row, &full_bar[s]);
-          if (SWIGLU) tma_load_2d(st + 2 * kDualABytes + kDualBBytes / 2, &tmU, kb * BK, b_row, &full_bar[s]);
+          tma_load_2d(st, mA, kb * BK, a_row0, &full_bar[s]);
+          if (d.ntiles == 2) tma_load_2d(st + kDualABytes, mA, kb * BK, a_row1, &full_bar[s]);
+          tma_load_2d(st + 2 * kDualABytes, mG, kb * BK, b_row, &full_bar[s]);
+          if (SWIGLU) tma_load_2d(st + 2 * kDualABytes + kDualBBytes / 2, mU, kb * BK, b_row, &full_bar[s]);
           ++issued;
           if (++s == STAGES) { s = 0; ph ^= 1u; }
         }
@@ -245,10 +283,12 @@ __global__ void __launch_bounds__(kDualThreads, 1)
         const int it = item_ring[rs];
         mbar_arrive(&item_empty[rs]);
         if (it >= total) break;
-        const DualItem d = dual_decode(it, NT, p, pref);
+        const DualItem d = dual_decode(it, NT, NT2, p, pref);
+        const bool ex = d.group == p.G;
+        const int KB = (ex ? p.x_K : p.K) / BK;
         const int slot0 = nxt, slot1 = nxt ^ 1;
         if (d.ntiles == 1) nxt ^= 1;
-        const int rows0 = group_count(p, d.group) - (d.tile0 - d.mt0) * 128;
+        const int rows0 = (ex ? p.x_rows : group_count(p, d.group)) - (d.tile0 - d.mt0) * 128;
         const uint32_t idesc0 = rows0 <= 64 ? IDESC_HALF : IDESC;
         const uint32_t idesc1 = rows0 - 128 <= 64 ? IDESC_HALF : IDESC;
         if (!mbar_wait_bounded(&tempty_bar[slot0], ((uses >> slot0) & 1u) ^ 1u, &abort_flag)) { ok = false; break; }
@@ -289,7 +329,8 @@ __global__ void __launch_bounds__(kDualThreads, 1)
     const int q = warp & 3;
     int nxt = 0;
     uint32_t uses = 0u;  // bit a: phase of slot a's accumulator
-    const bool v8 = ((reinterpret_cast<uintptr_t>(p.out) | (static_cast<uintptr_t>(p.ldo) * (SWIGLU ? 2 : 4))) & 31) == 0;
+    const bool v8_main = ((reinterpret_cast<uintptr_t>(p.out) | (static_cast<uintptr_t>(p.ldo) * (SWIGLU ? 2 : 4))) & 31) == 0;
+    const bool v8_x = ((reinterpret_cast<uintptr_t>(p.x_out) | (static_cast<uintptr_t>(p.x_ldo) * (SWIGLU ? 2 : 4))) & 31) == 0;
     bool ok = true;
     for (int i = 0; ok; ++i) {
       const int rs = i % R;
@@ -300,25 +341,30 @@ __global__ void __launch_bounds__(kDualThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&item_empty[rs]);
       if (it >= total) break;
-      const DualItem d = dual_decode(it, NT, p, pref);
+      const DualItem d = dual_decode(it, NT, NT2, p, pref);
+      const bool ex = d.group == p.G;
       const int slot0 = nxt, slot1 = nxt ^ 1;
       if (d.ntiles == 1) nxt ^= 1;
-      const int count = group_count(p, d.group);
+      const int count = ex ? p.x_rows : group_count(p, d.group);
       const int col0 = d.n_tile * OUT_COLS;
+      const int n_cols = ex ? p.x_N : p.N;
+      void* const out_base = ex ? p.x_out : p.out;
+      const int64_t ldo = ex ? p.x_ldo : p.ldo;
+      const bool v8 = ex ? v8_x : v8_main;
       for (int u = 0; u < d.ntiles && ok; ++u) {
         const int slot = u == 0 ? slot0 : slot1;
         ok = __all_sync(0xffffffffu, mbar_wait_bounded(&tfull_bar[slot], (uses >> slot) & 1u, &abort_flag));
         if (!ok) break;
         tc_fence_after();
         const int local0 = (d.tile0 + u - d.mt0) * 128;
-        const int row0 = p.masked_cap > 0 ? d.group * p.masked_cap + local0 : (d.tile0 + u) * 128;
+        const int row0 = (p.masked_cap > 0 && !ex) ? d.group * p.masked_cap + local0 : (d.tile0 + u) * 128;
         const bool half = count - local0 <= 64;
         const int trow = half ? q * 16 + lane : q * 32 + lane;
         const bool row_ok = (!half || lane < 16) && local0 + trow < count;
         const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + slot * 256;
         const long long orow = static_cast<long long>(row0) + trow;
         if constexpr (SWIGLU) {
-          __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out) + orow * p.ldo + col0;
+          __nv_bfloat16* out = static_cast<__nv_bfloat16*>(out_base) + orow * ldo + col0;
 #pragma unroll 1
           for (int c = 0; c < 128; c += 32) {
             uint32_t rg[32], ru[32];
@@ -331,7 +377,7 @@ __global__ void __launch_bounds__(kDualThreads, 1)
             for (int e = 0; e < 16; ++e)
               packed[e] = pack_bf16x2(silu_mul(__uint_as_float(rg[2 * e]), __uint_as_float(ru[2 * e])),
                                       silu_mul(__uint_as_float(rg[2 * e + 1]), __uint_as_float(ru[2 * e + 1])));
-            if (row_ok && col0 + c < p.N) {
+            if (row_ok && col0 + c < n_cols) {
               if (v8) {
                 st_global_v8(out + c, packed);
                 st_global_v8(out + c + 16, packed + 8);
@@ -344,14 +390,14 @@ __global__ void __launch_bounds__(kDualThreads, 1)
             }
           }
         } else if (p.out_f16) {
-          __half* out = static_cast<__half*>(p.out) + orow * p.ldo + col0;
+          __half* out = static_cast<__half*>(out_base) + orow * ldo + col0;
           bool range_ok = true;
 #pragma unroll 1
           for (int c = 0; c < 256; c += 32) {
             uint32_t r[32];
             tmem_ld_32x32b_x32(tbase + c, r);
             tmem_ld_wait(r);
-            if (row_ok && col0 + c < p.N) {
+            if (row_ok && col0 + c < n_cols) {
               uint32_t packed[16];
 #pragma unroll
               for (int e = 0; e < 16; ++e) {
@@ -366,20 +412,20 @@ __global__ void __launch_bounds__(kDualThreads, 1)
           }
           if (!range_ok) set_status(p.status, MOE_DEV_RANGE);
         } else {
-          float* out = static_cast<float*>(p.out) + orow * p.ldo + col0;
+          float* out = static_cast<float*>(out_base) + orow * ldo + col0;
 #pragma unroll 1
           for (int c = 0; c < 256; c += 32) {
             uint32_t r[32];
             tmem_ld_32x32b_x32(tbase + c, r);
             tmem_ld_wait(r);
-            if (row_ok && col0 + c < p.N) {
-              if (v8 && col0 + c + 32 <= p.N) {
+            if (row_ok && col0 + c < n_cols) {
+              if (v8 && col0 + c + 32 <= n_cols) {
 #pragma unroll
                 for (int v = 0; v < 4; ++v) st_global_v8(out + c + 8 * v, r + 8 * v);
               } else {
 #pragma unroll
                 for (int e = 0; e < 32; ++e)
-                  if (col0 + c + e < p.N) out[c + e] = __uint_as_float(r[e]);
+                  if (col0 + c + e < n_cols) out[c + e] = __uint_as_float(r[e]);
               }
             }
           }
