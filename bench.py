@@ -121,6 +121,9 @@ def _peaks():
 
 
 REFERENCE_BUDGET_S = 90.0   # oracle seconds for a whole --impl reference run
+# nominal dense peaks of one B200, for the spec-relative fractions beside the measured ones
+NOMINAL_BF16_TFLOPS = 2250.0
+NOMINAL_HBM_GBS = 8000.0    # the "~8 TB/s" the decode target is stated against
 FP8_OVER_BF16 = 2.0   # nominal dense e4m3 / bf16 tensor throughput (4.5 / 2.25 PFLOP/s)
 
 
@@ -146,8 +149,9 @@ def roofline_record(flops, nbytes, launch_ms, clk, fp8, peaks):
     launch times (ms): tensor-bound when flops/bytes reaches the ridge of the peaks,
     else HBM-bound.  `frac` is taken against the measured burst tensor peak (these
     kernels run for milliseconds inside steps of milliseconds); frac_of_sustained is
-    the same figure against the seconds-long power-capped loop.  e4m3 takes twice the
-    bf16 figure (the nominal dense ratio).  peaks = (bf16 burst TFLOP/s, bf16 sustained
+    the same figure against the seconds-long power-capped loop, frac_of_nominal against
+    the nominal dense peak (2.25 PFLOP/s bf16, ~8 TB/s HBM).  e4m3 takes twice the bf16
+    figure (the nominal dense ratio).  peaks = (bf16 burst TFLOP/s, bf16 sustained
     TFLOP/s, HBM GB/s, kind)."""
     burst, sustained, hbm_peak, peak_kind = peaks
     ratio = FP8_OVER_BF16 if fp8 else 1.0
@@ -163,7 +167,10 @@ def roofline_record(flops, nbytes, launch_ms, clk, fp8, peaks):
         achieved = nbytes / (avg / 1e3) / 1e9 if avg else None
         rec = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                "peak_kind": f"{peak_kind} HBM copy"}
-    rec.update({"frac": achieved / rec["peak"] if achieved else None, "launches_timed": len(launch_ms),
+    nominal = NOMINAL_BF16_TFLOPS * ratio if rec["bound"] == "tensor" else NOMINAL_HBM_GBS
+    rec.update({"frac": achieved / rec["peak"] if achieved else None,
+                "frac_of_nominal": achieved / nominal if achieved else None, "nominal_peak": nominal,
+                "launches_timed": len(launch_ms),
                 "avg_ms": avg, "algorithmic_flops_per_launch": flops, "algorithmic_bytes_per_launch": nbytes,
                 "tflops": flops / (avg / 1e3) / 1e12 if avg else None,
                 "gbs": nbytes / (avg / 1e3) / 1e9 if avg else None,

@@ -13,6 +13,8 @@ def test_tensor_bound_kernel_at_burst_clocks():
     assert abs(r["achieved"] - 1600.0) < 1e-9 and abs(r["frac"] - 1.0) < 1e-12
     assert abs(r["frac_of_sustained"] - 1600.0 / 1400.0) < 1e-12
     assert r["launches_timed"] == 2 and r["avg_ms"] == 1.25
+    # beside the measured peak, the nominal dense one (2.25 PFLOP/s bf16)
+    assert r["nominal_peak"] == 2250.0 and abs(r["frac_of_nominal"] - 1600.0 / 2250.0) < 1e-12
 
 
 def test_power_capped_run_keeps_the_burst_peak_and_is_flagged():
@@ -33,6 +35,7 @@ def test_power_capped_run_keeps_the_burst_peak_and_is_flagged():
 def test_e4m3_kernel_takes_twice_the_bf16_peak():
     r = bench.roofline_record(4.0e12, 2.5e9, [1.25], None, True, PEAKS)
     assert r["peak"] == 3200.0 and "x2" in r["peak_kind"]
+    assert r["nominal_peak"] == 4500.0 and abs(r["frac_of_nominal"] - 3200.0 / 4500.0) < 1e-12
 
 
 def test_decode_kernel_is_hbm_bound():
@@ -41,11 +44,13 @@ def test_decode_kernel_is_hbm_bound():
     assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["peak"] == 6400.0
     assert abs(r["achieved"] - 7.7e9 / 1.2e-3 / 1e9) < 1e-6
     assert abs(r["frac"] - r["achieved"] / 6400.0) < 1e-12
+    assert r["nominal_peak"] == 8000.0 and abs(r["frac_of_nominal"] - r["achieved"] / 8000.0) < 1e-12
 
 
 def test_no_launches_gives_no_fraction():
     r = bench.roofline_record(6.0e10, 7.7e9, [], None, False, PEAKS)
     assert r["achieved"] is None and r["frac"] is None and r["launches_timed"] == 0
+    assert r["frac_of_nominal"] is None
 
 
 def test_gate_up_kernel_sources_follow_the_library_rule():
