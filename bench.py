@@ -448,6 +448,20 @@ def _cpu_sample_tokens(wl):
 CPU_MIN_SECONDS = 2.0   # a sample shorter than this is repeated (same tokens) until it is not
 
 
+def host_cpu():
+    """(CPU model name, logical CPUs) of the host, from /proc/cpuinfo and os.cpu_count()."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo", encoding="utf-8", errors="replace") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return model, os.cpu_count()
+
+
 def cpu_baseline_record(wl, d):
     host_w = HostWeights(wl, d)
     n, dt, threads = _oracle_sample(wl, d, _cpu_sample_tokens(wl), host_w=host_w)
@@ -457,7 +471,9 @@ def cpu_baseline_record(wl, d):
         dt += t
         reps += 1
     what = f"{n} seeded tokens" + (f", {reps} times" if reps > 1 else "")
+    model, ncpu = host_cpu()
     return {"value": n * reps / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "cpu_model": model, "host_logical_cpus": ncpu,
             "sample": f"{what}, of {wl.name} through the fp64 oracle (route, experts, combine; the time "
                       f"to load expert weights as fp64 is not counted); {dt:.2f} s"}
 
@@ -741,6 +757,7 @@ def run_reference(args):
         "config": {"workload": f"{wl.name}: {_describe(wl)}", "global_batch": wl.T, "seq_len": 1,
                    "parallelism": "host cores"},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "cpu_model": host_cpu()[0], "host_logical_cpus": host_cpu()[1],
                          "sample": f"the same {n} seeded tokens every step through the fp64 oracle "
                                    f"(route, experts, combine; the time to load expert weights as "
                                    f"fp64 is not counted)"},

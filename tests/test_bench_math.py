@@ -170,3 +170,8 @@ def test_default_line_carries_every_workload_and_the_micro_record(monkeypatch, c
     assert line["micro"]["grouped_topk"]["unit"] == "us/call"
     assert calls[0] == ("dsv3_prefill", True, False)
     assert all(adapt for _, _, adapt in calls[1:])
+
+
+def test_host_cpu_reports_a_model_and_a_count():
+    model, n = bench.host_cpu()
+    assert isinstance(model, str) and model and isinstance(n, int) and n >= 1
