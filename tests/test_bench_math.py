@@ -175,3 +175,20 @@ def test_default_line_carries_every_workload_and_the_micro_record(monkeypatch, c
 def test_host_cpu_reports_a_model_and_a_count():
     model, n = bench.host_cpu()
     assert isinstance(model, str) and model and isinstance(n, int) and n >= 1
+
+
+def test_reference_arm_runs_the_oracle_on_the_host(monkeypatch, capsys):
+    """bench.py --impl reference on the tiny workload: the fp64 oracle alone, one JSON line
+    with impl, the CPU baseline (model, cores) and an end-to-end figure equal to the value."""
+    import argparse
+    import json
+    for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    monkeypatch.setattr(bench, "REFERENCE_BUDGET_S", 2.0)
+    bench.run_reference(argparse.Namespace(workload="tiny", steps=3, warmup=3))
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["dtype"] == "f64" and line["steps"] == 3
+    assert line["value"] > 0 and line["e2e"]["value"] == line["value"]
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["cpu_baseline"]["cpu_model"]
+    assert line["config"]["workload"].startswith("tiny")
