@@ -329,7 +329,11 @@ moe_status_t moe_selftest_bounded_wait(void* ws, int32_t limit_ms, void* stream)
 const char* moe_status_string(moe_status_t s);
 int32_t moe_abi_version(void);
 
-/* Kernel ids for tracing. */
+/* Kernel ids for tracing.  MOE_K_PERM_GATHER also covers the layer's token-order copy and
+ * MOE_K_SCALE_ATOMS the e4m3 weights' scale atoms.  Where moe_layer_forward runs the
+ * shared expert as one more group of the routed two-M-tile launches (bf16, more than 16384
+ * pairs, T*K >= 256*E), its work is inside MOE_K_GATEUP / MOE_K_DOWN and the two
+ * MOE_K_SHARED_* ids do not occur. */
 enum {
   MOE_K_ROUTER_GEMM = 0, MOE_K_TOPK = 1, MOE_K_PERM_COUNT = 2, MOE_K_PERM_SCAN = 3,
   MOE_K_PERM_RANK = 4, MOE_K_PERM_GATHER = 5, MOE_K_GATEUP = 6, MOE_K_DOWN = 7,
