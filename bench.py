@@ -462,6 +462,12 @@ def host_cpu():
     return model, os.cpu_count()
 
 
+def oracle_flops_per_token(wl) -> float:
+    """Multiply-add work of one token through the layer as the oracle computes it: router
+    logits, K routed SwiGLU FFNs, the shared expert (2 FLOP per multiply-add)."""
+    return 2.0 * wl.H * wl.E + wl.K * 6.0 * wl.H * wl.I + 6.0 * wl.H * wl.I_shared
+
+
 def cpu_baseline_record(wl, d):
     host_w = HostWeights(wl, d)
     n, dt, threads = _oracle_sample(wl, d, _cpu_sample_tokens(wl), host_w=host_w)
@@ -473,6 +479,7 @@ def cpu_baseline_record(wl, d):
     what = f"{n} seeded tokens" + (f", {reps} times" if reps > 1 else "")
     model, ncpu = host_cpu()
     return {"value": n * reps / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "gflops": n * reps / dt * oracle_flops_per_token(wl) / 1e9,
             "cpu_model": model, "host_logical_cpus": ncpu,
             "sample": f"{what}, of {wl.name} through the fp64 oracle (route, experts, combine; the time "
                       f"to load expert weights as fp64 is not counted); {dt:.2f} s"}
@@ -757,6 +764,7 @@ def run_reference(args):
         "config": {"workload": f"{wl.name}: {_describe(wl)}", "global_batch": wl.T, "seq_len": 1,
                    "parallelism": "host cores"},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "gflops": value * oracle_flops_per_token(wl) / 1e9,
                          "cpu_model": host_cpu()[0], "host_logical_cpus": host_cpu()[1],
                          "sample": f"the same {n} seeded tokens every step through the fp64 oracle "
                                    f"(route, experts, combine; the time to load expert weights as "

@@ -192,3 +192,16 @@ def test_reference_arm_runs_the_oracle_on_the_host(monkeypatch, capsys):
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["cpu_baseline"]["cpu_model"]
     assert line["config"]["workload"].startswith("tiny")
+    per_token = 2 * 256 * 8 + 2 * 6 * 256 * 128   # router + K=2 routed SwiGLU FFNs of the tiny layer
+    assert abs(line["cpu_baseline"]["gflops"] - line["value"] * per_token / 1e9) < 1e-9 * line["value"]
+
+
+def test_cpu_baseline_record_on_host_inputs():
+    """The oracle's CPU baseline of the tiny layer from host-resident inputs: tokens/s, the
+    GFLOP/s they imply, the cores used and the host CPU."""
+    from mixture_experts_ffn_08_b200 import inputs, workloads as W
+    d = inputs.make_inputs(W.TINY, seed=0, device="cpu")
+    r = bench.cpu_baseline_record(W.TINY, d)
+    assert r["kind"] == "oracle" and r["value"] > 0 and r["cores"] >= 1 and r["cpu_model"]
+    assert abs(r["gflops"] - r["value"] * bench.oracle_flops_per_token(W.TINY) / 1e9) < 1e-9 * r["value"]
+    assert bench.oracle_flops_per_token(W.DSV3_PREFILL) == 2 * 7168 * 256 + 8 * 6 * 7168 * 2048 + 6 * 7168 * 2048
