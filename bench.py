@@ -649,6 +649,7 @@ def measure(wl, steps, warmup, world=1, rank=0, local=0, cpu=True, adapt_steps=F
     return {
         "workload": f"{wl.name}: {_describe(wl)}",
         "value": tokens_per_s, "unit": "tokens/s", "ms_per_step": ms_step, "steps": steps,
+        "ms_per_step_median_rank0": statistics.median(step_ms),
         "dtype": "fp8xfp4" if w4 else ("fp8" if fp8 else "bf16"),
         "grouped_gemm_tflops": gemm_flops / (ms_step / 1e3) / 1e12 * world,
         "gemm_kernel_tflops": {k: f / (kernel_ms[k] / 1e3) / 1e12 for k, f in flops.items() if kernel_ms.get(k)},
