@@ -164,3 +164,16 @@ def test_fp4_launch_counts(lib):
     for wl in W.FP4.values():
         bf16 = 7 if wl.T * wl.K <= 2048 else 9
         assert B.moe_layer_launch_count(B.params(wl)) == bf16 + 1
+
+
+def test_trace_kernel_ids_match_the_header():
+    """The binding's kernel ids and names follow the header's MOE_K_* enum."""
+    src = open(os.path.join(ROOT, "include", "moe.h"), encoding="utf-8").read()
+    ids = {name: int(v) for name, v in re.findall(r"\bMOE_K_([A-Z0-9_]+)\s*=\s*(\d+)", src)}
+    assert ids["COUNT"] == len(B.KERNEL_NAMES)
+    assert (B.K_GATEUP, B.K_DOWN, B.K_SHARED_GATEUP, B.K_SHARED_DOWN, B.K_COMBINE, B.K_DEQUANT_X) == (
+        ids["GATEUP"], ids["DOWN"], ids["SHARED_GATEUP"], ids["SHARED_DOWN"], ids["COMBINE"], ids["DEQUANT_X"])
+    for name, i in ids.items():
+        if name != "COUNT":
+            # the names are the header's in lower case; the routed gate/up carries its SwiGLU
+            assert B.KERNEL_NAMES[i] == ("gateup_swiglu" if name == "GATEUP" else name.lower()), (name, i)
