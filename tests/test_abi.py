@@ -177,3 +177,11 @@ def test_trace_kernel_ids_match_the_header():
         if name != "COUNT":
             # the names are the header's in lower case; the routed gate/up carries its SwiGLU
             assert B.KERNEL_NAMES[i] == ("gateup_swiglu" if name == "GATEUP" else name.lower()), (name, i)
+
+
+def test_device_status_bits_match_the_header():
+    src = open(os.path.join(ROOT, "include", "moe.h"), encoding="utf-8").read()
+    bits = {name: int(v, 16) for name, v in re.findall(r"#define (MOE_DEV_[A-Z_]+) (0x[0-9a-fA-F]+)", src)}
+    assert bits == {"MOE_DEV_BAD_EXPERT_ID": B.MOE_DEV_BAD_EXPERT_ID, "MOE_DEV_TIMEOUT": B.MOE_DEV_TIMEOUT,
+                    "MOE_DEV_CAPACITY": B.MOE_DEV_CAPACITY, "MOE_DEV_RANGE": B.MOE_DEV_RANGE}
+    assert len(set(bits.values())) == len(bits) and all(v & (v - 1) == 0 for v in bits.values())
